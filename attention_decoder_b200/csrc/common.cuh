@@ -1,0 +1,77 @@
+// Device helpers shared by the LFM3 kernels (sm_100a only).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#define DEVI __device__ __forceinline__
+
+typedef __nv_bfloat16 bf16;
+
+// ---------------------------------------------------------------- numeric conversions
+DEVI float bf2f(bf16 x) { return __bfloat162float(x); }
+DEVI bf16 f2bf(float x) { return __float2bfloat16_rn(x); }
+DEVI float bflo(uint32_t w) { return __uint_as_float(w << 16); }
+DEVI float bfhi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+DEVI uint32_t pack_bf2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+DEVI float round_bf(float x) { return bf2f(f2bf(x)); }
+
+// ---------------------------------------------------------------- reductions
+DEVI float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+DEVI float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+// Sum over a block of NW warps; `red` holds NW floats. Every thread gets the total.
+template <int NW>
+DEVI float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) t += red[i];
+  return t;
+}
+
+// ---------------------------------------------------------------- memory
+// Streaming 16-byte load that skips L1 (weights are read once per step).
+DEVI uint4 ldg_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+DEVI uint4 ldg16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+DEVI void stg16(void* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels are launched with programmatic stream serialisation: each one may start while its
+// predecessor drains. pdl_wait() blocks until the predecessor grid has completed and its writes
+// are visible; every block calls it before touching data a previous kernel produced (and before
+// exiting), so completion stays transitive along the stream.
+DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+DEVI void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// ---------------------------------------------------------------- tensor-core fragment (legacy warp MMA)
+// D[16x8] += A[16x16] (row) * B[16x8] (col), bf16 inputs, fp32 accumulate.
+DEVI void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+DEVI float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
+DEVI float siluf_(float x) { return x / (1.f + __expf(-x)); }

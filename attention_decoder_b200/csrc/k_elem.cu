@@ -1,0 +1,353 @@
+// Small memory-bound kernels of the LFM3 forward: row bookkeeping, embedding, the fused
+// sandwich-norm/residual step, the gated short conv with its state, q/k RMSNorm + rotary +
+// KV placement, and the sliding-ring copies.
+#include "kernels.cuh"
+
+namespace lfm3 {
+
+thread_local int g_launches = 0;
+
+// ------------------------------------------------------------------------------------------
+// Row bookkeeping: prefill rows are consecutive positions of one slot; decode rows are one
+// position of each listed slot. Also clears the per-row greedy cells.
+__global__ void k_setup_rows(int prefill, int slot, const int32_t* __restrict__ d_slots,
+                             const int32_t* __restrict__ seq_len, int rows, int32_t* row_slot, int32_t* row_pos,
+                             unsigned long long* amax) {
+  pdl_wait();
+  pdl_launch_dependents();
+  int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  if (prefill) {
+    row_slot[r] = slot;
+    row_pos[r] = seq_len[slot] + r;
+  } else {
+    int s = d_slots[r];
+    row_slot[r] = s;
+    row_pos[r] = seq_len[s];
+  }
+  if (amax) amax[r] = 0ull;
+}
+
+cudaError_t setup_rows(int prefill, int slot, const int32_t* d_slots, const int32_t* seq_len, int rows,
+                       int32_t* row_slot, int32_t* row_pos, unsigned long long* amax, cudaStream_t s) {
+  return launch(k_setup_rows, dim3((rows + 127) / 128), dim3(128), 0, s, prefill, slot, d_slots, seq_len, rows,
+                row_slot, row_pos, amax);
+}
+
+// ------------------------------------------------------------------------------------------
+// Embedding (tied table) or input vectors -> fp32 residual stream.
+__global__ void __launch_bounds__(256) k_embed(const int32_t* __restrict__ tokens, const bf16* __restrict__ table,
+                                               const bf16* __restrict__ vecs, float* __restrict__ x_res,
+                                               float* __restrict__ dump) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = blockIdx.x;
+  const bf16* src = tokens ? table + (size_t)tokens[r] * D : vecs + (size_t)r * D;
+  const int i = threadIdx.x * 8;
+  uint4 w = ldg16(src + i);
+  float4 a = make_float4(bflo(w.x), bfhi(w.x), bflo(w.y), bfhi(w.y));
+  float4 b = make_float4(bflo(w.z), bfhi(w.z), bflo(w.w), bfhi(w.w));
+  float4* dst = reinterpret_cast<float4*>(x_res + (size_t)r * D + i);
+  dst[0] = a;
+  dst[1] = b;
+  if (dump) {
+    float4* dd = reinterpret_cast<float4*>(dump + (size_t)r * D + i);
+    dd[0] = a;
+    dd[1] = b;
+  }
+}
+
+cudaError_t embed_rows(const int32_t* tokens, const bf16* table, const bf16* vecs, int rows, float* x_res,
+                       float* dump, cudaStream_t s) {
+  return launch(k_embed, dim3(rows), dim3(256), 0, s, tokens, table, vecs, x_res, dump);
+}
+
+// ------------------------------------------------------------------------------------------
+// Sandwich-norm step on one row (d_model = 2048, 256 threads x 8):
+//   if n_part > 0:  m = sum_s part[s][r];  x += g_post * m * rsqrt(mean(m^2) + eps)
+//   dump[r] = x (optional);  xn = bf16(g_next * x * rsqrt(mean(x^2) + eps)) (optional)
+__global__ void __launch_bounds__(256) k_resid_norm(float* __restrict__ x_res, const float* __restrict__ part,
+                                                    int n_part, long part_stride, const bf16* __restrict__ g_post,
+                                                    const bf16* __restrict__ g_next, bf16* __restrict__ xn, float eps,
+                                                    float* __restrict__ dump) {
+  __shared__ float red[8];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = blockIdx.x;
+  const int i = threadIdx.x * 8;
+  float* xr = x_res + (size_t)r * D + i;
+  float x[8];
+  {
+    float4 a = reinterpret_cast<float4*>(xr)[0], b = reinterpret_cast<float4*>(xr)[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+  if (n_part > 0) {
+    float m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int s = 0; s < n_part; ++s) {
+      const float* p = part + s * part_stride + (size_t)r * D + i;
+      float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+      m[0] += a.x; m[1] += a.y; m[2] += a.z; m[3] += a.w; m[4] += b.x; m[5] += b.y; m[6] += b.z; m[7] += b.w;
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss += m[j] * m[j];
+    ss = block_sum<8>(ss, red);
+    const float inv = rsqrtf(ss * (1.0f / D) + eps);
+    uint4 gw = ldg16(g_post + i);
+    float g[8] = {bflo(gw.x), bfhi(gw.x), bflo(gw.y), bfhi(gw.y), bflo(gw.z), bfhi(gw.z), bflo(gw.w), bfhi(gw.w)};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] += g[j] * (m[j] * inv);
+    reinterpret_cast<float4*>(xr)[0] = make_float4(x[0], x[1], x[2], x[3]);
+    reinterpret_cast<float4*>(xr)[1] = make_float4(x[4], x[5], x[6], x[7]);
+  }
+  if (dump) {
+    float4* dd = reinterpret_cast<float4*>(dump + (size_t)r * D + i);
+    dd[0] = make_float4(x[0], x[1], x[2], x[3]);
+    dd[1] = make_float4(x[4], x[5], x[6], x[7]);
+  }
+  if (g_next) {
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss += x[j] * x[j];
+    ss = block_sum<8>(ss, red);
+    const float inv = rsqrtf(ss * (1.0f / D) + eps);
+    uint4 gw = ldg16(g_next + i);
+    float g[8] = {bflo(gw.x), bfhi(gw.x), bflo(gw.y), bfhi(gw.y), bflo(gw.z), bfhi(gw.z), bflo(gw.w), bfhi(gw.w)};
+    uint4 o;
+    o.x = pack_bf2(g[0] * (x[0] * inv), g[1] * (x[1] * inv));
+    o.y = pack_bf2(g[2] * (x[2] * inv), g[3] * (x[3] * inv));
+    o.z = pack_bf2(g[4] * (x[4] * inv), g[5] * (x[5] * inv));
+    o.w = pack_bf2(g[6] * (x[6] * inv), g[7] * (x[7] * inv));
+    stg16(xn + (size_t)r * D + i, o);
+  }
+}
+
+cudaError_t resid_norm(float* x_res, const float* part, int n_part, long part_stride, const bf16* g_post,
+                       const bf16* g_next, bf16* xn, int rows, float eps, float* dump, cudaStream_t s) {
+  return launch(k_resid_norm, dim3(rows), dim3(256), 0, s, x_res, part, n_part, part_stride, g_post, g_next, xn,
+                eps, dump);
+}
+
+// ------------------------------------------------------------------------------------------
+// Gated short conv (coreai-model-zoo "lfm3-1.7b-port", diff table row 1): with [B|C|x] the
+// in_proj output (fp32 accumulators), bx = bf16(B * x); over win = [state(6) | bx], z_t = sum_k w[c][k] win[t+k]
+// (tap 6 on the newest column); y = bf16(C * z); the new state is win[n : n + 6].
+// Decode: one row per stream, state [slot][6][D] shifts by one column.
+__global__ void __launch_bounds__(256) k_conv_decode(const float* __restrict__ bcx, const bf16* __restrict__ conv_w,
+                                                     bf16* __restrict__ state, const int32_t* __restrict__ row_slot,
+                                                     bf16* __restrict__ y) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int b = blockIdx.y;
+  const int c = blockIdx.x * 256 + threadIdx.x;
+  const float* row = bcx + (size_t)b * 3 * D;
+  const float Bv = row[c], Cv = row[D + c], Xv = row[2 * D + c];
+  const float bx = round_bf(Bv * Xv);
+  bf16* st = state + (size_t)row_slot[b] * CST * D + c;
+  float win[CST];
+#pragma unroll
+  for (int j = 0; j < CST; ++j) win[j] = bf2f(st[(size_t)j * D]);
+  const bf16* w = conv_w + (size_t)c * TAPS;
+  float z = 0.f;
+#pragma unroll
+  for (int k = 0; k < CST; ++k) z += bf2f(w[k]) * win[k];
+  z += bf2f(w[CST]) * bx;
+  y[(size_t)b * D + c] = f2bf(Cv * z);
+#pragma unroll
+  for (int j = 0; j < CST - 1; ++j) st[(size_t)j * D] = f2bf(win[j + 1]);
+  st[(size_t)(CST - 1) * D] = f2bf(bx);
+}
+
+cudaError_t conv_decode(const float* bcx, const bf16* conv_w, bf16* state_layer, const int32_t* row_slot, int rows,
+                        bf16* y, cudaStream_t s) {
+  return launch(k_conv_decode, dim3(D / 256, rows), dim3(256), 0, s, bcx, conv_w, state_layer, row_slot, y);
+}
+
+// Prefill: n consecutive rows of one slot. Block (channel group, row group of 32). Only the
+// first row group reads the carried state (rows < 6), and it also writes the new state, so
+// the read precedes the write within one thread.
+constexpr int CONV_RG = 32;
+__global__ void __launch_bounds__(128) k_conv_prefill(const float* __restrict__ bcx, const bf16* __restrict__ conv_w,
+                                                      bf16* __restrict__ state, int n, bf16* __restrict__ y) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int c = blockIdx.x * 128 + threadIdx.x;
+  const int r0 = blockIdx.y * CONV_RG;
+  const int r1 = min(n, r0 + CONV_RG);
+  float w[TAPS];
+#pragma unroll
+  for (int k = 0; k < TAPS; ++k) w[k] = bf2f(conv_w[(size_t)c * TAPS + k]);
+  auto bx_at = [&](int t) -> float {  // bx of row t of this chunk (stored state precision: bf16)
+    const float* row = bcx + (size_t)t * 3 * D;
+    return round_bf(row[c] * row[2 * D + c]);
+  };
+  auto win_at = [&](int i) -> float {  // win[i] = state[i] for i < 6, bx[i - 6] after
+    return i < CST ? bf2f(state[(size_t)i * D + c]) : bx_at(i - CST);
+  };
+  float win[TAPS];
+#pragma unroll
+  for (int k = 0; k < CST; ++k) win[k] = win_at(r0 + k);
+  for (int t = r0; t < r1; ++t) {
+    win[CST] = bx_at(t);
+    float z = 0.f;
+#pragma unroll
+    for (int k = 0; k < TAPS; ++k) z += w[k] * win[k];
+    y[(size_t)t * D + c] = f2bf(bcx[(size_t)t * 3 * D + D + c] * z);
+#pragma unroll
+    for (int k = 0; k < CST; ++k) win[k] = win[k + 1];
+  }
+  if (blockIdx.y == 0) {
+    float ns[CST];
+#pragma unroll
+    for (int j = 0; j < CST; ++j) ns[j] = win_at(n + j);
+#pragma unroll
+    for (int j = 0; j < CST; ++j) state[(size_t)j * D + c] = f2bf(ns[j]);
+  }
+}
+
+cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot, int n, bf16* y, cudaStream_t s) {
+  return launch(k_conv_prefill, dim3(D / 128, (n + CONV_RG - 1) / CONV_RG), dim3(128), 0, s, bcx, conv_w,
+                state_slot, n, y);
+}
+
+// ------------------------------------------------------------------------------------------
+// Per-head q/k RMSNorm (gain of length 128 shared across heads), rotary on pairs (i, i+64) with
+// a per-position table (zero-tail pairs carry cos 1, sin 0), and placement of k/v.
+// Block = (row, head among q | k | v), 128 threads = head_dim.
+__global__ void __launch_bounds__(128) k_qk_norm_rope_kv(const float* __restrict__ part, int n_part,
+                                                         long part_stride, const bf16* __restrict__ q_norm,
+                                                         const bf16* __restrict__ k_norm,
+                                                         const float* __restrict__ rope_cos,
+                                                         const float* __restrict__ rope_sin, Rows rows, float eps,
+                                                         bf16* __restrict__ q_out, float* __restrict__ gate_out,
+                                                         KvWrite kv) {
+  __shared__ float red[4];
+  __shared__ float xs[HD];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = blockIdx.x, hh = blockIdx.y, i = threadIdx.x;
+  const int col0 = hh * HD;  // q heads, then k heads, then v heads are consecutive in qkvg
+  float x = 0.f;
+  for (int s = 0; s < n_part; ++s) x += part[s * part_stride + (size_t)r * NQKVG + col0 + i];
+  const int pos = rows.pos[r];
+  if (hh < HQ + HKV) {
+    const bf16* g = hh < HQ ? q_norm : k_norm;
+    float ss = block_sum<4>(x * x, red);
+    x = bf2f(g[i]) * (x * rsqrtf(ss * (1.0f / HD) + eps));
+    xs[i] = x;
+    __syncthreads();
+    const int j = i & (HD / 2 - 1);
+    const float c = rope_cos[(size_t)pos * (HD / 2) + j], sn = rope_sin[(size_t)pos * (HD / 2) + j];
+    x = i < HD / 2 ? x * c - xs[i + HD / 2] * sn : x * c + xs[i - HD / 2] * sn;
+  }
+  if (hh < HQ) {
+    q_out[((size_t)r * HQ + hh) * HD + i] = f2bf(x);
+    if (i == 0) {
+      float gsum = 0.f;
+      for (int s = 0; s < n_part; ++s) gsum += part[s * part_stride + (size_t)r * NQKVG + HQ * HD + 2 * HKV * HD + hh];
+      gate_out[r * HQ + hh] = gsum;
+    }
+    return;
+  }
+  const bool isk = hh < HQ + HKV;
+  const int kvh = isk ? hh - HQ : hh - HQ - HKV;
+  bf16* base = isk ? kv.k : kv.v;
+  size_t off;
+  if (kv.mode == KV_PAGES) {
+    const int slot = rows.slot[r];
+    const int page = kv.page_table[(size_t)slot * kv.max_pages + pos / PAGE];
+    off = (((size_t)page * HKV + kvh) * PAGE + pos % PAGE) * HD;
+  } else if (kv.mode == KV_RING) {
+    const int slot = rows.slot[r];
+    off = (((size_t)slot * HKV + kvh) * WIN + pos % WIN) * HD;
+  } else {
+    off = ((size_t)kvh * kv.scratch_rows + WIN + r) * HD;
+  }
+  base[off + i] = f2bf(x);
+}
+
+cudaError_t qk_norm_rope_kv(const float* part, int n_part, long part_stride, const bf16* q_norm, const bf16* k_norm,
+                            const float* rope_cos, const float* rope_sin, Rows rows, float eps, bf16* q_out,
+                            float* gate_out, KvWrite kv, cudaStream_t s) {
+  return launch(k_qk_norm_rope_kv, dim3(rows.n, HQ + 2 * HKV), dim3(HD), 0, s, part, n_part, part_stride, q_norm,
+                k_norm, rope_cos, rope_sin, rows, eps, q_out, gate_out, kv);
+}
+
+// ------------------------------------------------------------------------------------------
+// Sliding layers in a prompt pass: the ring's last WIN positions before the chunk are copied
+// into scratch rows [0, WIN) (index i <-> position p0 - WIN + i; rows before position 0 are
+// zero), the chunk's own k/v land in rows WIN + r, and after attention the chunk's last
+// min(n, WIN) positions go back to their ring slots.
+__global__ void __launch_bounds__(128) k_ring_to_scratch(const bf16* __restrict__ rk, const bf16* __restrict__ rv,
+                                                         int slot, int p0, bf16* __restrict__ sk,
+                                                         bf16* __restrict__ sv, int scratch_rows) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int i = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+  const int pos = p0 - WIN + i;
+  bf16 kx = f2bf(0.f), vx = f2bf(0.f);
+  if (pos >= 0) {
+    const size_t o = (((size_t)slot * HKV + h) * WIN + pos % WIN) * HD + d;
+    kx = rk[o];
+    vx = rv[o];
+  }
+  const size_t so = ((size_t)h * scratch_rows + i) * HD + d;
+  sk[so] = kx;
+  sv[so] = vx;
+}
+
+cudaError_t ring_to_scratch(const bf16* ring_k, const bf16* ring_v, int slot, int max_streams, int p0, bf16* sk,
+                            bf16* sv, int scratch_rows, cudaStream_t s) {
+  (void)max_streams;
+  return launch(k_ring_to_scratch, dim3(WIN, HKV), dim3(HD), 0, s, ring_k, ring_v, slot, p0, sk, sv, scratch_rows);
+}
+
+__global__ void __launch_bounds__(128) k_scratch_to_ring(const bf16* __restrict__ sk, const bf16* __restrict__ sv,
+                                                         int scratch_rows, int n, int p0, bf16* __restrict__ rk,
+                                                         bf16* __restrict__ rv, int slot) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int m = min(n, WIN);
+  const int r = n - m + blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+  const int pos = p0 + r;
+  const size_t so = ((size_t)h * scratch_rows + WIN + r) * HD + d;
+  const size_t o = (((size_t)slot * HKV + h) * WIN + pos % WIN) * HD + d;
+  rk[o] = sk[so];
+  rv[o] = sv[so];
+}
+
+cudaError_t scratch_to_ring(const bf16* sk, const bf16* sv, int scratch_rows, int n, int p0, bf16* ring_k,
+                            bf16* ring_v, int slot, int max_streams, cudaStream_t s) {
+  (void)max_streams;
+  return launch(k_scratch_to_ring, dim3(n < WIN ? n : WIN, HKV), dim3(HD), 0, s, sk, sv, scratch_rows, n, p0, ring_k,
+                ring_v, slot);
+}
+
+// ------------------------------------------------------------------------------------------
+// End of a call: advance seq_len and publish greedy ids (the cells hold (ordered value << 32) |
+// (0xffffffff - id), so the max is the largest logit with the lowest id among ties).
+__global__ void k_finish(int32_t* seq_len, const int32_t* __restrict__ row_slot, int rows, int add_prefill,
+                         int prefill_slot, const unsigned long long* __restrict__ amax, int32_t* argmax_out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = threadIdx.x;
+  if (add_prefill) {
+    if (r == 0) {
+      seq_len[prefill_slot] += add_prefill;
+      if (argmax_out && amax) argmax_out[0] = (int32_t)(0xffffffffu - (uint32_t)(amax[0] & 0xffffffffull));
+    }
+    return;
+  }
+  if (r < rows) {
+    seq_len[row_slot[r]] += 1;
+    if (argmax_out && amax) argmax_out[r] = (int32_t)(0xffffffffu - (uint32_t)(amax[r] & 0xffffffffull));
+  }
+}
+
+cudaError_t finish_step(int32_t* seq_len, const int32_t* row_slot, int rows, int add_prefill, int prefill_slot,
+                        const unsigned long long* amax, int32_t* argmax_out, cudaStream_t s) {
+  return launch(k_finish, dim3(1), dim3(64), 0, s, seq_len, row_slot, rows, add_prefill, prefill_slot, amax,
+                argmax_out);
+}
+
+}  // namespace lfm3

@@ -1,0 +1,139 @@
+// Internal launch interface of the LFM3 kernels (host side). Not part of the C ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <utility>
+
+#include "common.cuh"
+
+namespace lfm3 {
+
+// Geometry the kernels implement (the LFM3-1.7B decoder).
+constexpr int D = 2048;        // d_model
+constexpr int F = 7680;        // d_ffn
+constexpr int HQ = 16;         // query heads
+constexpr int HKV = 4;         // kv heads
+constexpr int HD = 128;        // head_dim
+constexpr int TAPS = 7;        // conv taps
+constexpr int CST = TAPS - 1;  // conv state columns
+constexpr int WIN = 256;       // sliding window
+constexpr int PAGE = 64;       // positions per KV page
+constexpr int NQKVG = HQ * HD + 2 * HKV * HD + HQ;  // 3088 fused projection rows
+constexpr int GQA = HQ / HKV;
+
+// Launch counter of the calling thread (reset by the API at each call).
+extern thread_local int g_launches;
+
+// Every kernel is launched with programmatic stream serialisation (see pdl_wait()).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ++g_launches;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Where the rows of a call sit: row r belongs to slot row_slot[r] at position row_pos[r].
+struct Rows {
+  const int32_t* slot;
+  const int32_t* pos;
+  int n;
+};
+
+// ---------------------------------------------------------------- elementwise / small kernels
+cudaError_t setup_rows(int prefill, int slot, const int32_t* d_slots, const int32_t* seq_len, int rows,
+                       int32_t* row_slot, int32_t* row_pos, unsigned long long* amax, cudaStream_t s);
+cudaError_t embed_rows(const int32_t* tokens, const bf16* table, const bf16* vecs, int rows, float* x_res,
+                       float* dump, cudaStream_t s);
+// x_res[r] += g_post * RMS(sum_s part[s][r]) (if n_part > 0); dump x_res; xn = g_next * RMS(x_res)
+cudaError_t resid_norm(float* x_res, const float* part, int n_part, long part_stride, const bf16* g_post,
+                       const bf16* g_next, bf16* xn, int rows, float eps, float* dump, cudaStream_t s);
+cudaError_t conv_decode(const float* bcx, const bf16* conv_w, bf16* state_layer, const int32_t* row_slot,
+                        int rows, bf16* y, cudaStream_t s);
+cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot, int n, bf16* y, cudaStream_t s);
+
+enum KvDst { KV_PAGES = 0, KV_RING = 1, KV_SCRATCH = 2 };
+struct KvWrite {
+  int mode;
+  bf16* k;               // pages: pool base of this layer; ring: ring base of this layer; scratch base
+  bf16* v;
+  const int32_t* page_table;
+  int max_pages;         // page-table width
+  int max_streams;
+  int scratch_rows;      // WIN + max_chunk (scratch mode)
+};
+cudaError_t qk_norm_rope_kv(const float* part, int n_part, long part_stride, const bf16* q_norm,
+                            const bf16* k_norm, const float* rope_cos, const float* rope_sin, Rows rows,
+                            float eps, bf16* q_out, float* gate_out, KvWrite kv, cudaStream_t s);
+cudaError_t ring_to_scratch(const bf16* ring_k, const bf16* ring_v, int slot, int max_streams, int p0,
+                            bf16* sk, bf16* sv, int scratch_rows, cudaStream_t s);
+cudaError_t scratch_to_ring(const bf16* sk, const bf16* sv, int scratch_rows, int n, int p0, bf16* ring_k,
+                            bf16* ring_v, int slot, int max_streams, cudaStream_t s);
+cudaError_t finish_step(int32_t* seq_len, const int32_t* row_slot, int rows, int add_prefill, int prefill_slot,
+                        const unsigned long long* amax, int32_t* argmax_out, cudaStream_t s);
+
+// ---------------------------------------------------------------- decode GEMV (weights streamed once)
+enum GemvEpi { GEMV_PARTIAL = 0, GEMV_SWIGLU = 1, GEMV_CONV = 2, GEMV_HEAD = 3 };
+struct GemvArgs {
+  const bf16* w;   // [N][K]   (SwiGLU: w1; conv: in_proj [3D][D])
+  const bf16* w3;  // SwiGLU: w3 [F][K]
+  const uint8_t* codes;  const uint8_t* scales;   // NVFP4 (w1 for SwiGLU)
+  const uint8_t* codes3; const uint8_t* scales3;  // NVFP4 w3
+  float tscale;    // NVFP4 tensor scale
+  const bf16* x;   // [rows][K] activations
+  int K, N, rows, splits;
+  float* part;     // GEMV_PARTIAL: [splits][rows][N]; GEMV_HEAD: logits [rows][N] (may be null)
+  bf16* out;       // GEMV_SWIGLU: u [rows][N]
+  // conv epilogue
+  const bf16* conv_w; bf16* conv_state; const int32_t* row_slot; int max_streams; bf16* y;
+  // head epilogue
+  unsigned long long* amax;
+};
+cudaError_t gemv(int epi, int nvfp4, const GemvArgs& a, cudaStream_t s);
+cudaError_t gemv_init();  // one-time function attributes (before any capture)
+
+// ---------------------------------------------------------------- attention
+struct AttnLayer {
+  int full;               // 1 full (pages), 0 sliding
+  const bf16* k; const bf16* v;   // pages: this layer's pool; ring: this layer's ring base
+  const int32_t* page_table;
+  int max_pages, max_streams;
+};
+cudaError_t attn_decode(const bf16* q, Rows rows, AttnLayer L, int splits, float* part, const float* gate,
+                        bf16* y, cudaStream_t s);
+// Prefill attention for the n rows of one slot starting at position p0.
+//  full: keys through the page table; sliding: keys in scratch [HKV][scratch_rows][HD], index i <-> p0-WIN+i
+cudaError_t attn_init();
+cudaError_t attn_prefill(const bf16* q, int n, int p0, int slot, AttnLayer L, const bf16* sk, const bf16* sv,
+                         int scratch_rows, const float* gate, bf16* y, cudaStream_t s);
+
+// ---------------------------------------------------------------- tensor-core GEMM (prefill)
+enum GemmEpi { GEMM_F32 = 0, GEMM_BF16 = 1, GEMM_SWIGLU = 2 };
+struct GemmPlan {
+  CUtensorMap a;      // activations [M][K] bf16, box 64 x 128
+  CUtensorMap b;      // weights [N][K] bf16 (SwiGLU: w1)
+  CUtensorMap b3;     // SwiGLU: w3
+  int epi, M, N, K;
+  void* out;          // fp32 or bf16 [M][ld]
+  int ld;
+  float alpha;        // scales the accumulator (NVFP4 tensor scale; 1 otherwise)
+};
+bool tma_init();
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+cudaError_t gemm(const GemmPlan& p, int M, int* err, cudaStream_t s);
+cudaError_t gemm_init();
+// NVFP4 prefill: dequantise a weight to bf16 [N][K] in scratch, then run the bf16 GEMM.
+cudaError_t nvfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, float tscale, int N, int K, bf16* out,
+                          cudaStream_t s);
+
+}  // namespace lfm3

@@ -1,0 +1,791 @@
+// C ABI of the LFM3 decoder forward: host-side validation, workspace layout and the launch
+// sequence of a prompt pass (lfm3_prefill) and of a decode step (lfm3_decode_step).
+// The declarations and conventions are in include/lfm3.h.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "kernels.cuh"
+#include "lfm3.h"
+
+using namespace lfm3;
+
+namespace {
+
+// Decode GEMV K splits (partial sums are added by the consumer).
+constexpr int SPLIT_QKVG = 2, SPLIT_DD = 2, SPLIT_W2 = 6, SPLIT_W2_FP4 = 5, SPLIT_MAX = 8;
+constexpr int GEMV_MAX_ROWS = 16;
+
+struct LayerPlan {
+  GemmPlan in_proj, out_proj, qkvg, o_proj, w13, w2;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+struct lfm3_ctx {
+  lfm3_config cfg;
+  std::vector<lfm3_layer_weights> L;
+  const bf16* embed = nullptr;
+  const bf16* final_norm = nullptr;
+  int n_conv = 0, n_full = 0, n_sliding = 0;
+  std::vector<int> kidx;
+  int max_pos = 0, R = 0, max_splits = 0, scratch_rows = 0;
+  size_t ws_bytes = 0;
+  bool bound = false;
+  // workspace carve
+  int* err = nullptr;
+  int32_t* row_slot = nullptr;
+  int32_t* row_pos = nullptr;
+  unsigned long long* amax = nullptr;
+  float* x_res = nullptr;
+  bf16* xn = nullptr;
+  bf16* big = nullptr;
+  bf16* y = nullptr;
+  float* part = nullptr;
+  bf16* q = nullptr;
+  float* gate = nullptr;
+  bf16* sk = nullptr;
+  bf16* sv = nullptr;
+  float* attn_part = nullptr;
+  float* rope_cos[2] = {nullptr, nullptr};  // [0] full layers, [1] sliding layers
+  float* rope_sin[2] = {nullptr, nullptr};
+  bf16* deq = nullptr;
+  std::vector<LayerPlan> plans;
+  GemmPlan deq_w13, deq_w2;  // NVFP4: maps over the dequantised weights (b, b3)
+  std::string msg;
+  int launches = 0;
+  // decode-step CUDA graphs, keyed by batch, split count and every device pointer the step reads
+  struct GraphEntry {
+    std::vector<const void*> key;
+    cudaGraphExec_t exec;
+    int launches;
+  };
+  std::vector<GraphEntry> graphs;
+  cudaStream_t cap_stream = nullptr;  // capture only; graphs launch on the caller's stream
+  bool graphs_on = true;
+  // measurement brackets (lfm3_profile_*)
+  bool prof = false;
+  std::vector<cudaEvent_t> ev;
+  std::vector<double> ev_bytes, ev_flops;
+  int ev_used = 0, ev_overflow = 0;
+};
+
+namespace {
+
+thread_local std::string g_create_msg;  // message of the last failed lfm3_create on this thread
+
+lfm3_status fail(lfm3_ctx* c, lfm3_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  if (c) c->msg = buf;
+  return s;
+}
+
+#define CK(x)                                                                                     \
+  do {                                                                                            \
+    cudaError_t e_ = (x);                                                                         \
+    if (e_ != cudaSuccess) return fail(ctx, LFM3_E_CUDA, "%s: %s", #x, cudaGetErrorString(e_));   \
+  } while (0)
+
+// Workspace layout; with base == nullptr only sizes it.
+size_t layout(lfm3_ctx* c, char* base) {
+  const lfm3_config& g = c->cfg;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> char* {
+    off = align_up(off, 256);
+    char* p = base ? base + off : nullptr;
+    off += bytes;
+    return p;
+  };
+  const size_t R = c->R;
+  c->err = reinterpret_cast<int*>(take(256));
+  c->row_slot = reinterpret_cast<int32_t*>(take(4 * R));
+  c->row_pos = reinterpret_cast<int32_t*>(take(4 * R));
+  c->amax = reinterpret_cast<unsigned long long*>(take(8 * R));
+  c->x_res = reinterpret_cast<float*>(take(4 * R * D));
+  c->xn = reinterpret_cast<bf16*>(take(2 * R * D));
+  c->big = reinterpret_cast<bf16*>(take(2 * R * F));
+  c->y = reinterpret_cast<bf16*>(take(2 * R * D));
+  // fp32 projection outputs: the conv in_proj [R][3D], qkvg [R][3088], or decode K-split partials
+  c->part = reinterpret_cast<float*>(take(4 * std::max(R * 3 * D, (size_t)SPLIT_MAX * g.max_batch * NQKVG)));
+  c->q = reinterpret_cast<bf16*>(take(2 * R * HQ * HD));
+  c->gate = reinterpret_cast<float*>(take(4 * R * HQ));
+  c->sk = reinterpret_cast<bf16*>(take(2 * (size_t)HKV * c->scratch_rows * HD));
+  c->sv = reinterpret_cast<bf16*>(take(2 * (size_t)HKV * c->scratch_rows * HD));
+  c->attn_part = reinterpret_cast<float*>(take(4 * (size_t)g.max_batch * HQ * c->max_splits * (HD + 2)));
+  for (int k = 0; k < 2; ++k) {
+    c->rope_cos[k] = reinterpret_cast<float*>(take(4 * (size_t)c->max_pos * (HD / 2)));
+    c->rope_sin[k] = reinterpret_cast<float*>(take(4 * (size_t)c->max_pos * (HD / 2)));
+  }
+  c->deq = g.ffn_format == LFM3_FFN_NVFP4 ? reinterpret_cast<bf16*>(take(2 * (size_t)2 * F * D)) : nullptr;
+  return align_up(off, 256);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+lfm3_status check_config(lfm3_ctx* c, const lfm3_config* g) {
+  if (g->n_layers < 1 || g->n_layers > LFM3_MAX_LAYERS)
+    return fail(c, LFM3_E_CONFIG, "n_layers %d outside 1..%d", g->n_layers, LFM3_MAX_LAYERS);
+  for (int i = 0; i < g->n_layers; ++i)
+    if (g->layer_type[i] < 0 || g->layer_type[i] > 2)
+      return fail(c, LFM3_E_CONFIG, "layer_type[%d] = %d is not conv/full/sliding", i, (int)g->layer_type[i]);
+  struct { const char* name; long got, want; } fixed[] = {
+      {"d_model", g->d_model, D}, {"d_ffn", g->d_ffn, F}, {"n_q", g->n_q, HQ}, {"n_kv", g->n_kv, HKV},
+      {"head_dim", g->head_dim, HD}, {"conv_taps", g->conv_taps, TAPS}, {"window", g->window, WIN},
+      {"page_size", g->page_size, PAGE}};
+  for (auto& f : fixed)
+    if (f.got != f.want)
+      return fail(c, LFM3_E_UNSUPPORTED, "Lfm3UnsupportedGeometry: %s = %ld (the kernels implement %ld)", f.name,
+                  f.got, f.want);
+  if (g->rope_pairs_full < 0 || g->rope_pairs_full > HD / 2)
+    return fail(c, LFM3_E_CONFIG, "rope_pairs_full %d outside 0..%d", g->rope_pairs_full, HD / 2);
+  if (!(g->theta_full > 0.f) || !(g->theta_sliding > 0.f) || !(g->eps > 0.f))
+    return fail(c, LFM3_E_CONFIG, "rotary bases and eps must be positive");
+  if (g->ffn_format != LFM3_FFN_BF16 && g->ffn_format != LFM3_FFN_NVFP4)
+    return fail(c, LFM3_E_UNSUPPORTED, "Lfm3UnsupportedFfnFormat: %d", g->ffn_format);
+  if (g->has_head && (g->vocab <= 0 || g->vocab % 16))
+    return fail(c, LFM3_E_UNSUPPORTED, "Lfm3UnsupportedVocab: vocab %d must be a positive multiple of 16", g->vocab);
+  if (g->max_streams < 1) return fail(c, LFM3_E_CONFIG, "max_streams %d < 1", g->max_streams);
+  if (g->max_pages_per_stream < 1) return fail(c, LFM3_E_CONFIG, "max_pages_per_stream < 1");
+  if ((long)g->max_pages_per_stream * PAGE > (1 << 20))
+    return fail(c, LFM3_E_CONFIG, "a slot of %d pages exceeds 2^20 positions", g->max_pages_per_stream);
+  if (g->max_chunk < 1 || g->max_chunk > 2048) return fail(c, LFM3_E_CONFIG, "max_chunk %d outside 1..2048", g->max_chunk);
+  if (g->max_batch < 1 || g->max_batch > 64) return fail(c, LFM3_E_CONFIG, "max_batch %d outside 1..64", g->max_batch);
+  if (g->max_batch > g->max_streams) return fail(c, LFM3_E_CONFIG, "max_batch > max_streams");
+  int nf = 0;
+  for (int i = 0; i < g->n_layers; ++i) nf += g->layer_type[i] == LFM3_LAYER_FULL;
+  if (nf && g->n_pages < 1) return fail(c, LFM3_E_CONFIG, "full-attention layers need n_pages >= 1");
+  return LFM3_OK;
+}
+
+lfm3_status check_weights(lfm3_ctx* c, const lfm3_config* g, const lfm3_weights* w) {
+  if (!w->layers) return fail(c, LFM3_E_ARG, "weights.layers is NULL");
+  if (g->has_head && (!w->embed || !w->final_norm)) return fail(c, LFM3_E_ARG, "has_head needs embed and final_norm");
+  if (g->has_head && (!aligned16(w->embed) || !aligned16(w->final_norm)))
+    return fail(c, LFM3_E_ARG, "embed/final_norm must be 16-byte aligned");
+  for (int i = 0; i < g->n_layers; ++i) {
+    const lfm3_layer_weights& L = w->layers[i];
+    const void* need[16];
+    int n = 0;
+    need[n++] = L.op_norm; need[n++] = L.post_op_norm; need[n++] = L.ffn_norm; need[n++] = L.post_ffn_norm;
+    if (g->layer_type[i] == LFM3_LAYER_CONV) {
+      need[n++] = L.in_proj; need[n++] = L.conv; need[n++] = L.out_proj;
+    } else {
+      need[n++] = L.qkvg; need[n++] = L.q_norm; need[n++] = L.k_norm; need[n++] = L.o_proj;
+    }
+    if (g->ffn_format == LFM3_FFN_BF16) {
+      need[n++] = L.w1; need[n++] = L.w3; need[n++] = L.w2;
+    } else {
+      need[n++] = L.w1_codes; need[n++] = L.w1_scales; need[n++] = L.w3_codes; need[n++] = L.w3_scales;
+      need[n++] = L.w2_codes; need[n++] = L.w2_scales;
+    }
+    for (int j = 0; j < n; ++j) {
+      if (!need[j]) return fail(c, LFM3_E_ARG, "layer %d: a required weight pointer is NULL (field %d)", i, j);
+      if (!aligned16(need[j])) return fail(c, LFM3_E_ARG, "layer %d: weight field %d is not 16-byte aligned", i, j);
+    }
+  }
+  return LFM3_OK;
+}
+
+const bf16* B(const void* p) { return reinterpret_cast<const bf16*>(p); }
+
+// Brackets one projection launch with events when measurement is on.
+struct Bracket {
+  lfm3_ctx* c;
+  cudaStream_t s;
+  int i = -1;
+  Bracket(lfm3_ctx* c_, cudaStream_t s_, double bytes, double flops) : c(c_), s(s_) {
+    if (!c->prof) return;
+    if (c->ev_used >= (int)c->ev_bytes.size()) { ++c->ev_overflow; return; }
+    i = c->ev_used++;
+    c->ev_bytes[i] = bytes;
+    c->ev_flops[i] = flops;
+    cudaEventRecord(c->ev[2 * i], s);
+  }
+  ~Bracket() {
+    if (i >= 0) cudaEventRecord(c->ev[2 * i + 1], s);
+  }
+};
+
+double gemv_bytes(const GemvArgs& a, int nvfp4) {
+  const double w = nvfp4 ? (double)a.N * a.K / 2 + (double)a.N * a.K / 16 : 2.0 * a.N * a.K;
+  return w + 2.0 * a.rows * a.K + 4.0 * a.rows * a.N;
+}
+double gemv_flops(const GemvArgs& a) { return 2.0 * a.rows * a.N * a.K; }
+double gemm_flops(const GemmPlan& p, int M) {
+  return 2.0 * M * (double)p.N * p.K * (p.epi == GEMM_SWIGLU ? 2 : 1);
+}
+double gemm_bytes(const GemmPlan& p, int M) {
+  const int nw = p.epi == GEMM_SWIGLU ? 2 : 1;
+  return 2.0 * nw * p.N * (double)p.K + 2.0 * M * p.K + (p.epi == GEMM_F32 ? 4.0 : 2.0) * M * p.N;
+}
+
+cudaError_t run_gemv(lfm3_ctx* c, int epi, int fp4, const GemvArgs& a, cudaStream_t s) {
+  Bracket b(c, s, gemv_bytes(a, fp4), gemv_flops(a));
+  return gemv(epi, fp4, a, s);
+}
+cudaError_t run_gemm(lfm3_ctx* c, const GemmPlan& p, int M, cudaStream_t s) {
+  Bracket b(c, s, gemm_bytes(p, M), gemm_flops(p, M));
+  return gemm(p, M, c->err, s);
+}
+
+bool plan_gemm(GemmPlan* p, int epi, const void* a, int a_rows, const void* b, const void* b3, int N, int K, void* out,
+               int ld, float alpha) {
+  p->epi = epi;
+  p->N = N;
+  p->K = K;
+  p->M = a_rows;
+  p->out = out;
+  p->ld = ld;
+  p->alpha = alpha;
+  const uint32_t box_b = (epi == GEMM_SWIGLU) ? 128 : (N > 4096 ? 256 : 128);
+  if (!make_tmap_bf16(&p->a, a, a_rows, K, 128)) return false;
+  if (!make_tmap_bf16(&p->b, b, N, K, box_b)) return false;
+  if (b3 && !make_tmap_bf16(&p->b3, b3, N, K, box_b)) return false;
+  if (!b3) p->b3 = p->b;
+  return true;
+}
+
+// Host check that every position a call writes or reads in slot s, [0, end), has a page.
+lfm3_status check_pages(lfm3_ctx* ctx, const lfm3_state* st, int slot, long end) {
+  const lfm3_config& g = ctx->cfg;
+  if (end > ctx->max_pos)
+    return fail(ctx, LFM3_E_CAPACITY, "slot %d: %ld positions exceed the slot's %d pages of %d", slot, end,
+                g.max_pages_per_stream, PAGE);
+  if (ctx->n_full == 0) return LFM3_OK;
+  if (!st->h_page_table) return fail(ctx, LFM3_E_ARG, "h_page_table is NULL");
+  const long npg = (end + PAGE - 1) / PAGE;
+  for (long p = 0; p < npg; ++p) {
+    const int32_t pg = st->h_page_table[(size_t)slot * g.max_pages_per_stream + p];
+    if (pg < 0 || pg >= g.n_pages)
+      return fail(ctx, LFM3_E_CAPACITY, "slot %d: page %ld of its table is %d, outside the pool of %d", slot, p, pg,
+                  g.n_pages);
+  }
+  return LFM3_OK;
+}
+
+lfm3_status check_state(lfm3_ctx* ctx, const lfm3_state* st) {
+  if (!st) return fail(ctx, LFM3_E_ARG, "state is NULL");
+  if (!st->seq_len || !st->h_seq_len) return fail(ctx, LFM3_E_ARG, "seq_len / h_seq_len is NULL");
+  if (ctx->n_conv && !st->conv_state) return fail(ctx, LFM3_E_ARG, "conv_state is NULL");
+  if (ctx->n_sliding && (!st->ring_k || !st->ring_v)) return fail(ctx, LFM3_E_ARG, "ring_k / ring_v is NULL");
+  if (ctx->n_full && (!st->kv_k || !st->kv_v || !st->page_table)) return fail(ctx, LFM3_E_ARG, "kv_k/kv_v/page_table is NULL");
+  return LFM3_OK;
+}
+
+// ---------------------------------------------------------------- per-layer pieces
+struct Views {
+  bf16* conv_layer;  // conv state of this conv layer, all slots
+  bf16* ring_k; bf16* ring_v;
+  bf16* kv_k; bf16* kv_v;
+};
+
+Views views(lfm3_ctx* ctx, const lfm3_state* st, int l) {
+  const lfm3_config& g = ctx->cfg;
+  Views v{};
+  const int j = ctx->kidx[l];
+  switch (g.layer_type[l]) {
+    case LFM3_LAYER_CONV:
+      v.conv_layer = reinterpret_cast<bf16*>(st->conv_state) + (size_t)j * g.max_streams * CST * D;
+      break;
+    case LFM3_LAYER_SLIDING: {
+      const size_t per = (size_t)g.max_streams * HKV * WIN * HD;
+      v.ring_k = reinterpret_cast<bf16*>(st->ring_k) + j * per;
+      v.ring_v = reinterpret_cast<bf16*>(st->ring_v) + j * per;
+      break;
+    }
+    default: {
+      const size_t per = (size_t)g.n_pages * HKV * PAGE * HD;
+      v.kv_k = reinterpret_cast<bf16*>(st->kv_k) + j * per;
+      v.kv_v = reinterpret_cast<bf16*>(st->kv_v) + j * per;
+    }
+  }
+  return v;
+}
+
+AttnLayer attn_layer(lfm3_ctx* ctx, const lfm3_state* st, int l, const Views& v) {
+  const lfm3_config& g = ctx->cfg;
+  AttnLayer a{};
+  a.full = g.layer_type[l] == LFM3_LAYER_FULL;
+  a.k = a.full ? v.kv_k : v.ring_k;
+  a.v = a.full ? v.kv_v : v.ring_v;
+  a.page_table = st->page_table;
+  a.max_pages = g.max_pages_per_stream;
+  a.max_streams = g.max_streams;
+  return a;
+}
+
+// FFN of n rows (prefill or large-batch decode) on the tensor-core GEMM: u = SwiGLU -> big, w2 -> part.
+lfm3_status ffn_gemm(lfm3_ctx* ctx, int l, int n, cudaStream_t s) {
+  const lfm3_layer_weights& W = ctx->L[l];
+  if (ctx->cfg.ffn_format == LFM3_FFN_NVFP4) {
+    CK(nvfp4_to_bf16(W.w1_codes, W.w1_scales, W.w13_scale, F, D, ctx->deq, s));
+    CK(nvfp4_to_bf16(W.w3_codes, W.w3_scales, W.w13_scale, F, D, ctx->deq + (size_t)F * D, s));
+    GemmPlan p = ctx->deq_w13;
+    p.alpha = W.w13_scale;
+    CK(run_gemm(ctx, p, n, s));
+    CK(nvfp4_to_bf16(W.w2_codes, W.w2_scales, W.w2_scale, D, F, ctx->deq, s));
+    GemmPlan p2 = ctx->deq_w2;
+    p2.alpha = W.w2_scale;
+    CK(run_gemm(ctx, p2, n, s));
+  } else {
+    CK(run_gemm(ctx, ctx->plans[l].w13, n, s));
+    CK(run_gemm(ctx, ctx->plans[l].w2, n, s));
+  }
+  return LFM3_OK;
+}
+
+}  // namespace
+
+// ======================================================================================== ABI
+
+extern "C" lfm3_status lfm3_create(const lfm3_config* cfg, const lfm3_weights* w, size_t* workspace_bytes,
+                                   lfm3_ctx** out) {
+  if (!cfg || !w || !workspace_bytes || !out) return LFM3_E_ARG;
+  *out = nullptr;
+  lfm3_ctx* c = new lfm3_ctx();
+  lfm3_status st = check_config(c, cfg);
+  if (st == LFM3_OK) st = check_weights(c, cfg, w);
+  if (st != LFM3_OK) {
+    g_create_msg = c->msg;
+    delete c;
+    return st;
+  }
+  g_create_msg.clear();
+  c->cfg = *cfg;
+  c->L.assign(w->layers, w->layers + cfg->n_layers);
+  c->embed = B(w->embed);
+  c->final_norm = B(w->final_norm);
+  for (int i = 0; i < cfg->n_layers; ++i) {
+    const int t = cfg->layer_type[i];
+    c->kidx.push_back(t == LFM3_LAYER_CONV ? c->n_conv++ : t == LFM3_LAYER_FULL ? c->n_full++ : c->n_sliding++);
+  }
+  c->max_pos = cfg->max_pages_per_stream * PAGE;
+  c->R = std::max(cfg->max_chunk, cfg->max_batch);
+  c->max_splits = std::max((c->max_pos + 255) / 256, 4);
+  c->scratch_rows = WIN + cfg->max_chunk;
+  c->ws_bytes = layout(c, nullptr);
+  *workspace_bytes = c->ws_bytes;
+  *out = c;
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t bytes) {
+  if (!ctx) return LFM3_E_ARG;
+  if (!d_ws || (reinterpret_cast<uintptr_t>(d_ws) & 255))
+    return fail(ctx, LFM3_E_ARG, "workspace must be non-NULL and 256-byte aligned");
+  if (bytes < ctx->ws_bytes)
+    return fail(ctx, LFM3_E_ARG, "workspace of %zu bytes is smaller than the %zu required", bytes, ctx->ws_bytes);
+  if (!tma_init()) return fail(ctx, LFM3_E_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  CK(gemv_init());
+  CK(gemm_init());
+  CK(attn_init());
+  layout(ctx, reinterpret_cast<char*>(d_ws));
+  const lfm3_config& g = ctx->cfg;
+  const int R = ctx->R;
+  // rotary tables in double precision, stored fp32: [pos][i] for pairs (i, i + 64)
+  {
+    std::vector<float> cs((size_t)ctx->max_pos * (HD / 2)), sn(cs.size());
+    for (int k = 0; k < 2; ++k) {
+      const double theta = k == 0 ? g.theta_full : g.theta_sliding;
+      const int pairs = k == 0 ? g.rope_pairs_full : HD / 2;
+      for (int i = 0; i < HD / 2; ++i) {
+        const double inv = i < pairs ? std::pow(theta, -2.0 * i / HD) : 0.0;
+        for (int p = 0; p < ctx->max_pos; ++p) {
+          cs[(size_t)p * (HD / 2) + i] = (float)std::cos(p * inv);
+          sn[(size_t)p * (HD / 2) + i] = (float)std::sin(p * inv);
+        }
+      }
+      CK(cudaMemcpy(ctx->rope_cos[k], cs.data(), cs.size() * 4, cudaMemcpyHostToDevice));
+      CK(cudaMemcpy(ctx->rope_sin[k], sn.data(), sn.size() * 4, cudaMemcpyHostToDevice));
+    }
+  }
+  CK(cudaMemset(ctx->err, 0, 256));
+  // GEMM plans (tensor maps over the weights and the workspace activations)
+  ctx->plans.assign(g.n_layers, LayerPlan{});
+  for (int l = 0; l < g.n_layers; ++l) {
+    const lfm3_layer_weights& W = ctx->L[l];
+    LayerPlan& P = ctx->plans[l];
+    bool ok = true;
+    if (g.layer_type[l] == LFM3_LAYER_CONV) {
+      ok &= plan_gemm(&P.in_proj, GEMM_F32, ctx->xn, R, W.in_proj, nullptr, 3 * D, D, ctx->part, 3 * D, 1.f);
+      ok &= plan_gemm(&P.out_proj, GEMM_F32, ctx->y, R, W.out_proj, nullptr, D, D, ctx->part, D, 1.f);
+    } else {
+      ok &= plan_gemm(&P.qkvg, GEMM_F32, ctx->xn, R, W.qkvg, nullptr, NQKVG, D, ctx->part, NQKVG, 1.f);
+      ok &= plan_gemm(&P.o_proj, GEMM_F32, ctx->y, R, W.o_proj, nullptr, D, HQ * HD, ctx->part, D, 1.f);
+    }
+    if (g.ffn_format == LFM3_FFN_BF16) {
+      ok &= plan_gemm(&P.w13, GEMM_SWIGLU, ctx->xn, R, W.w1, W.w3, F, D, ctx->big, F, 1.f);
+      ok &= plan_gemm(&P.w2, GEMM_F32, ctx->big, R, W.w2, nullptr, D, F, ctx->part, D, 1.f);
+    }
+    if (!ok) return fail(ctx, LFM3_E_CUDA, "layer %d: tensor map encoding failed", l);
+  }
+  if (g.ffn_format == LFM3_FFN_NVFP4) {
+    bool ok = plan_gemm(&ctx->deq_w13, GEMM_SWIGLU, ctx->xn, R, ctx->deq, ctx->deq + (size_t)F * D, F, D, ctx->big, F, 1.f);
+    ok &= plan_gemm(&ctx->deq_w2, GEMM_F32, ctx->big, R, ctx->deq, nullptr, D, F, ctx->part, D, 1.f);
+    if (!ok) return fail(ctx, LFM3_E_CUDA, "NVFP4 tensor map encoding failed");
+  }
+  CK(cudaDeviceSynchronize());
+  ctx->graphs_on = getenv("LFM3_NO_GRAPH") == nullptr;
+  ctx->bound = true;
+  ctx->msg.clear();
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slot, const int32_t* d_tokens,
+                                    const void* d_embeds, int n, float* d_logits, int32_t* d_argmax, float* d_hidden,
+                                    void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
+  const lfm3_config& g = ctx->cfg;
+  lfm3_status vs = check_state(ctx, st);
+  if (vs != LFM3_OK) return vs;
+  if (slot < 0 || slot >= g.max_streams) return fail(ctx, LFM3_E_ARG, "slot %d outside 0..%d", slot, g.max_streams - 1);
+  if (n < 1) return fail(ctx, LFM3_E_ARG, "n = %d rows", n);
+  if (g.has_head && !d_tokens) return fail(ctx, LFM3_E_ARG, "has_head needs d_tokens");
+  if (!g.has_head && !d_embeds) return fail(ctx, LFM3_E_ARG, "a model without embedding needs d_embeds");
+  if (!g.has_head && (d_logits || d_argmax)) return fail(ctx, LFM3_E_ARG, "a model without head has no logits");
+  const long p_start = st->h_seq_len[slot];
+  if (p_start < 0) return fail(ctx, LFM3_E_ARG, "h_seq_len[%d] = %ld", slot, p_start);
+  vs = check_pages(ctx, st, slot, p_start + n);
+  if (vs != LFM3_OK) return vs;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  g_launches = 0;
+  const float eps = g.eps;
+  for (int c0 = 0; c0 < n; c0 += g.max_chunk) {
+    const int nc = std::min(g.max_chunk, n - c0);
+    const int p0 = (int)p_start + c0;
+    const bool last = c0 + nc == n;
+    CK(setup_rows(1, slot, nullptr, st->seq_len, nc, ctx->row_slot, ctx->row_pos, ctx->amax, s));
+    const Rows rows{ctx->row_slot, ctx->row_pos, nc};
+    CK(embed_rows(d_tokens ? d_tokens + c0 : nullptr, ctx->embed,
+                  d_embeds ? B(d_embeds) + (size_t)c0 * D : nullptr, nc, ctx->x_res,
+                  d_hidden ? d_hidden + (size_t)c0 * D : nullptr, s));
+    CK(resid_norm(ctx->x_res, nullptr, 0, 0, nullptr, B(ctx->L[0].op_norm), ctx->xn, nc, eps, nullptr, s));
+    for (int l = 0; l < g.n_layers; ++l) {
+      const lfm3_layer_weights& W = ctx->L[l];
+      const LayerPlan& P = ctx->plans[l];
+      const Views v = views(ctx, st, l);
+      if (g.layer_type[l] == LFM3_LAYER_CONV) {
+        CK(run_gemm(ctx, P.in_proj, nc, s));
+        CK(conv_prefill(ctx->part, B(W.conv), v.conv_layer + (size_t)slot * CST * D, nc, ctx->y, s));
+        CK(run_gemm(ctx, P.out_proj, nc, s));
+      } else {
+        const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
+        CK(run_gemm(ctx, P.qkvg, nc, s));
+        if (!full)
+          CK(ring_to_scratch(v.ring_k, v.ring_v, slot, g.max_streams, p0, ctx->sk, ctx->sv, ctx->scratch_rows, s));
+        KvWrite kw{};
+        kw.mode = full ? KV_PAGES : KV_SCRATCH;
+        kw.k = full ? v.kv_k : ctx->sk;
+        kw.v = full ? v.kv_v : ctx->sv;
+        kw.page_table = st->page_table;
+        kw.max_pages = g.max_pages_per_stream;
+        kw.max_streams = g.max_streams;
+        kw.scratch_rows = ctx->scratch_rows;
+        const int k = full ? 0 : 1;
+        CK(qk_norm_rope_kv(ctx->part, 1, 0, B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], rows, eps,
+                           ctx->q, ctx->gate, kw, s));
+        CK(attn_prefill(ctx->q, nc, p0, slot, attn_layer(ctx, st, l, v), ctx->sk, ctx->sv, ctx->scratch_rows,
+                        ctx->gate, ctx->y, s));
+        if (!full)
+          CK(scratch_to_ring(ctx->sk, ctx->sv, ctx->scratch_rows, nc, p0, v.ring_k, v.ring_v, slot, g.max_streams, s));
+        CK(run_gemm(ctx, P.o_proj, nc, s));
+      }
+      CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nc, eps, nullptr, s));
+      lfm3_status fs = ffn_gemm(ctx, l, nc, s);
+      if (fs != LFM3_OK) return fs;
+      const bf16* gnext = l + 1 < g.n_layers ? B(ctx->L[l + 1].op_norm) : (g.has_head ? ctx->final_norm : nullptr);
+      CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_ffn_norm), gnext, ctx->xn, nc, eps,
+                    d_hidden ? d_hidden + ((size_t)(l + 1) * n + c0) * D : nullptr, s));
+    }
+    const bool head = last && g.has_head && (d_logits || d_argmax);
+    if (head) {
+      GemvArgs a{};
+      a.w = ctx->embed;
+      a.x = ctx->xn + (size_t)(nc - 1) * D;
+      a.K = D;
+      a.N = g.vocab;
+      a.rows = 1;
+      a.splits = 1;
+      a.part = d_logits;
+      a.amax = ctx->amax;
+      CK(run_gemv(ctx, GEMV_HEAD, 0, a, s));
+    }
+    CK(finish_step(st->seq_len, ctx->row_slot, nc, nc, slot, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
+  }
+  st->h_seq_len[slot] += n;
+  ctx->launches = g_launches;
+  return LFM3_OK;
+}
+
+namespace {
+
+// Every launch of one decode step, in order, on stream s.
+lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* d_slots,
+                           const int32_t* d_tokens, const void* d_embeds, float* d_logits, int32_t* d_argmax,
+                           float* d_hidden, int splits_full, cudaStream_t s) {
+  const lfm3_config& g = ctx->cfg;
+  const float eps = g.eps;
+  const bool gv = nb <= GEMV_MAX_ROWS;
+  const bool fp4 = g.ffn_format == LFM3_FFN_NVFP4;
+  CK(setup_rows(0, 0, d_slots, st->seq_len, nb, ctx->row_slot, ctx->row_pos, ctx->amax, s));
+  const Rows rows{ctx->row_slot, ctx->row_pos, nb};
+  CK(embed_rows(d_tokens, ctx->embed, B(d_embeds), nb, ctx->x_res, d_hidden, s));
+  CK(resid_norm(ctx->x_res, nullptr, 0, 0, nullptr, B(ctx->L[0].op_norm), ctx->xn, nb, eps, nullptr, s));
+  for (int l = 0; l < g.n_layers; ++l) {
+    const lfm3_layer_weights& W = ctx->L[l];
+    const LayerPlan& P = ctx->plans[l];
+    const Views v = views(ctx, st, l);
+    int np = 1;
+    long pstride = 0;
+    GemvArgs a{};
+    a.rows = nb;
+    a.row_slot = ctx->row_slot;
+    a.max_streams = g.max_streams;
+    if (g.layer_type[l] == LFM3_LAYER_CONV) {
+      if (gv) {
+        a.w = B(W.in_proj); a.x = ctx->xn; a.K = D; a.N = 3 * D; a.splits = 1;
+        a.conv_w = B(W.conv); a.conv_state = v.conv_layer; a.y = ctx->y;
+        CK(run_gemv(ctx, GEMV_CONV, 0, a, s));
+        GemvArgs o{};
+        o.w = B(W.out_proj); o.x = ctx->y; o.K = D; o.N = D; o.rows = nb; o.splits = SPLIT_DD; o.part = ctx->part;
+        CK(run_gemv(ctx, GEMV_PARTIAL, 0, o, s));
+        np = SPLIT_DD;
+        pstride = (long)nb * D;
+      } else {
+        CK(run_gemm(ctx, P.in_proj, nb, s));
+        CK(conv_decode(ctx->part, B(W.conv), v.conv_layer, ctx->row_slot, nb, ctx->y, s));
+        CK(run_gemm(ctx, P.out_proj, nb, s));
+      }
+    } else {
+      const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
+      int nq = 1;
+      long qstride = 0;
+      if (gv) {
+        a.w = B(W.qkvg); a.x = ctx->xn; a.K = D; a.N = NQKVG; a.splits = SPLIT_QKVG; a.part = ctx->part;
+        CK(run_gemv(ctx, GEMV_PARTIAL, 0, a, s));
+        nq = SPLIT_QKVG;
+        qstride = (long)nb * NQKVG;
+      } else {
+        CK(run_gemm(ctx, P.qkvg, nb, s));
+      }
+      KvWrite kw{};
+      kw.mode = full ? KV_PAGES : KV_RING;
+      kw.k = full ? v.kv_k : v.ring_k;
+      kw.v = full ? v.kv_v : v.ring_v;
+      kw.page_table = st->page_table;
+      kw.max_pages = g.max_pages_per_stream;
+      kw.max_streams = g.max_streams;
+      const int k = full ? 0 : 1;
+      CK(qk_norm_rope_kv(ctx->part, nq, qstride, B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], rows,
+                         eps, ctx->q, ctx->gate, kw, s));
+      CK(attn_decode(ctx->q, rows, attn_layer(ctx, st, l, v), full ? splits_full : WIN / 64, ctx->attn_part,
+                     ctx->gate, ctx->y, s));
+      if (gv) {
+        GemvArgs o{};
+        o.w = B(W.o_proj); o.x = ctx->y; o.K = HQ * HD; o.N = D; o.rows = nb; o.splits = SPLIT_DD; o.part = ctx->part;
+        CK(run_gemv(ctx, GEMV_PARTIAL, 0, o, s));
+        np = SPLIT_DD;
+        pstride = (long)nb * D;
+      } else {
+        CK(run_gemm(ctx, P.o_proj, nb, s));
+      }
+    }
+    CK(resid_norm(ctx->x_res, ctx->part, np, pstride, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nb, eps, nullptr, s));
+    np = 1;
+    pstride = 0;
+    if (gv) {
+      GemvArgs f{};
+      f.rows = nb; f.x = ctx->xn; f.K = D; f.N = F; f.splits = 1; f.out = ctx->big;
+      if (fp4) {
+        f.codes = W.w1_codes; f.scales = W.w1_scales; f.codes3 = W.w3_codes; f.scales3 = W.w3_scales;
+        f.tscale = W.w13_scale;
+      } else {
+        f.w = B(W.w1); f.w3 = B(W.w3);
+      }
+      CK(run_gemv(ctx, GEMV_SWIGLU, fp4, f, s));
+      GemvArgs d{};
+      d.rows = nb; d.x = ctx->big; d.K = F; d.N = D; d.part = ctx->part;
+      d.splits = fp4 ? SPLIT_W2_FP4 : SPLIT_W2;
+      if (fp4) {
+        d.codes = W.w2_codes; d.scales = W.w2_scales; d.tscale = W.w2_scale;
+      } else {
+        d.w = B(W.w2);
+      }
+      CK(run_gemv(ctx, GEMV_PARTIAL, fp4, d, s));
+      np = d.splits;
+      pstride = (long)nb * D;
+    } else {
+      lfm3_status fs = ffn_gemm(ctx, l, nb, s);
+      if (fs != LFM3_OK) return fs;
+    }
+    const bf16* gnext = l + 1 < g.n_layers ? B(ctx->L[l + 1].op_norm) : (g.has_head ? ctx->final_norm : nullptr);
+    CK(resid_norm(ctx->x_res, ctx->part, np, pstride, B(W.post_ffn_norm), gnext, ctx->xn, nb, eps,
+                  d_hidden ? d_hidden + (size_t)(l + 1) * nb * D : nullptr, s));
+  }
+  const bool head = g.has_head && (d_logits || d_argmax);
+  if (head) {
+    for (int b0 = 0; b0 < nb; b0 += GEMV_MAX_ROWS) {
+      GemvArgs a{};
+      a.w = ctx->embed;
+      a.x = ctx->xn + (size_t)b0 * D;
+      a.K = D;
+      a.N = g.vocab;
+      a.rows = std::min(GEMV_MAX_ROWS, nb - b0);
+      a.splits = 1;
+      a.part = d_logits ? d_logits + (size_t)b0 * g.vocab : nullptr;
+      a.amax = ctx->amax + b0;
+      CK(run_gemv(ctx, GEMV_HEAD, 0, a, s));
+    }
+  }
+  CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
+  return LFM3_OK;
+}
+
+}  // namespace
+
+extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* h_slots,
+                                        const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
+                                        float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
+  const lfm3_config& g = ctx->cfg;
+  lfm3_status vs = check_state(ctx, st);
+  if (vs != LFM3_OK) return vs;
+  if (nb < 1 || nb > g.max_batch) return fail(ctx, LFM3_E_ARG, "n_streams %d outside 1..%d", nb, g.max_batch);
+  if (!h_slots || !d_slots) return fail(ctx, LFM3_E_ARG, "h_slots / d_slots is NULL");
+  if (g.has_head && !d_tokens) return fail(ctx, LFM3_E_ARG, "has_head needs d_tokens");
+  if (!g.has_head && !d_embeds) return fail(ctx, LFM3_E_ARG, "a model without embedding needs d_embeds");
+  if (!g.has_head && (d_logits || d_argmax)) return fail(ctx, LFM3_E_ARG, "a model without head has no logits");
+  int maxpos = 0;
+  for (int b = 0; b < nb; ++b) {
+    const int s = h_slots[b];
+    if (s < 0 || s >= g.max_streams) return fail(ctx, LFM3_E_ARG, "slot %d outside 0..%d", s, g.max_streams - 1);
+    for (int c = 0; c < b; ++c)
+      if (h_slots[c] == s) return fail(ctx, LFM3_E_ARG, "slot %d listed twice", s);
+    vs = check_pages(ctx, st, s, (long)st->h_seq_len[s] + 1);
+    if (vs != LFM3_OK) return vs;
+    maxpos = std::max(maxpos, (int)st->h_seq_len[s]);
+  }
+
+  // full-layer split count, quantised to a power of two so that one graph serves a range of contexts
+  int splits_full = 1;
+  while (splits_full < maxpos / 256 + 1) splits_full *= 2;
+  splits_full = std::min(splits_full, ctx->max_splits);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  g_launches = 0;
+  if (!ctx->graphs_on || ctx->prof) {
+    lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                                    splits_full, s);
+    if (es != LFM3_OK) return es;
+    ctx->launches = g_launches;
+  } else {
+    std::vector<const void*> key = {reinterpret_cast<const void*>((intptr_t)nb),
+                                    reinterpret_cast<const void*>((intptr_t)splits_full), d_slots, d_tokens, d_embeds,
+                                    d_logits, d_argmax, d_hidden, st->conv_state, st->ring_k, st->ring_v, st->kv_k,
+                                    st->kv_v, st->page_table, st->seq_len};
+    lfm3_ctx::GraphEntry* hit = nullptr;
+    for (auto& e : ctx->graphs)
+      if (e.key == key) hit = &e;
+    if (!hit) {
+      if (!ctx->cap_stream) CK(cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking));
+      if (ctx->graphs.size() >= 32) {
+        for (auto& e : ctx->graphs) cudaGraphExecDestroy(e.exec);
+        ctx->graphs.clear();
+      }
+      cudaGraph_t graph = nullptr;
+      CK(cudaStreamBeginCapture(ctx->cap_stream, cudaStreamCaptureModeThreadLocal));
+      lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                                      splits_full, ctx->cap_stream);
+      cudaError_t ce = cudaStreamEndCapture(ctx->cap_stream, &graph);
+      if (es != LFM3_OK) {
+        if (graph) cudaGraphDestroy(graph);
+        return es;
+      }
+      CK(ce);
+      cudaGraphExec_t exec = nullptr;
+      ce = cudaGraphInstantiate(&exec, graph, 0);
+      cudaGraphDestroy(graph);
+      CK(ce);
+      ctx->graphs.push_back({key, exec, g_launches});
+      hit = &ctx->graphs.back();
+    }
+    CK(cudaGraphLaunch(hit->exec, s));
+    ctx->launches = hit->launches;
+  }
+  for (int b = 0; b < nb; ++b) st->h_seq_len[h_slots[b]] += 1;
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_check_device_errors(lfm3_ctx* ctx, void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
+  CK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  int e = 0;
+  CK(cudaMemcpy(&e, ctx->err, sizeof e, cudaMemcpyDeviceToHost));
+  if (e) {
+    CK(cudaMemset(ctx->err, 0, sizeof e));
+    return fail(ctx, LFM3_E_TIMEOUT, "a device-side bounded wait gave up (status %d)", e);
+  }
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_profile_enable(lfm3_ctx* ctx, int on, int capacity) {
+  if (!ctx) return LFM3_E_ARG;
+  if (on && capacity < 1) return fail(ctx, LFM3_E_ARG, "capacity %d", capacity);
+  for (cudaEvent_t e : ctx->ev) cudaEventDestroy(e);
+  ctx->ev.clear();
+  ctx->ev_bytes.clear();
+  ctx->ev_flops.clear();
+  ctx->ev_used = ctx->ev_overflow = 0;
+  ctx->prof = on != 0;
+  if (!on) return LFM3_OK;
+  ctx->ev.resize(2 * (size_t)capacity);
+  for (auto& e : ctx->ev) CK(cudaEventCreate(&e));
+  ctx->ev_bytes.assign(capacity, 0.0);
+  ctx->ev_flops.assign(capacity, 0.0);
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_profile_read(lfm3_ctx* ctx, int* launches, double* ms, double* bytes, double* flops) {
+  if (!ctx || !launches || !ms || !bytes || !flops) return LFM3_E_ARG;
+  *launches = 0;
+  *ms = *bytes = *flops = 0.0;
+  for (int i = 0; i < ctx->ev_used; ++i) {
+    CK(cudaEventSynchronize(ctx->ev[2 * i + 1]));
+    float t = 0.f;
+    CK(cudaEventElapsedTime(&t, ctx->ev[2 * i], ctx->ev[2 * i + 1]));
+    *ms += t;
+    *bytes += ctx->ev_bytes[i];
+    *flops += ctx->ev_flops[i];
+  }
+  *launches = ctx->ev_used;
+  const int over = ctx->ev_overflow;
+  ctx->ev_used = ctx->ev_overflow = 0;
+  if (over) return fail(ctx, LFM3_E_CAPACITY, "%d launches ran unbracketed (capacity exceeded)", over);
+  return LFM3_OK;
+}
+
+extern "C" int lfm3_last_launch_count(const lfm3_ctx* ctx) { return ctx ? ctx->launches : 0; }
+
+extern "C" const char* lfm3_last_error(const lfm3_ctx* ctx) { return ctx ? ctx->msg.c_str() : g_create_msg.c_str(); }
+
+extern "C" void lfm3_free(lfm3_ctx* ctx) {
+  if (!ctx) return;
+  for (cudaEvent_t e : ctx->ev) cudaEventDestroy(e);
+  for (auto& e : ctx->graphs) cudaGraphExecDestroy(e.exec);
+  if (ctx->cap_stream) cudaStreamDestroy(ctx->cap_stream);
+  delete ctx;
+}

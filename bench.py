@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""LFM3-1.7B decode / prefill throughput on B200 through liblfm3.so (one JSON line on rank 0).
+
+Headline (value): greedy decode tok/s of the bf16 24-layer model, batch 1, at a 2048-token
+context (the prompt is prefilled by the library first); one step = embed -> 24 layers -> tied
+head -> argmax for one token, with the next token fed back on the device. Inputs are synthetic
+(seeded random-init weights, uniform token ids); every step streams the 3.46 GB of weights, far
+more than the 126 MB L2, so no explicit L2 flush is needed between steps.
+
+Also reported under "extra": prefill tok/s of an 8192-token prompt in 2048-token chunks over
+shuffled 64-token pages (bf16), and NVFP4-FFN decode tok/s at 1 / 8 streams (2048 context) and
+64 streams (contexts uniform in [256, 8192] on drawn state).
+
+--impl reference times the CPU oracle (float64 NumPy) on the same metric.
+Multi-GPU (torchrun, --gpus N): independent replicas, no collective on the data path; value is
+the sum over ranks (N x steps / max-over-ranks time).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tok/s @1/8/64 streams; prefill tok/s @8k; % of HBM/TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------------------------------- clocks
+class Clocks:
+    """nvidia-smi sampled every 100 ms while the GPU phases run."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                pw = float(r[3])
+            except ValueError:
+                continue
+            if pw < 200:  # idle samples (between phases) do not describe the load
+                continue
+            for i, nm in enumerate(names):
+                if r[5 + i].strip().lower() in ("active", "1"):
+                    reasons.add(nm)
+        loaded = [float(r[1]) for r in rows if len(r) > 3 and _f(r[3]) >= 200]
+        return {"sm_mhz": statistics.median(loaded) if loaded else (statistics.median(sm) if sm else None),
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+def _f(x):
+    try:
+        return float(x)
+    except ValueError:
+        return 0.0
+
+
+# ---------------------------------------------------------------------------------------- oracle baseline
+def oracle_decode_rate(max_steps=3, prompt=64, warm=1):
+    """The CPU oracle (float64 NumPy, all host cores) on a bounded sample of the decode workload:
+    the bf16 24-layer model, a `prompt`-token prompt, then timed greedy decode steps."""
+    from lfm3_inputs import lfm3_1p7b, make_weights, make_tokens
+    from oracle import Lfm3Oracle
+    g = lfm3_1p7b()
+    o = Lfm3Oracle(make_weights(g, 0))
+    st = o.new_state()
+    out = o.forward_chunk(st, tokens=make_tokens(1, "prompt", prompt, g.vocab))
+    tok = int(np.argmax(out["logits"]))
+    for _ in range(warm):
+        tok = int(np.argmax(o.forward_chunk(st, tokens=np.array([tok]))["logits"]))
+    t0 = time.perf_counter()
+    for _ in range(max_steps):
+        tok = int(np.argmax(o.forward_chunk(st, tokens=np.array([tok]))["logits"]))
+    dt = time.perf_counter() - t0
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            threads = max(i.get("num_threads", 0) for i in info)
+    except Exception:
+        pass
+    return max_steps / dt, threads, dt
+
+
+# ---------------------------------------------------------------------------------------- GPU arm
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(world, x):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(world, fn, steps, stream):
+    """Device time of `steps` calls of fn(), CUDA events on the launching stream, max over ranks."""
+    import torch
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(world, e0.elapsed_time(e1))
+
+
+def traffic_record(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if its source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(ROOT, rec["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        return rec["dram_bytes_per_launch"] if h == rec["sha256"] else None
+    except Exception:
+        return None
+
+
+def run_ours(args):
+    import torch
+    from attention_decoder_b200.model import Lfm3Model
+    from lfm3_inputs import lfm3_1p7b, make_weights, make_tokens, page_permutation, context_lengths
+
+    world, rank, local = dist_setup(args)
+    pk, pk_kind = peaks()
+    stream = torch.cuda.current_stream()
+    K, Wm = args.steps, args.warmup
+    clocks = Clocks(local)
+    g = lfm3_1p7b()
+    if args.small:
+        # profiling case: 4 layers (conv, sliding, full, conv) + the tied head, 256-token context
+        g = lfm3_1p7b(layer_types=(0, 2, 1, 0))
+        args.no_extra = True
+    res = {}
+
+    # ---------------- bf16 model: decode at batch 1 (headline) and prefill 8k
+    W = make_weights(g, 0)
+    ctx0 = 256 if args.small else 2048
+    need = ctx0 + Wm + K + 8
+    mpp = max(128, (need + 63) // 64 + 1)
+    m = Lfm3Model(W, max_streams=1, max_pages_per_stream=mpp, max_batch=1)
+    del W
+    prompt = torch.from_numpy(make_tokens(1, "prompt", 2048, g.vocab)[:ctx0]).cuda()
+
+    def fresh_state(model, page_table=None):
+        st = model.new_state(page_table=page_table)
+        o = model.prefill(st, 0, tokens=prompt)
+        return st, o
+
+    st, o = fresh_state(m)
+    bufs = {"argmax": o["argmax"].clone(), "logits": torch.empty(1, g.vocab, device="cuda")}
+    slots_d = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step():
+        m.decode(st, [0], tokens=bufs["argmax"], d_slots=slots_d, out=bufs)
+
+    for _ in range(Wm):
+        step()
+    ms = timed(world, step, K, stream)
+    launches_per_step = m.last_launch_count()
+    res["decode_b1"] = {"ms_per_step": ms / K, "tok_s": K / (ms / 1e3)}
+
+    # kernel roofline: the weight-streaming GEMV (dominant kernel), event-bracketed pass
+    st, o = fresh_state(m)
+    bufs["argmax"].copy_(o["argmax"])
+    m.profile(True, capacity=200 * (K + 1))
+    for _ in range(K):
+        step()
+    prof = m.profile_read()
+    m.profile(False)
+    gemv_gbs = prof["bytes"] / (prof["ms"] / 1e3) / 1e9
+    step_bytes = prof["bytes"] / K
+
+    # end to end through the public API with host buffers: pinned token in, greedy id out, each step
+    st, o = fresh_state(m)
+    h_tok = torch.empty(1, dtype=torch.int32).pin_memory()
+    h_out = torch.empty(1, dtype=torch.int32).pin_memory()
+    h_tok.copy_(o["argmax"].cpu())
+    d_tok = torch.empty(1, dtype=torch.int32, device="cuda")
+
+    def e2e_step():
+        d_tok.copy_(h_tok, non_blocking=True)
+        m.decode(st, [0], tokens=d_tok, d_slots=slots_d, out=bufs)
+        h_out.copy_(bufs["argmax"], non_blocking=True)
+        stream.synchronize()
+        h_tok.copy_(h_out)
+
+    for _ in range(min(Wm, 3)):
+        e2e_step()
+    barrier(world)
+    t0 = time.perf_counter()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(world, e0.elapsed_time(e1))
+
+    # prefill 8k (chunks of 2048) over shuffled pages
+    if not args.no_extra:
+        n8 = 8192
+        mp = Lfm3Model(make_weights(g, 0), max_streams=1, max_pages_per_stream=n8 // 64, max_batch=1)
+        pt = page_permutation(1, "pages8k", n8 // 64).reshape(1, -1)
+        tok8 = torch.from_numpy(make_tokens(1, "prompt8k", n8, g.vocab)).cuda()
+        sts = [mp.new_state(page_table=pt) for _ in range(2)]
+        it = [0]
+
+        def pstep():
+            s = sts[it[0] % 2]
+            it[0] += 1
+            s.h_seq_len[:] = 0
+            s.seq_len.zero_()
+            mp.prefill(s, 0, tokens=tok8)
+
+        for _ in range(2):
+            pstep()
+        pk_steps = max(2, min(K, 8))
+        pms = timed(world, pstep, pk_steps, stream)
+        mp.profile(True, capacity=400)
+        pstep()
+        pprof = mp.profile_read()
+        mp.profile(False)
+        res["prefill_8k"] = {"tok_s": n8 * pk_steps / (pms / 1e3), "ms": pms / pk_steps,
+                             "gemm_tflops": pprof["flops"] / (pprof["ms"] / 1e3) / 1e12,
+                             "gemm_share": pprof["ms"] / (pms / pk_steps)}
+        del mp, sts
+    del m, st
+    torch.cuda.empty_cache()
+
+    # ---------------- NVFP4 FFN model: decode at 1 / 8 streams (2048 ctx) and 64 streams
+    if not args.no_extra:
+        Wq = make_weights(g, 0, ffn="nvfp4")
+        S = 64
+        ctx64 = context_lengths(1, "ctx64", S, 256, 8192)
+        steps_q = max(4, min(K, 32))
+        mpp_q = (8192 + Wm + steps_q + 16) // 64 + 2
+        mq = Lfm3Model(Wq, max_streams=S, max_pages_per_stream=mpp_q, max_batch=S)
+        del Wq
+        stq = mq.new_state(page_table=page_permutation(1, "pages64", S * mpp_q).reshape(S, mpp_q))
+        for s in range(8):
+            mq.prefill(stq, s, tokens=prompt)
+        qb = {}
+        for B in (1, 8):
+            sl = torch.arange(B, dtype=torch.int32, device="cuda")
+            ob = {"argmax": torch.zeros(B, dtype=torch.int32, device="cuda"),
+                  "logits": torch.empty(B, g.vocab, device="cuda")}
+
+            def qstep():
+                mq.decode(stq, list(range(B)), tokens=ob["argmax"], d_slots=sl, out=ob)
+
+            for _ in range(Wm):
+                qstep()
+            qms = timed(world, qstep, steps_q, stream)
+            qb[B] = B * steps_q / (qms / 1e3)
+        # 64 streams on drawn state: K/V, rings and conv columns N(0,1) drawn on the device
+        gen = torch.Generator(device="cuda").manual_seed(1)
+        for t in (stq.kv_k, stq.kv_v, stq.ring_k, stq.ring_v, stq.conv):
+            t.normal_(generator=gen)
+        stq.h_seq_len[:] = ctx64
+        stq.seq_len.copy_(torch.from_numpy(stq.h_seq_len))
+        sl = torch.arange(S, dtype=torch.int32, device="cuda")
+        ob = {"argmax": torch.from_numpy(make_tokens(1, "tok64", S, g.vocab)).cuda(),
+              "logits": torch.empty(S, g.vocab, device="cuda")}
+
+        def q64():
+            mq.decode(stq, list(range(S)), tokens=ob["argmax"], d_slots=sl, out=ob)
+
+        for _ in range(Wm):
+            q64()
+        qms = timed(world, q64, steps_q, stream)
+        qb[64] = S * steps_q / (qms / 1e3)
+        res["decode_nvfp4"] = {f"b{b}_tok_s": v for b, v in qb.items()}
+        res["decode_nvfp4"]["b64_contexts"] = "uniform [256, 8192], mean %.0f" % float(np.mean(ctx64))
+        del mq, stq
+    clk = clocks.stop()
+
+    tok_s_rank = res["decode_b1"]["tok_s"]
+    value = world * tok_s_rank
+    hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tok/s", "n_gpus": world, "steps": K, "warmup": Wm,
+        "ms_per_step": round(res["decode_b1"]["ms_per_step"], 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded random-init weights, uniform token ids)",
+        "config": {"workload": ("LFM3-1.7B bf16 24-layer decode, 1 stream per GPU, greedy, 2048-token context "
+                                "(prefilled), tied 128000 head") if not args.small else
+                               "profiling case: 4-layer LFM3 slice + head, bf16 decode, 256-token context",
+                   "streams_per_gpu": 1, "context": ctx0,
+                   "l2": "no flush: each step streams 3.46 GB of weights, > 126 MB L2",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "kernel": "k_gemv (decode weight-streaming projections)",
+                     "achieved": round(gemv_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gemv_gbs / hbm, 4),
+                     "peak_kind": pk_kind, "traffic": traffic_record("k_gemv"),
+                     "bytes_per_step": round(step_bytes), "kernel_launches_timed": prof["launches"]},
+        "e2e": {"value": round(world * K / (e2e_ms / 1e3), 2), "unit": "tok/s", "h2d_bytes_per_step": 4,
+                "d2h_bytes_per_step": 4},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+        "extra": res,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        rate, threads, dt = oracle_decode_rate()
+        line["cpu_baseline"] = {"value": round(rate, 4), "unit": "tok/s", "cores": threads, "kind": "oracle",
+                                "sample": f"float64 NumPy oracle, bf16 24-layer model, 64-token prompt then 3 timed "
+                                          f"greedy decode steps ({dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    K = min(args.steps, 30)
+    rate, threads, dt = oracle_decode_rate(max_steps=K, prompt=64, warm=min(args.warmup, 1))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(rate, 4), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / rate, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded random-init weights)",
+        "config": {"workload": "LFM3-1.7B bf16 24-layer decode, 1 stream, greedy (CPU oracle)"},
+        "cpu_baseline": {"value": round(rate, 4), "unit": "tok/s", "cores": threads, "kind": "oracle",
+                         "sample": f"float64 NumPy oracle: 64-token prompt, then {K} timed greedy decode steps "
+                                   f"({dt:.1f} s; at most 30 steps are timed)"},
+        "e2e": {"value": round(rate, 4), "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="headline decode only")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--small", action="store_true", help="4-layer profiling case (not a bench line)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * lfm3.h - C ABI of the LFM3-1.7B hybrid decoder forward on one NVIDIA B200 (sm_100a).
+ *
+ * What it computes (coreai-model-zoo note "lfm3-1.7b-port", LFM2.5 -> LFM3 diff table, and
+ * TensorFold issue #1491, "Architecture"): a 24-layer decoder at width 2048 made of
+ *   - 13 gated short-conv blocks: in_proj 2048 -> B | C | x, Bx = B * x, a 7-tap causal
+ *     depthwise conv over Bx whose state keeps the last 6 columns, y = C * conv, out_proj;
+ *   - 6 full-attention and 5 sliding-window (256) GQA blocks: 16 q / 4 kv heads of 128,
+ *     per-head q/k RMSNorm, rotary theta 1e6 on 32 of 64 pairs (full) or theta 1e4 on all
+ *     pairs (sliding), a sigmoid(gate_proj(x)) scalar per head multiplied in before o_proj;
+ *   - sandwich RMSNorms (eps 1e-5) around every mixer and FFN;
+ *   - a SwiGLU FFN of 7680, bf16 or NVFP4 weight-only (TensorFold PR #1508, "What");
+ *   - a tied 128000-row head with greedy (argmax, ties to the lowest id) selection.
+ *
+ * Conventions for every entry point
+ *   - Ownership: the CALLER owns all device memory (weights, state, workspace, outputs) and
+ *     every host array passed in. The library owns only its host-side context.
+ *   - All pointers named d_* or documented "device" are device pointers; h_* are host.
+ *   - bf16 tensors are IEEE bfloat16 bit patterns, row-major, densely packed.
+ *   - Calls enqueue work on the given CUDA stream (a cudaStream_t passed as void*; NULL =
+ *     legacy default stream) and return without synchronising.
+ *   - Errors: arguments, configuration and capacity are checked on the host BEFORE anything
+ *     is enqueued; on any error nothing is launched and no state is modified. CUDA launch
+ *     errors map to LFM3_E_CUDA. lfm3_last_error() gives a message naming the refusal.
+ *   - The library never allocates device memory and never reads /writes device memory from
+ *     the host, except lfm3_bind_workspace (which uploads constant tables into the workspace)
+ *     and lfm3_check_device_errors (which reads one status word).
+ */
+#ifndef LFM3_H
+#define LFM3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct lfm3_ctx lfm3_ctx; /* opaque; created by lfm3_create, freed by lfm3_free */
+
+typedef enum {
+  LFM3_OK = 0,
+  LFM3_E_ARG = -1,         /* a NULL or out-of-range argument                        */
+  LFM3_E_CONFIG = -2,      /* an inconsistent configuration                           */
+  LFM3_E_CAPACITY = -3,    /* rows past a slot's pages, or more rows than the workspace */
+  LFM3_E_CUDA = -4,        /* a CUDA runtime/driver call failed                       */
+  LFM3_E_UNSUPPORTED = -5, /* a geometry the kernels do not implement (named in the message) */
+  LFM3_E_TIMEOUT = -6,     /* a device-side bounded wait gave up (see lfm3_check_device_errors) */
+  LFM3_E_STATE = -7        /* workspace not bound, or the context was used after an error */
+} lfm3_status;
+
+enum { LFM3_LAYER_CONV = 0, LFM3_LAYER_FULL = 1, LFM3_LAYER_SLIDING = 2 };
+enum { LFM3_FFN_BF16 = 0, LFM3_FFN_NVFP4 = 1 };
+#define LFM3_MAX_LAYERS 64
+
+/* Geometry and capacity. The kernels implement d_model 2048, d_ffn 7680, 16 q / 4 kv heads of
+ * 128, 7 conv taps, window 256 and page size 64; other values are refused with
+ * LFM3_E_UNSUPPORTED. n_layers and the layer pattern are free (1..64 layers). */
+typedef struct {
+  int n_layers;
+  int8_t layer_type[LFM3_MAX_LAYERS]; /* LFM3_LAYER_* per layer, in order                 */
+  int d_model, d_ffn, n_q, n_kv, head_dim, conv_taps, window, vocab;
+  float theta_full, theta_sliding; /* rotary bases: full layers, sliding layers           */
+  int rope_pairs_full;             /* rotated (i, i + head_dim/2) pairs on full layers (32) */
+  float eps;                       /* RMSNorm epsilon (1e-5)                              */
+  int has_head;                    /* 1: token ids in, embedding + tied head + argmax out; 0: vectors in/out */
+  int ffn_format;                  /* LFM3_FFN_BF16 or LFM3_FFN_NVFP4                     */
+  int page_size;                   /* positions per KV page (64)                          */
+  int n_pages;                     /* pages in the pool, per full-attention layer         */
+  int max_streams;                 /* slots in the state                                  */
+  int max_pages_per_stream;        /* page-table width; a slot holds at most this x page_size positions */
+  int max_chunk;                   /* rows per prefill pass (1..2048); longer prompts run in chunks */
+  int max_batch;                   /* streams per decode step (1..64)                     */
+} lfm3_config;
+
+/* One layer's weights: device pointers, bf16 unless stated; unused fields may be NULL. */
+typedef struct {
+  const void* op_norm;       /* [d_model] operator_norm gain                              */
+  const void* post_op_norm;  /* [d_model] post_operator_norm gain                         */
+  const void* ffn_norm;      /* [d_model]                                                 */
+  const void* post_ffn_norm; /* [d_model]                                                 */
+  /* conv layers */
+  const void* in_proj;  /* [3*d_model][d_model], output rows B | C | x                    */
+  const void* conv;     /* [d_model][conv_taps], tap conv_taps-1 multiplies the newest column */
+  const void* out_proj; /* [d_model][d_model]                                              */
+  /* attention layers */
+  const void* qkvg;   /* [n_q*hd + 2*n_kv*hd + n_q][d_model]: q rows, k rows, v rows, gate rows */
+  const void* q_norm; /* [head_dim], shared by all q heads                                 */
+  const void* k_norm; /* [head_dim], shared by all k heads                                 */
+  const void* o_proj; /* [d_model][n_q*head_dim]                                           */
+  /* bf16 FFN */
+  const void* w1; /* [d_ffn][d_model] */
+  const void* w3; /* [d_ffn][d_model] */
+  const void* w2; /* [d_model][d_ffn] */
+  /* NVFP4 FFN: E2M1 codes packed two per byte along the input dimension (element 2b in the low
+   * nibble), one E4M3 scale byte per 16 inputs, row-major; w = e2m1 * e4m3 * tensor scale.   */
+  const uint8_t* w1_codes;  /* [d_ffn][d_model/2]  */
+  const uint8_t* w1_scales; /* [d_ffn][d_model/16] */
+  const uint8_t* w3_codes;
+  const uint8_t* w3_scales;
+  const uint8_t* w2_codes;  /* [d_model][d_ffn/2]  */
+  const uint8_t* w2_scales; /* [d_model][d_ffn/16] */
+  float w13_scale;          /* fp32 tensor scale shared by w1 and w3 */
+  float w2_scale;
+} lfm3_layer_weights;
+
+typedef struct {
+  const void* embed;                /* [vocab][d_model] (tied head); NULL when has_head == 0 */
+  const void* final_norm;           /* [d_model] embedding_norm gain; NULL when has_head == 0 */
+  const lfm3_layer_weights* layers; /* HOST array [n_layers], copied by lfm3_create          */
+} lfm3_weights;
+
+/* Decode state, caller-owned device memory (bf16 unless stated). Layouts:
+ *   conv_state  [n_conv][max_streams][conv_taps-1][d_model]   oldest column first
+ *   ring_k/v    [n_sliding][max_streams][n_kv][window][head_dim]   slot = position % window
+ *   kv_k/v      [n_full][n_pages][n_kv][page_size][head_dim]      position p of slot s lives in
+ *               page page_table[s][p / page_size], row p % page_size
+ *   page_table  device int32 [max_streams][max_pages_per_stream] (values in [0, n_pages))
+ *   seq_len     device int32 [max_streams]: tokens already consumed by each slot; the next row
+ *               of a slot sits at position seq_len[slot]
+ *   h_seq_len   HOST int32 [max_streams]: the same values; the library reads it to check
+ *               capacity and updates it when it enqueues work (the device copy is updated by
+ *               the enqueued kernels).
+ *   h_page_table HOST int32 [max_streams][max_pages_per_stream]: mirror used only to check that
+ *               every page a call writes is in range. */
+typedef struct {
+  void* conv_state;
+  void* ring_k;
+  void* ring_v;
+  void* kv_k;
+  void* kv_v;
+  const int32_t* page_table;
+  int32_t* seq_len;
+  int32_t* h_seq_len;
+  const int32_t* h_page_table;
+} lfm3_state;
+
+/* Validates cfg and w (no device access, no launches) and returns the number of workspace
+ * bytes the context needs. On success *out owns a context (free with lfm3_free); on failure
+ * *out is NULL and lfm3_last_error(NULL) names the refusal. */
+lfm3_status lfm3_create(const lfm3_config* cfg, const lfm3_weights* w, size_t* workspace_bytes,
+                        lfm3_ctx** out);
+
+/* Binds caller-owned device workspace (>= the size lfm3_create reported, 256-byte aligned) and
+ * uploads the rotary tables into it (synchronous). Must precede prefill/decode. */
+lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_workspace, size_t bytes);
+
+/* Prompt pass for one slot: consumes n rows at positions h_seq_len[slot] .. +n-1, in chunks
+ * of at most max_chunk rows, updating conv state, ring, pages and seq_len in place.
+ *   d_tokens    device int32 [n] (has_head == 1) or NULL
+ *   d_embeds    device bf16 [n][d_model] input vectors (has_head == 0) or NULL
+ *   d_logits    device fp32 [vocab]: logits of the LAST row (has_head == 1), or NULL
+ *   d_argmax    device int32 [1]: greedy id of the last row, or NULL
+ *   d_hidden    device fp32 [n_layers+1][n][d_model]: the residual stream entering layer 0 and
+ *               leaving every layer (the per-layer parity tap), or NULL
+ * Refuses with LFM3_E_CAPACITY if the slot's pages cannot hold seq_len + n positions. */
+lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slot, const int32_t* d_tokens,
+                         const void* d_embeds, int n, float* d_logits, int32_t* d_argmax,
+                         float* d_hidden, void* stream);
+
+/* One decode step for n_streams distinct slots (one row each, at position seq_len[slot]).
+ *   h_slots     HOST int32 [n_streams] slot ids (checked; must equal d_slots)
+ *   d_slots     device int32 [n_streams]
+ *   d_tokens    device int32 [n_streams] (has_head == 1) or NULL; may alias d_argmax of the
+ *               previous step for a device-resident greedy loop
+ *   d_embeds    device bf16 [n_streams][d_model] (has_head == 0) or NULL
+ *   d_logits    device fp32 [n_streams][vocab] or NULL
+ *   d_argmax    device int32 [n_streams] greedy ids, or NULL
+ *   d_hidden    device fp32 [n_layers+1][n_streams][d_model] or NULL                        */
+lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int n_streams, const int32_t* h_slots,
+                             const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
+                             float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream);
+
+/* Synchronises the stream and reads the device status word that bounded device-side waits set
+ * when they give up. Returns LFM3_OK or LFM3_E_TIMEOUT (and clears the word). */
+lfm3_status lfm3_check_device_errors(lfm3_ctx* ctx, void* stream);
+
+/* Kernel timing for measurement. While enabled, every projection kernel that prefill/decode
+ * enqueue (the weight-streaming GEMVs of decode and the tensor-core GEMMs of prefill) is
+ * bracketed by two CUDA events recorded on the call's stream. Event handles are host objects
+ * created here (up to `capacity` brackets between reads); no device memory is allocated. */
+lfm3_status lfm3_profile_enable(lfm3_ctx* ctx, int on, int capacity);
+
+/* Synchronises on the recorded events and returns, summed over the brackets since the last
+ * read: the number of launches, their device time in ms, their algorithmic bytes (weights +
+ * activations in + results out) and their algorithmic FLOPs (2 * rows * N * K). Clears the
+ * record. Returns LFM3_E_CAPACITY if more brackets were requested than `capacity` (the
+ * excess launches ran unbracketed). */
+lfm3_status lfm3_profile_read(lfm3_ctx* ctx, int* launches, double* ms, double* bytes, double* flops);
+
+/* Number of kernels the last prefill/decode call enqueued. */
+int lfm3_last_launch_count(const lfm3_ctx* ctx);
+
+/* Message for the last error on this context (never NULL; "" after success). With ctx == NULL:
+ * the message of the last failed lfm3_create on the calling thread. */
+const char* lfm3_last_error(const lfm3_ctx* ctx);
+
+/* Frees the host context. Device memory is the caller's and is not touched. */
+void lfm3_free(lfm3_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LFM3_H */

@@ -9,7 +9,9 @@ attention at 3, 7, 11, 15, 19, 21 and the gated short conv everywhere else:
 """
 from __future__ import annotations
 
+import os
 import zlib
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field, replace
 
 import numpy as np
@@ -141,44 +143,57 @@ def nvfp4_draw(seed: int, tag: str, n: int, k: int):
 NVFP4_TENSOR_SCALE = np.float32(2.0 ** -8)
 
 
-def make_weights(geom: Lfm3Geometry, seed: int = 0, ffn: str = "bf16") -> dict:
+def make_weights(geom: Lfm3Geometry, seed: int = 0, ffn: str = "bf16", threads: int | None = None) -> dict:
     """Random-init weights: linear and conv weights N(0, 0.02), norm gains 1 + N(0, 0.02),
-    all rounded to bf16 once. ``ffn='nvfp4'`` draws the FFN (w1, w3, w2) as NVFP4."""
+    all rounded to bf16 once. ``ffn='nvfp4'`` draws the FFN (w1, w3, w2) as NVFP4.
+    Each tensor has its own seeded stream, so tensors are drawn in parallel threads."""
+    if ffn not in ("bf16", "nvfp4"):
+        raise ValueError(ffn)
     D, F, d = geom.d_model, geom.d_ffn, geom.head_dim
     W = {"geometry": geom, "ffn": ffn, "layers": []}
+    jobs = []  # (container, key, callable)
     if geom.has_head:
-        W["embed"] = _normal_bf16(seed, "embed", (geom.vocab, D), 0.02)
-        W["final_norm"] = _normal_bf16(seed, "final_norm", (D,), 0.02, 1.0)
+        jobs.append((W, "embed", lambda: _normal_bf16(seed, "embed", (geom.vocab, D), 0.02)))
+        jobs.append((W, "final_norm", lambda: _normal_bf16(seed, "final_norm", (D,), 0.02, 1.0)))
     for li, kind in enumerate(geom.layer_types):
         p = f"layer{li}."
         L = {"kind": kind}
-        for nm in ("op_norm", "post_op_norm", "ffn_norm", "post_ffn_norm"):
-            L[nm] = _normal_bf16(seed, p + nm, (D,), 0.02, 1.0)
-        if kind == CONV:
-            L["in_proj"] = _normal_bf16(seed, p + "in_proj", (3 * D, D), 0.02)
-            L["conv"] = _normal_bf16(seed, p + "conv", (D, geom.conv_taps), 0.02)
-            L["out_proj"] = _normal_bf16(seed, p + "out_proj", (D, D), 0.02)
-        else:
-            L["q_proj"] = _normal_bf16(seed, p + "q_proj", (geom.n_q * d, D), 0.02)
-            L["k_proj"] = _normal_bf16(seed, p + "k_proj", (geom.n_kv * d, D), 0.02)
-            L["v_proj"] = _normal_bf16(seed, p + "v_proj", (geom.n_kv * d, D), 0.02)
-            L["gate_proj"] = _normal_bf16(seed, p + "gate_proj", (geom.n_q, D), 0.02)
-            L["q_norm"] = _normal_bf16(seed, p + "q_norm", (d,), 0.02, 1.0)
-            L["k_norm"] = _normal_bf16(seed, p + "k_norm", (d,), 0.02, 1.0)
-            L["o_proj"] = _normal_bf16(seed, p + "o_proj", (D, geom.n_q * d), 0.02)
-        if ffn == "bf16":
-            L["w1"] = _normal_bf16(seed, p + "w1", (F, D), 0.02)
-            L["w3"] = _normal_bf16(seed, p + "w3", (F, D), 0.02)
-            L["w2"] = _normal_bf16(seed, p + "w2", (D, F), 0.02)
-        elif ffn == "nvfp4":
-            L["w1_codes"], L["w1_scales"] = nvfp4_draw(seed, p + "w1", F, D)
-            L["w3_codes"], L["w3_scales"] = nvfp4_draw(seed, p + "w3", F, D)
-            L["w13_scale2"] = NVFP4_TENSOR_SCALE
-            L["w2_codes"], L["w2_scales"] = nvfp4_draw(seed, p + "w2", D, F)
-            L["w2_scale2"] = NVFP4_TENSOR_SCALE
-        else:
-            raise ValueError(ffn)
         W["layers"].append(L)
+
+        def normal(key, shape, std, mean=0.0, L=L, p=p):
+            jobs.append((L, key, lambda: _normal_bf16(seed, p + key, shape, std, mean)))
+
+        for nm in ("op_norm", "post_op_norm", "ffn_norm", "post_ffn_norm"):
+            normal(nm, (D,), 0.02, 1.0)
+        if kind == CONV:
+            normal("in_proj", (3 * D, D), 0.02)
+            normal("conv", (D, geom.conv_taps), 0.02)
+            normal("out_proj", (D, D), 0.02)
+        else:
+            normal("q_proj", (geom.n_q * d, D), 0.02)
+            normal("k_proj", (geom.n_kv * d, D), 0.02)
+            normal("v_proj", (geom.n_kv * d, D), 0.02)
+            normal("gate_proj", (geom.n_q, D), 0.02)
+            normal("q_norm", (d,), 0.02, 1.0)
+            normal("k_norm", (d,), 0.02, 1.0)
+            normal("o_proj", (D, geom.n_q * d), 0.02)
+        if ffn == "bf16":
+            normal("w1", (F, D), 0.02)
+            normal("w3", (F, D), 0.02)
+            normal("w2", (D, F), 0.02)
+        else:
+            for nm, (n, k) in (("w1", (F, D)), ("w3", (F, D)), ("w2", (D, F))):
+                jobs.append((L, nm, lambda nm=nm, n=n, k=k, p=p: nvfp4_draw(seed, p + nm, n, k)))
+            L["w13_scale2"] = NVFP4_TENSOR_SCALE
+            L["w2_scale2"] = NVFP4_TENSOR_SCALE
+    workers = threads or min(16, os.cpu_count() or 1)
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        results = list(ex.map(lambda j: j[2](), jobs))
+    for (box, key, _), val in zip(jobs, results):
+        if isinstance(val, tuple):
+            box[key + "_codes"], box[key + "_scales"] = val
+        else:
+            box[key] = val
     return W
 
 

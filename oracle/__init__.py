@@ -7,7 +7,8 @@ CUDA path in ``attention_decoder_b200`` shares no code with it; the two meet
 only through the seeded generators in ``lfm3_inputs``.
 
 It is plain NumPy in float64 (fp32 optional for long timing runs), written
-from the method's definition:
+from the method's definition, optionally with the bf16 activation boundaries
+the pages fix (``bf16=True``; see lfm3.py):
 
 * ``lfm3.py`` - RMSNorm, the gated 7-tap short conv and its state, partial /
   full rotary, full and sliding-window GQA attention with the per-head sigmoid
@@ -22,5 +23,5 @@ brute force, closed forms, invariants and the pages' own totals). The one
 thing the pages give no worked numbers for - whole-model values - is
 "parity unpinned" beyond those invariants and brute-force pins.
 """
-from .lfm3 import Lfm3Oracle, OracleState, rms_norm, rope_inv_freq, apply_rope  # noqa: F401
+from .lfm3 import Lfm3Oracle, OracleState, rms_norm, rope_inv_freq, apply_rope, round_bf16  # noqa: F401
 from .nvfp4 import e2m1_value, e4m3_value, nvfp4_dequant  # noqa: F401

@@ -22,6 +22,16 @@ Sources (coreai-model-zoo note "lfm3-1.7b-port" unless stated):
 * chunked-prefill / pad-tail paragraphs - the new conv state is columns
   [n, n+6) of [state | Bx] for a chunk of n rows.
 
+Precision. TensorFold issue #1491 ("Goal and current state") keeps "BF16 activation
+boundaries, and FP32 reductions", and PR #1508 ("Verification") checks the engine against a
+float64 reference with "the engine's bf16 rounding points" added. With ``bf16=True`` this
+oracle does the same: arithmetic stays float64, and a value is rounded to bf16 exactly where it
+becomes a stored operand of a matrix product or attention, or persistent state - the normed
+inputs of every projection (and of the head), Bx (the conv state), y = C * conv, q and k after
+norm and rotary, v, the gated attention output and the SwiGLU product. Projection accumulators,
+gate logits, norms, softmax and the residual stream are reductions and stay unrounded. With
+``bf16=False`` (default) nothing is rounded: the plain float64 definition.
+
 Readings where the pages are silent (each also listed in the design doc):
 in_proj rows are B, C, x in that order; the conv is causal with tap 6 on the
 current column and zero history at sequence start; no biases; q/k RMSNorm
@@ -44,6 +54,13 @@ from .nvfp4 import nvfp4_block_values
 def _bf16(bits) -> np.ndarray:
     """bf16 bit patterns -> float32 (exact)."""
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def round_bf16(x):
+    """Nearest bf16 value (8 significant bits, ties to even) of each float, as float64."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                 # x = m * 2^e, |m| in [0.5, 1)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
 
 
 def rms_norm(x, g, eps):
@@ -122,9 +139,10 @@ class OracleState:
 class Lfm3Oracle:
     """Forward of one decoder on seeded weights from ``lfm3_inputs.make_weights``."""
 
-    def __init__(self, weights: dict, dtype=np.float64, gate=True, rope_all_dims=False, window=True):
+    def __init__(self, weights: dict, dtype=np.float64, gate=True, rope_all_dims=False, window=True, bf16=False):
         self.g = weights["geometry"]
         self.dtype = dtype
+        self._rb = round_bf16 if bf16 else (lambda x: x)
         # negative controls (planted mistakes for the tests): drop the gate, rotate every
         # dimension on full layers, remove the window
         self.use_gate = gate
@@ -174,13 +192,15 @@ class Lfm3Oracle:
         return x @ w.T.astype(self.dtype, copy=False)
 
     def _ffn(self, hn, O):
+        hn = self._rb(hn)
         a = O["s13"] * self._lin(hn, O["w1"])
         b = O["s13"] * self._lin(hn, O["w3"])
-        u = silu(a) * b
+        u = self._rb(silu(a) * b)
         return O["s2"] * self._lin(u, O["w2"])
 
     def _qkvg(self, xn, O):
         g = self.g
+        xn = self._rb(xn)
         T = xn.shape[0]
         q = self._lin(xn, O["q_proj"]).reshape(T, g.n_q, g.head_dim)
         k = self._lin(xn, O["k_proj"]).reshape(T, g.n_kv, g.head_dim)
@@ -188,7 +208,7 @@ class Lfm3Oracle:
         gate = self._lin(xn, O["gate_proj"])                       # [T, n_q]
         q = rms_norm(q, O["q_norm"], g.eps)
         k = rms_norm(k, O["k_norm"], g.eps)
-        return q, k, v, gate
+        return q, k, self._rb(v), gate
 
     def _attend(self, q, qpos, k, v, kpos, window, gate):
         """Softmax attention of queries q[Tq, Hq, d] at qpos over keys k/v[Tk, Hkv, d] at
@@ -212,7 +232,7 @@ class Lfm3Oracle:
             o[:, h, :] = p @ v[:, kvh, :]
         if self.use_gate:
             o = o * sigmoid(gate)[:, :, None]
-        return o.reshape(q.shape[0], -1)
+        return self._rb(o.reshape(q.shape[0], -1))
 
     def _window(self, kind):
         return self.g.window if (kind == SLIDING and self.use_window) else None
@@ -223,15 +243,15 @@ class Lfm3Oracle:
         """Whole sequence from zero history: z[t] = sum over lags l = 0..taps-1 of
         w[:, taps-1-l] * bx[t-l], with bx[t<0] = 0."""
         D = self.g.d_model
-        bcx = self._lin(xn, O["in_proj"])
+        bcx = self._lin(self._rb(xn), O["in_proj"])
         b, c, xc = bcx[:, :D], bcx[:, D:2 * D], bcx[:, 2 * D:]
-        z = causal_conv_full(b * xc, O["conv"])
-        return self._lin(c * z, O["out_proj"])
+        z = causal_conv_full(self._rb(b * xc), O["conv"])
+        return self._lin(self._rb(c * z), O["out_proj"])
 
     def _attn_full(self, xn, O, pos, kind):
         q, k, v, gate = self._qkvg(xn, O)
-        q = apply_rope(q, pos, self.inv_freq[kind])
-        k = apply_rope(k, pos, self.inv_freq[kind])
+        q = self._rb(apply_rope(q, pos, self.inv_freq[kind]))
+        k = self._rb(apply_rope(k, pos, self.inv_freq[kind]))
         o = self._attend(q, pos, k, v, pos, self._window(kind), gate)
         return self._lin(o, O["o_proj"])
 
@@ -248,7 +268,7 @@ class Lfm3Oracle:
         return self.embed[np.asarray(tokens)].astype(self.dtype)
 
     def logits(self, x):
-        xn = rms_norm(x, self.final_norm, self.g.eps)
+        xn = self._rb(rms_norm(x, self.final_norm, self.g.eps))
         return xn @ self.embed.T.astype(self.dtype, copy=False)
 
     def forward_full(self, tokens=None, x0=None, logits="last"):
@@ -314,16 +334,16 @@ class Lfm3Oracle:
         """Chunk of n rows over the carried columns: win = [state | bx],
         z[t] = sum_k w[:, k] * win[t + k]; the new state is win[n : n + taps - 1]."""
         D = self.g.d_model
-        bcx = self._lin(xn, O["in_proj"])
+        bcx = self._lin(self._rb(xn), O["in_proj"])
         b, c, xc = bcx[:, :D], bcx[:, D:2 * D], bcx[:, 2 * D:]
-        z, st.conv[j] = causal_conv_chunk(st.conv[j], b * xc, O["conv"])
-        return self._lin(c * z, O["out_proj"])
+        z, st.conv[j] = causal_conv_chunk(st.conv[j], self._rb(b * xc), O["conv"])
+        return self._lin(self._rb(c * z), O["out_proj"])
 
     def _attn_chunk(self, xn, O, kind, st, j, pos):
         g = self.g
         q, k, v, gate = self._qkvg(xn, O)
-        q = apply_rope(q, pos, self.inv_freq[kind])
-        k = apply_rope(k, pos, self.inv_freq[kind])
+        q = self._rb(apply_rope(q, pos, self.inv_freq[kind]))
+        k = self._rb(apply_rope(k, pos, self.inv_freq[kind]))
         if kind == FULL:
             st.full_k[j] = np.concatenate([st.full_k[j], k], axis=0)
             st.full_v[j] = np.concatenate([st.full_v[j], v], axis=0)

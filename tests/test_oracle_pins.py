@@ -410,3 +410,38 @@ def test_sandwich_norm_structure():
     W4["layers"][0]["post_op_norm"] = bf16_bits(np.ones(g.d_model, np.float32))
     d = Lfm3Oracle(W4).forward_full(x0=x)["hidden"][-1] - x
     assert np.allclose(np.sqrt(np.mean(d * d, axis=1)), 1.0, rtol=1e-3)
+
+
+# ---------------------------------------------------------------- bf16 activation boundaries
+
+def test_round_bf16_against_torch_and_ties():
+    from oracle import round_bf16
+    r = np.random.default_rng(13)
+    x = (r.standard_normal(10000) * np.exp(r.uniform(-20, 20, 10000))).astype(np.float32).astype(np.float64)
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(round_bf16(x), ref)
+    # idempotent, exact on bf16 values, ties to even (1 + 2^-8 lies halfway between 1 and 1 + 2^-7)
+    assert np.array_equal(round_bf16(ref), ref)
+    assert round_bf16(1.0 + 2.0 ** -8) == 1.0
+    assert round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert round_bf16(-(1.0 + 2.0 ** -8 + 2.0 ** -30)) == -(1.0 + 2.0 ** -7)
+
+
+def test_bf16_boundary_mode_keeps_the_invariants_and_stores_bf16_state():
+    from oracle import round_bf16
+    g = tiny_geometry()
+    W = make_weights(g, 0)
+    tok = np.arange(21) * 5 % g.vocab
+    o = Lfm3Oracle(W, bf16=True)
+    full = o.forward_full(tokens=tok, logits="all")
+    st = o.new_state()
+    parts = [o.forward_chunk(st, tokens=tok[:9], logits="all")] + \
+            [o.forward_chunk(st, tokens=tok[t:t + 1], logits="all") for t in range(9, 21)]
+    assert np.allclose(np.concatenate([p["logits"] for p in parts]), full["logits"], rtol=1e-10, atol=1e-10)
+    # the carried conv columns and the cached keys/values are bf16 values
+    for a in st.conv + st.full_k + st.full_v + st.ring_k + st.ring_v:
+        assert np.array_equal(round_bf16(a), a)
+    # close to the unrounded definition, but not equal to it
+    exact = Lfm3Oracle(W).forward_full(tokens=tok, logits="all")
+    d = np.abs(full["hidden"][-1] - exact["hidden"][-1]).max() / np.abs(exact["hidden"][-1]).max()
+    assert 1e-5 < d < 5e-2
