@@ -16,7 +16,8 @@ STATUS = {0: "LFM3_OK", -1: "LFM3_E_ARG", -2: "LFM3_E_CONFIG", -3: "LFM3_E_CAPAC
           -5: "LFM3_E_UNSUPPORTED", -6: "LFM3_E_TIMEOUT", -7: "LFM3_E_STATE"}
 
 # exported entry points (every one declared in include/lfm3.h)
-SYMBOLS = ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_decode_step", "lfm3_check_device_errors",
+SYMBOLS = ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_decode_step", "lfm3_decode_step_noalloc",
+           "lfm3_check_device_errors",
            "lfm3_profile_enable", "lfm3_profile_read", "lfm3_last_launch_count", "lfm3_last_error", "lfm3_free")
 
 
@@ -63,6 +64,7 @@ def lib():
     L.lfm3_bind_workspace.argtypes = [vp, vp, C.c_size_t]
     L.lfm3_prefill.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, vp, vp, C.c_int, vp, vp, vp, vp]
     L.lfm3_decode_step.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, i32p, vp, vp, vp, vp, vp, vp, vp]
+    L.lfm3_decode_step_noalloc.argtypes = L.lfm3_decode_step.argtypes
     L.lfm3_check_device_errors.argtypes = [vp, vp]
     L.lfm3_profile_enable.argtypes = [vp, C.c_int, C.c_int]
     dp = C.POINTER(C.c_double)
@@ -72,7 +74,7 @@ def lib():
     L.lfm3_last_error.restype = C.c_char_p
     L.lfm3_free.argtypes = [vp]
     L.lfm3_free.restype = None
-    for name in ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_decode_step",
+    for name in ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_decode_step", "lfm3_decode_step_noalloc",
                  "lfm3_check_device_errors", "lfm3_profile_enable", "lfm3_profile_read", "lfm3_last_launch_count"):
         getattr(L, name).restype = C.c_int
     _lib = L
@@ -108,6 +110,12 @@ def lfm3_prefill(ctx, st, slot, d_tokens, d_embeds, n, d_logits, d_argmax, d_hid
 def lfm3_decode_step(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden, stream):
     return lib().lfm3_decode_step(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax,
                                   d_hidden, stream)
+
+
+def lfm3_decode_step_noalloc(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                             stream):
+    return lib().lfm3_decode_step_noalloc(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits,
+                                          d_argmax, d_hidden, stream)
 
 
 def lfm3_check_device_errors(ctx, stream):

@@ -12,6 +12,8 @@
 //
 // Prefill: flash attention on the tensor cores (m16n8k16), one block per (32 query rows, kv
 // head): 8 warps = 4 heads x 2 row groups share every K/V tile staged in shared memory.
+#include <mutex>
+
 #include "kernels.cuh"
 
 namespace lfm3 {
@@ -132,6 +134,32 @@ __global__ void __launch_bounds__(128) k_attn_merge(const float* __restrict__ pa
   }
   const float gt = sigmoidf_(gate[b * HQ + h]);
   y[(size_t)b * HQ * HD + h * HD + d] = f2bf(gt * (o / l));
+}
+
+// Fixed scratch for callers that cannot allocate device memory (lfm3_decode_step_noalloc): 4 MiB
+// of split-KV partials, one copy per GPU that loads the library, kept until the process exits.
+// Host code never names the array directly: the symbol is a host-side stand-in, so its device
+// address is looked up once per device (with that device current) and passed to the kernels.
+constexpr size_t ATTN_STATIC_FLOATS = (size_t(4) << 20) / sizeof(float);
+static __device__ __align__(256) float g_attn_static[ATTN_STATIC_FLOATS];
+
+cudaError_t attn_static_scratch(float** ptr, size_t* nfloats) {
+  static std::mutex mu;
+  static float* addr[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_attn_static);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<float*>(p);
+  }
+  *ptr = addr[dev];
+  *nfloats = ATTN_STATIC_FLOATS;
+  return cudaSuccess;
 }
 
 cudaError_t attn_decode(const bf16* q, Rows rows, AttnLayer L, int splits, float* part, const float* gate, bf16* y,

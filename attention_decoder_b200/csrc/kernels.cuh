@@ -114,6 +114,8 @@ cudaError_t attn_decode(const bf16* q, Rows rows, AttnLayer L, int splits, float
 // Prefill attention for the n rows of one slot starting at position p0.
 //  full: keys through the page table; sliding: keys in scratch [HKV][scratch_rows][HD], index i <-> p0-WIN+i
 cudaError_t attn_init();
+// Device address and size (floats) of the library's fixed attention scratch on the current device.
+cudaError_t attn_static_scratch(float** ptr, size_t* nfloats);
 cudaError_t attn_prefill(const bf16* q, int n, int p0, int slot, AttnLayer L, const bf16* sk, const bf16* sv,
                          int scratch_rows, const float* gate, bf16* y, cudaStream_t s);
 

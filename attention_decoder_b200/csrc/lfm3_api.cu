@@ -535,7 +535,7 @@ namespace {
 // Every launch of one decode step, in order, on stream s.
 lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* d_slots,
                            const int32_t* d_tokens, const void* d_embeds, float* d_logits, int32_t* d_argmax,
-                           float* d_hidden, int splits_full, cudaStream_t s) {
+                           float* d_hidden, int splits_full, float* attn_part, cudaStream_t s) {
   const lfm3_config& g = ctx->cfg;
   const float eps = g.eps;
   const bool gv = nb <= GEMV_MAX_ROWS;
@@ -591,8 +591,8 @@ lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const in
       const int k = full ? 0 : 1;
       CK(qk_norm_rope_kv(ctx->part, nq, qstride, B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], rows,
                          eps, ctx->q, ctx->gate, kw, s));
-      CK(attn_decode(ctx->q, rows, attn_layer(ctx, st, l, v), full ? splits_full : WIN / 64, ctx->attn_part,
-                     ctx->gate, ctx->y, s));
+      CK(attn_decode(ctx->q, rows, attn_layer(ctx, st, l, v), full ? splits_full : WIN / 64, attn_part, ctx->gate,
+                     ctx->y, s));
       if (gv) {
         GemvArgs o{};
         o.w = B(W.o_proj); o.x = ctx->y; o.K = HQ * HD; o.N = D; o.rows = nb; o.splits = SPLIT_DD; o.part = ctx->part;
@@ -656,10 +656,13 @@ lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const in
 
 }  // namespace
 
-extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* h_slots,
-                                        const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
-                                        float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream) {
-  if (!ctx) return LFM3_E_ARG;
+namespace {
+
+// Host checks of a decode step and its full-layer split count (quantised to a power of two so
+// that one captured graph serves a range of contexts).
+lfm3_status validate_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* h_slots,
+                            const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
+                            const float* d_logits, const int32_t* d_argmax, int* splits_out) {
   if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
   const lfm3_config& g = ctx->cfg;
   lfm3_status vs = check_state(ctx, st);
@@ -679,16 +682,27 @@ extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int
     if (vs != LFM3_OK) return vs;
     maxpos = std::max(maxpos, (int)st->h_seq_len[s]);
   }
-
-  // full-layer split count, quantised to a power of two so that one graph serves a range of contexts
   int splits_full = 1;
   while (splits_full < maxpos / 256 + 1) splits_full *= 2;
-  splits_full = std::min(splits_full, ctx->max_splits);
+  *splits_out = std::min(splits_full, ctx->max_splits);
+  return LFM3_OK;
+}
+
+}  // namespace
+
+extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* h_slots,
+                                        const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
+                                        float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  int splits_full = 1;
+  lfm3_status vs = validate_decode(ctx, st, nb, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax,
+                                   &splits_full);
+  if (vs != LFM3_OK) return vs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   g_launches = 0;
   if (!ctx->graphs_on || ctx->prof) {
     lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
-                                    splits_full, s);
+                                    splits_full, ctx->attn_part, s);
     if (es != LFM3_OK) return es;
     ctx->launches = g_launches;
   } else {
@@ -708,7 +722,7 @@ extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int
       cudaGraph_t graph = nullptr;
       CK(cudaStreamBeginCapture(ctx->cap_stream, cudaStreamCaptureModeThreadLocal));
       lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
-                                      splits_full, ctx->cap_stream);
+                                      splits_full, ctx->attn_part, ctx->cap_stream);
       cudaError_t ce = cudaStreamEndCapture(ctx->cap_stream, &graph);
       if (es != LFM3_OK) {
         if (graph) cudaGraphDestroy(graph);
@@ -725,6 +739,37 @@ extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int
     CK(cudaGraphLaunch(hit->exec, s));
     ctx->launches = hit->launches;
   }
+  for (int b = 0; b < nb; ++b) st->h_seq_len[h_slots[b]] += 1;
+  return LFM3_OK;
+}
+
+// A decode step that allocates nothing: the split-KV attention keeps its per-split partial
+// results in the library's own fixed device array (see attn_static_scratch) instead of the
+// bound workspace, and the step is launched directly rather than through a captured graph.
+extern "C" lfm3_status lfm3_decode_step_noalloc(lfm3_ctx* ctx, const lfm3_state* st, int nb,
+                                                const int32_t* h_slots, const int32_t* d_slots,
+                                                const int32_t* d_tokens, const void* d_embeds, float* d_logits,
+                                                int32_t* d_argmax, float* d_hidden, void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  int splits_full = 1;
+  lfm3_status vs = validate_decode(ctx, st, nb, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax,
+                                   &splits_full);
+  if (vs != LFM3_OK) return vs;
+  float* scratch = nullptr;
+  size_t cap = 0;
+  CK(attn_static_scratch(&scratch, &cap));
+  const size_t need = (size_t)nb * HQ * std::max(splits_full, WIN / 64) * (HD + 2);
+  if (need > cap)
+    return fail(ctx, LFM3_E_CAPACITY,
+                "lfm3_decode_step_noalloc: %d streams x %d key splits need %zu bytes of attention scratch, more "
+                "than the fixed %zu bytes",
+                nb, splits_full, need * sizeof(float), cap * sizeof(float));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  g_launches = 0;
+  lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                                  splits_full, scratch, s);
+  if (es != LFM3_OK) return es;
+  ctx->launches = g_launches;
   for (int b = 0; b < nb; ++b) st->h_seq_len[h_slots[b]] += 1;
   return LFM3_OK;
 }

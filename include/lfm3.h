@@ -171,6 +171,28 @@ lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int n_streams,
                              const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
                              float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream);
 
+/* The same decode step as lfm3_decode_step, for callers that cannot allocate device memory at
+ * the point of the call - a host program that hands this library a finished arena and forbids
+ * later allocation, or code running where an allocation would synchronise the device. The
+ * pages have no counterpart: it is a service of this library, not part of the method.
+ *   Arguments, checks, state updates and results are those of lfm3_decode_step (a context with
+ *   a bound workspace is still required). The difference: the attention's per-split partial
+ *   results go to a fixed 4 MiB array inside the library's own device image instead of the
+ *   workspace, and the step is launched kernel by kernel (no captured graph).
+ *   Limit: n_streams x 16 heads x splits x 130 floats must fit in the 4 MiB, where splits is
+ *   max(4, the smallest power of two >= (longest context / 256) + 1); larger calls are refused
+ *   with LFM3_E_CAPACITY and a message giving both sizes. One stream fits up to 126 splits
+ *   (the whole 32k context); 64 streams fit 7 (contexts below 1792).
+ *   Nothing in the array has to start at zero: every call writes all the partials it reads.
+ *   The array is one per GPU for the whole process and every call shares it, so calls that can
+ *   overlap on the GPU (different streams, different contexts) race on it; serialise them.
+ *   The first call on each device looks the array's address up (cudaGetSymbolAddress) with that
+ *   device current; make that first call before any stream capture. No device memory is
+ *   allocated or freed by this call. */
+lfm3_status lfm3_decode_step_noalloc(lfm3_ctx* ctx, const lfm3_state* st, int n_streams, const int32_t* h_slots,
+                                     const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
+                                     float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream);
+
 /* Synchronises the stream and reads the device status word that bounded device-side waits set
  * when they give up. Returns LFM3_OK or LFM3_E_TIMEOUT (and clears the word). */
 lfm3_status lfm3_check_device_errors(lfm3_ctx* ctx, void* stream);
