@@ -75,3 +75,38 @@ DEVI void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32
 
 DEVI float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
 DEVI float siluf_(float x) { return x / (1.f + __expf(-x)); }
+
+// ---------------------------------------------------------------- mbarriers and bulk copies
+constexpr uint32_t WAIT_LIMIT = 1u << 22;  // try_wait rounds before a wait gives up
+
+DEVI uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+DEVI void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+DEVI void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+DEVI void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+DEVI bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait: returns false (and sets *err) if the phase did not complete in time.
+DEVI bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+  for (uint32_t i = 0; i < WAIT_LIMIT; ++i)
+    if (mbar_try(bar, parity)) return true;
+  atomicExch(err, 1);
+  return false;
+}
+// One contiguous global -> shared copy (16-byte aligned, size a multiple of 16) that completes
+// `bytes` of the barrier's transaction count.
+DEVI void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}

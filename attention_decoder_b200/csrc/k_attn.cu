@@ -5,9 +5,10 @@
 // p - k < 256. Scores are q.k / sqrt(128), softmax in fp32, and the per-head gate sigmoid(g_h)
 // multiplies each head's output before o_proj (fused into the epilogues here).
 //
-// Decode: split-KV. Block (split, kv head, stream) scores its key range for the 4 query heads
-// of the group, writes unnormalised (max, sum, o) partials; the merge kernel combines splits,
-// applies the gate and writes bf16 o. Full layers read keys through the page table (64
+// Decode: split-KV. Block (split, kv head, stream) stages its key range (up to 128 keys) of K and
+// V in shared memory with asynchronous copies, scores it for the 4 query heads of the group and
+// writes unnormalised (max, sum, o) partials; the merge kernel combines splits, applies the gate
+// and writes bf16 o. Full layers read keys through the page table (64
 // positions per page); sliding layers read the 256-slot ring (slot = position % 256).
 //
 // Prefill: flash attention on the tensor cores (m16n8k16), one block per (32 query rows, kv
@@ -18,11 +19,19 @@
 
 namespace lfm3 {
 
-constexpr int DEC_SPLIT = 256;     // keys per split on full layers
-constexpr int DEC_SPLIT_RING = 64; // ring slots per split on sliding layers
+constexpr int DEC_SPLIT = DEC_KEYS_FULL;       // two 64-position pages
+constexpr int DEC_SPLIT_RING = DEC_KEYS_RING;
+constexpr int DEC_SMEM = 2 * DEC_SPLIT * HD * 2;  // K and V tiles, bf16
+
+// 16-byte chunk c of key row r in a K tile: rotated by the row so that one key per thread reads
+// distinct banks.
+DEVI int krot(int r, int c) { return r * HD + ((c + r) & 15) * 8; }
 
 __global__ void __launch_bounds__(128) k_attn_decode(const bf16* __restrict__ q, Rows rows, AttnLayer L, int splits,
                                                      float* __restrict__ part) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  bf16* ks = reinterpret_cast<bf16*>(dsm);
+  bf16* vs = ks + DEC_SPLIT * HD;
   __shared__ float qs[GQA][HD];
   __shared__ float sc[GQA][DEC_SPLIT];
   __shared__ float ored[2][GQA][HD];
@@ -34,33 +43,42 @@ __global__ void __launch_bounds__(128) k_attn_decode(const bf16* __restrict__ q,
   const int slot = rows.slot[b], pos = rows.pos[b];
   const int span = L.full ? DEC_SPLIT : DEC_SPLIT_RING;
   const int nkeys = L.full ? pos + 1 : min(pos + 1, WIN);  // ring: slots 0..nkeys-1 are live
-  const int j0 = sp * span, j1 = min(nkeys, j0 + span);
-  const float scale = rsqrtf((float)HD);
+  const int j0 = sp * span, j1 = min(nkeys, j0 + span), cnt = j1 - j0;
   float* out = part + (((size_t)b * HQ + kvh * GQA) * splits + sp) * (HD + 2);
-  if (j0 >= j1) {  // empty split
+  if (cnt <= 0) {  // empty split
     for (int e = tid; e < GQA * (HD + 2); e += blockDim.x) {
       const int h = e / (HD + 2), k = e % (HD + 2);
       out[(size_t)h * splits * (HD + 2) + k] = (k == HD) ? -INFINITY : 0.f;
     }
     return;
   }
-  for (int e = tid; e < GQA * HD; e += blockDim.x)
-    qs[e / HD][e % HD] = bf2f(q[((size_t)b * HQ + kvh * GQA + e / HD) * HD + e % HD]) * scale;
-  __syncthreads();
-  auto krow = [&](const bf16* base, int j) -> const bf16* {
+  // stage the split's keys and values: cnt rows x 16 chunks of 16 B each, all in flight at once
+  auto row_ptr = [&](const bf16* base, int j) -> const bf16* {
     if (L.full) {
       const int page = L.page_table[(size_t)slot * L.max_pages + j / PAGE];
       return base + (((size_t)page * HKV + kvh) * PAGE + j % PAGE) * HD;
     }
     return base + (((size_t)slot * HKV + kvh) * WIN + j) * HD;
   };
-  // scores: one key per thread
-  for (int j = j0 + tid; j < j1; j += blockDim.x) {
-    const bf16* kp = krow(L.k, j);
+  for (int e = tid; e < cnt * 16; e += blockDim.x) {
+    const int r = e >> 4, c = e & 15;
+    const uint32_t kd = (uint32_t)__cvta_generic_to_shared(ks + krot(r, c));
+    const uint32_t vd = (uint32_t)__cvta_generic_to_shared(vs + r * HD + c * 8);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(kd), "l"(row_ptr(L.k, j0 + r) + c * 8));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vd), "l"(row_ptr(L.v, j0 + r) + c * 8));
+  }
+  asm volatile("cp.async.commit_group;");
+  const float scale = rsqrtf((float)HD);
+  for (int e = tid; e < GQA * HD; e += blockDim.x)
+    qs[e / HD][e % HD] = bf2f(q[((size_t)b * HQ + kvh * GQA + e / HD) * HD + e % HD]) * scale;
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  // scores: one key per thread (span <= 128)
+  if (tid < cnt) {
     float s[GQA] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
-    for (int c = 0; c < HD / 8; ++c) {
-      const uint4 w = ldg16(kp + c * 8);
+    for (int c = 0; c < 16; ++c) {
+      const uint4 w = *reinterpret_cast<const uint4*>(ks + krot(tid, c));
       const float kv[8] = {bflo(w.x), bfhi(w.x), bflo(w.y), bfhi(w.y), bflo(w.z), bfhi(w.z), bflo(w.w), bfhi(w.w)};
 #pragma unroll
       for (int h = 0; h < GQA; ++h)
@@ -68,12 +86,11 @@ __global__ void __launch_bounds__(128) k_attn_decode(const bf16* __restrict__ q,
         for (int e = 0; e < 8; ++e) s[h] += qs[h][c * 8 + e] * kv[e];
     }
 #pragma unroll
-    for (int h = 0; h < GQA; ++h) sc[h][j - j0] = s[h];
+    for (int h = 0; h < GQA; ++h) sc[h][tid] = s[h];
   }
   __syncthreads();
-  // softmax pieces: warp h owns head h
   {
-    const int h = warp, cnt = j1 - j0;
+    const int h = warp;
     float m = -INFINITY;
     for (int j = lane; j < cnt; j += 32) m = fmaxf(m, sc[h][j]);
     m = warp_max(m);
@@ -87,16 +104,16 @@ __global__ void __launch_bounds__(128) k_attn_decode(const bf16* __restrict__ q,
     if (lane == 0) { ml[h][0] = m; ml[h][1] = l; }
   }
   __syncthreads();
-  // o = sum_j p_j v_j: thread = (key parity, dim pair)
   {
     const int par = tid >> 6, dp = (tid & 63) * 2;
     float o[GQA][2] = {};
-    for (int j = j0 + par; j < j1; j += 2) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(krow(L.v, j) + dp);
+#pragma unroll 4
+    for (int j = par; j < cnt; j += 2) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(vs + j * HD + dp);
       const float v0 = bflo(w), v1 = bfhi(w);
 #pragma unroll
       for (int h = 0; h < GQA; ++h) {
-        const float p = sc[h][j - j0];
+        const float p = sc[h][j];
         o[h][0] += p * v0;
         o[h][1] += p * v1;
       }
@@ -164,7 +181,7 @@ cudaError_t attn_static_scratch(float** ptr, size_t* nfloats) {
 
 cudaError_t attn_decode(const bf16* q, Rows rows, AttnLayer L, int splits, float* part, const float* gate, bf16* y,
                         cudaStream_t s) {
-  cudaError_t e = launch(k_attn_decode, dim3(splits, HKV, rows.n), dim3(128), 0, s, q, rows, L, splits, part);
+  cudaError_t e = launch(k_attn_decode, dim3(splits, HKV, rows.n), dim3(128), DEC_SMEM, s, q, rows, L, splits, part);
   if (e != cudaSuccess) return e;
   return launch(k_attn_merge, dim3(rows.n, HQ), dim3(HD), 0, s, part, splits, gate, y);
 }
@@ -395,6 +412,8 @@ cudaError_t attn_prefill(const bf16* q, int n, int p0, int slot, AttnLayer L, co
 }
 
 cudaError_t attn_init() {
+  cudaError_t e = cudaFuncSetAttribute(k_attn_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM);
+  if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(k_attn_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, 4 * PA_TILE_BYTES);
 }
 

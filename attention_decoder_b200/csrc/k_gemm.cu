@@ -1,26 +1,28 @@
 // Prefill projections on the 5th-generation tensor cores: C[M][N] = alpha * A[M][K] . W[N][K]^T
 // with A the bf16 activations of a prompt chunk and W a bf16 weight, both K-major.
 //
-// One block per 128 x BN output tile (BN = 128 or 256), 6 warps:
+// Persistent blocks (one per SM, 6 warps) walk 128 x BN output tiles (BN = 128 or 256):
 //   warp 0      TMA producer: 128x64 A box and BNx64 W box per stage (128-byte swizzle), into a
-//               4-stage ring guarded by full/empty mbarriers;
-//   warp 1      allocates BN TMEM columns; one elected lane issues tcgen05.mma (kind::f16,
-//               M=128, N=BN, K=16 per instruction, fp32 accumulate in TMEM) and commits each
-//               stage back to the producer, then the finished accumulator to the epilogue;
+//               4- or 6-stage ring guarded by full/empty mbarriers;
+//   warp 1      allocates 2 x BN TMEM columns (two accumulators); one elected lane issues
+//               tcgen05.mma (kind::f16, M=128, N=BN, K=16 per instruction, fp32 accumulate in TMEM),
+//               commits each stage back to the producer and each finished accumulator to the
+//               epilogue, and moves on to the next tile in the other accumulator;
 //   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time (warp w reads TMEM lanes
-//               32*(w%4) ..), apply the fused epilogue, store to global.
+//               32*(w%4) ..), apply the fused epilogue, store, release the accumulator.
 // Epilogues: fp32 out, bf16 out, and SwiGLU (the tile's 256 columns are 128 rows of w1 and the
 // same 128 rows of w3: u = silu(alpha a) * (alpha b), bf16).
 // Every mbarrier wait is bounded; a wait that gives up sets the device error word and the
 // block runs to completion without further MMAs so that TMEM is always released.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace lfm3 {
 
-constexpr int GM_BM = 128, GM_BK = 64, GM_STAGES = 4;
-constexpr uint32_t WAIT_LIMIT = 1u << 22;
+constexpr int GM_BM = 128, GM_BK = 64;
 
 static PFN_cuTensorMapEncodeTiled_v12000 p_encode = nullptr;
 
@@ -49,28 +51,6 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
 }
 
 // ---------------------------------------------------------------- PTX wrappers
-DEVI uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-DEVI void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-DEVI void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-DEVI bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-  return ok != 0;
-}
-// Bounded wait: returns false (and sets *err) if the phase did not complete in time.
-DEVI bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
-  for (uint32_t i = 0; i < WAIT_LIMIT; ++i)
-    if (mbar_try(bar, parity)) return true;
-  atomicExch(err, 1);
-  return false;
-}
 DEVI void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
@@ -120,36 +100,52 @@ struct GemmArgs {
   int* err;
 };
 
+template <int BN>
+struct GemmGeom {
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr uint32_t A_BYTES = GM_BM * GM_BK * 2;
+  static constexpr uint32_t B_BYTES = BN * GM_BK * 2;
+  static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+};
+
+// Persistent: block b takes tiles b, b + gridDim.x, ... (M tiles fastest, so consecutive blocks
+// share a weight tile through L2). TMEM holds two BN-column accumulators: the MMA thread fills
+// one while the epilogue warps drain the other (acc_full / acc_empty barriers).
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtensorMap ta,
                                                  const __grid_constant__ CUtensorMap tb,
                                                  const __grid_constant__ CUtensorMap tb3, const GemmArgs g) {
-  constexpr uint32_t A_BYTES = GM_BM * GM_BK * 2;
-  constexpr uint32_t B_BYTES = BN * GM_BK * 2;
-  constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+  using G = GemmGeom<BN>;
+  constexpr int S = G::STAGES;
+  constexpr int NOUT = EPI == GEMM_SWIGLU ? BN / 2 : BN;  // output columns per tile
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + GM_STAGES * STAGE);
-  const uint32_t full0 = su32(bars), empty0 = su32(bars + GM_STAGES), accf = su32(bars + 2 * GM_STAGES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * GM_STAGES + 1);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * G::STAGE);
+  const uint32_t full0 = su32(bars), empty0 = su32(bars + S);
+  const uint32_t accf0 = su32(bars + 2 * S), acce0 = su32(bars + 2 * S + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * GM_BM;
-  const int n0 = blockIdx.x * (EPI == GEMM_SWIGLU ? BN / 2 : BN);
+  const int num_m = (g.M + GM_BM - 1) / GM_BM, num_n = (g.N + NOUT - 1) / NOUT;
+  const int ntiles = num_m * num_n;
   const int nk = g.K / GM_BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < GM_STAGES; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf0 + 8 * b, 1);
+      mbar_init(acce0 + 8 * b, 4);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&ta)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tb)) : "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)), "r"(BN));
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                 "r"(2 * BN));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -162,20 +158,26 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
 
   if (warp == 0) {
     if (lane == 0) {
+      int it = 0;
       bool ok = true;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % GM_STAGES;
-        const uint32_t ph = (kb / GM_STAGES) & 1;
-        if (ok) ok = mbar_wait(empty0 + 8 * s, ph ^ 1, g.err);
-        if (!ok) break;
-        const uint32_t a_s = su32(smem + s * STAGE), b_s = a_s + A_BYTES;
-        mbar_expect_tx(full0 + 8 * s, STAGE);
-        tma_load_2d(a_s, &ta, kb * GM_BK, m0, full0 + 8 * s);
-        if constexpr (EPI == GEMM_SWIGLU) {
-          tma_load_2d(b_s, &tb, kb * GM_BK, n0, full0 + 8 * s);
-          tma_load_2d(b_s + B_BYTES / 2, &tb3, kb * GM_BK, n0, full0 + 8 * s);
-        } else {
-          tma_load_2d(b_s, &tb, kb * GM_BK, n0, full0 + 8 * s);
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % num_m) * GM_BM, n0 = (tile / num_m) * NOUT;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, g.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_s = su32(smem + s * G::STAGE), b_s = a_s + G::A_BYTES;
+          mbar_expect_tx(full0 + 8 * s, G::STAGE);
+          tma_load_2d(a_s, &ta, kb * GM_BK, m0, full0 + 8 * s);
+          if constexpr (EPI == GEMM_SWIGLU) {
+            tma_load_2d(b_s, &tb, kb * GM_BK, n0, full0 + 8 * s);
+            tma_load_2d(b_s + G::B_BYTES / 2, &tb3, kb * GM_BK, n0, full0 + 8 * s);
+          } else {
+            tma_load_2d(b_s, &tb, kb * GM_BK, n0, full0 + 8 * s);
+          }
         }
       }
     }
@@ -183,35 +185,46 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
     if (lane == 0) {
       constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                  ((uint32_t)(GM_BM >> 4) << 24);
+      int it = 0, i = 0, after_fail = 0;
       bool ok = true;
-      int after_fail = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % GM_STAGES;
-        const uint32_t ph = (kb / GM_STAGES) & 1;
-        // after a failed wait keep draining (bounded) the stages the producer may still have in
-        // flight - it runs at most GM_STAGES ahead - so no copy lands after the block exits
-        if (!ok && ++after_fail > GM_STAGES) break;
-        const bool got = mbar_wait(full0 + 8 * s, ph, g.err);
-        ok = ok && got;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+        const int buf = i & 1;
+        if (ok && !mbar_wait(acce0 + 8 * buf, ((i >> 1) & 1) ^ 1, g.err)) ok = false;
         tc_fence_after();
-        if (ok) {
-          const uint64_t ad = sw128_desc(su32(smem + s * STAGE));
-          const uint64_t bd = sw128_desc(su32(smem + s * STAGE + A_BYTES));
+        const uint32_t td = tmem + buf * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          // after a failure keep draining (bounded) the stages the producer may still have in
+          // flight - it runs at most S ahead - so no copy lands after the block exits
+          if (!ok && ++after_fail > S) break;
+          const bool got = mbar_wait(full0 + 8 * s, ph, g.err);
+          ok = ok && got;
+          tc_fence_after();
+          if (ok) {
+            const uint64_t ad = sw128_desc(su32(smem + s * G::STAGE));
+            const uint64_t bd = sw128_desc(su32(smem + s * G::STAGE + G::A_BYTES));
 #pragma unroll
-          for (int k = 0; k < GM_BK / 16; ++k)
-            umma_f16(tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+            for (int k = 0; k < GM_BK / 16; ++k) umma_f16(td, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+          }
+          umma_commit(empty0 + 8 * s);
         }
-        umma_commit(empty0 + 8 * s);
+        umma_commit(accf0 + 8 * buf);
+        if (after_fail > S) break;
       }
-      umma_commit(accf);
     }
   } else {
     const int quarter = warp & 3;
-    const int row = m0 + quarter * 32 + lane;
-    const bool got = mbar_wait(accf, 0, g.err);
-    tc_fence_after();
-    const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16);
-    if (got) {
+    int i = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
+      const int buf = i & 1;
+      const int m0 = (tile % num_m) * GM_BM, n0 = (tile / num_m) * NOUT;
+      const int row = m0 + quarter * 32 + lane;
+      ok = mbar_wait(accf0 + 8 * buf, (i >> 1) & 1, g.err);
+      tc_fence_after();
+      if (!ok) break;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
       if constexpr (EPI == GEMM_SWIGLU) {
         bf16* out = reinterpret_cast<bf16*>(g.out);
 #pragma unroll 1
@@ -226,9 +239,9 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
               uint32_t w[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const int i = q * 8 + e * 2;
-                w[e] = pack_bf2(siluf_(g.alpha * va[i]) * (g.alpha * vb[i]),
-                                siluf_(g.alpha * va[i + 1]) * (g.alpha * vb[i + 1]));
+                const int j = q * 8 + e * 2;
+                w[e] = pack_bf2(siluf_(g.alpha * va[j]) * (g.alpha * vb[j]),
+                                siluf_(g.alpha * va[j + 1]) * (g.alpha * vb[j + 1]));
               }
               dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
             }
@@ -246,12 +259,12 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
               if (col + 32 <= g.N) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q)
-                  reinterpret_cast<float4*>(dst)[q] =
-                      make_float4(g.alpha * v[4 * q], g.alpha * v[4 * q + 1], g.alpha * v[4 * q + 2], g.alpha * v[4 * q + 3]);
+                  reinterpret_cast<float4*>(dst)[q] = make_float4(g.alpha * v[4 * q], g.alpha * v[4 * q + 1],
+                                                                  g.alpha * v[4 * q + 2], g.alpha * v[4 * q + 3]);
               } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                  if (i < g.N - col) dst[i] = g.alpha * v[i];
+                for (int j = 0; j < 32; ++j)
+                  if (j < g.N - col) dst[j] = g.alpha * v[j];
               }
             } else {
               bf16* dst = reinterpret_cast<bf16*>(g.out) + (size_t)row * g.ld + col;
@@ -265,23 +278,28 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
                 }
               } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                  if (i < g.N - col) dst[i] = f2bf(g.alpha * v[i]);
+                for (int j = 0; j < 32; ++j)
+                  if (j < g.N - col) dst[j] = f2bf(g.alpha * v[j]);
               }
             }
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce0 + 8 * buf);
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN));
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN));
 }
 
 template <int BN>
-constexpr size_t gemm_smem() { return 1024 + GM_STAGES * (size_t)(GM_BM * GM_BK * 2 + BN * GM_BK * 2) + 256; }
+constexpr size_t gemm_smem() { return 1024 + GemmGeom<BN>::STAGES * (size_t)GemmGeom<BN>::STAGE + 256; }
+
+static int g_gemm_sms = 0;
 
 template <int BN, int EPI>
 static cudaError_t launch_gemm(const GemmPlan& p, int M, int* err, cudaStream_t s) {
@@ -289,12 +307,16 @@ static cudaError_t launch_gemm(const GemmPlan& p, int M, int* err, cudaStream_t 
   auto k = k_gemm<BN, EPI>;
   GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err};
   const int ntile = EPI == GEMM_SWIGLU ? BN / 2 : BN;
-  dim3 grid((p.N + ntile - 1) / ntile, (M + GM_BM - 1) / GM_BM);
+  const int tiles = ((p.N + ntile - 1) / ntile) * ((M + GM_BM - 1) / GM_BM);
+  dim3 grid(std::min(tiles, g_gemm_sms > 0 ? g_gemm_sms : 148));
   return launch(k, grid, dim3(192), smem, s, p.a, p.b, EPI == GEMM_SWIGLU ? p.b3 : p.b, g);
 }
 
 cudaError_t gemm_init() {
   cudaError_t e;
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&g_gemm_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(k_gemm<128, GEMM_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem<128>())))
     return e;
   if ((e = cudaFuncSetAttribute(k_gemm<256, GEMM_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem<256>())))

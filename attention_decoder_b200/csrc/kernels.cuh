@@ -82,27 +82,35 @@ cudaError_t scratch_to_ring(const bf16* sk, const bf16* sv, int scratch_rows, in
 cudaError_t finish_step(int32_t* seq_len, const int32_t* row_slot, int rows, int add_prefill, int prefill_slot,
                         const unsigned long long* amax, int32_t* argmax_out, cudaStream_t s);
 
-// ---------------------------------------------------------------- decode GEMV (weights streamed once)
+// ---------------------------------------------------------------- decode projection epilogues
 enum GemvEpi { GEMV_PARTIAL = 0, GEMV_SWIGLU = 1, GEMV_CONV = 2, GEMV_HEAD = 3 };
-struct GemvArgs {
-  const bf16* w;   // [N][K]   (SwiGLU: w1; conv: in_proj [3D][D])
-  const bf16* w3;  // SwiGLU: w3 [F][K]
-  const uint8_t* codes;  const uint8_t* scales;   // NVFP4 (w1 for SwiGLU)
-  const uint8_t* codes3; const uint8_t* scales3;  // NVFP4 w3
-  float tscale;    // NVFP4 tensor scale
-  const bf16* x;   // [rows][K] activations
+
+// ---------------------------------------------------------------- decode weight streaming (persistent)
+enum WsPro { WS_PRO_LOAD = 0, WS_PRO_NORM = 1 };
+struct WsArgs {
+  const bf16* w; const bf16* w3;                   // bf16 weights [N][K] (SwiGLU: w1, w3)
+  const uint8_t* codes; const uint8_t* scales;     // NVFP4 (SwiGLU: w1)
+  const uint8_t* codes3; const uint8_t* scales3;   // NVFP4 w3
+  float tscale;
   int K, N, rows, splits;
-  float* part;     // GEMV_PARTIAL: [splits][rows][N]; GEMV_HEAD: logits [rows][N] (may be null)
-  bf16* out;       // GEMV_SWIGLU: u [rows][N]
-  // conv epilogue
-  const bf16* conv_w; bf16* conv_state; const int32_t* row_slot; int max_streams; bf16* y;
-  // head epilogue
-  unsigned long long* amax;
+  int pro;                                         // WS_PRO_LOAD: x bf16 [rows][K]; WS_PRO_NORM: see below
+  const bf16* x;
+  // WS_PRO_NORM (K == d_model): x' = x_in + g_post * RMS(sum_s parts[s]) (no parts: x' = x_in),
+  // written to x_out (+ dump) by block (0,0); activations = bf16(g_next * RMS(x'))
+  const float* x_in; float* x_out; const float* parts; int n_parts; long part_stride;
+  const bf16* g_post; const bf16* g_next; float eps; float* dump;
+  float* part_out;                                 // PARTIAL: [splits][rows][N]
+  bf16* out;                                       // SWIGLU: [rows][N]
+  const bf16* conv_w; bf16* conv_state; const int32_t* row_slot; bf16* y;  // CONV
+  unsigned long long* amax; float* logits;         // HEAD (logits may be null)
+  int* err;
 };
-cudaError_t gemv(int epi, int nvfp4, const GemvArgs& a, cudaStream_t s);
-cudaError_t gemv_init();  // one-time function attributes (before any capture)
+cudaError_t wstream(int epi, int nvfp4, const WsArgs& a, cudaStream_t s);
+cudaError_t wstream_init();
 
 // ---------------------------------------------------------------- attention
+constexpr int DEC_KEYS_FULL = 128;  // keys per decode split on full layers
+constexpr int DEC_KEYS_RING = 64;   // ring slots per decode split on sliding layers
 struct AttnLayer {
   int full;               // 1 full (pages), 0 sliding
   const bf16* k; const bf16* v;   // pages: this layer's pool; ring: this layer's ring base

@@ -18,7 +18,7 @@ using namespace lfm3;
 namespace {
 
 // Decode GEMV K splits (partial sums are added by the consumer).
-constexpr int SPLIT_QKVG = 2, SPLIT_DD = 2, SPLIT_W2 = 6, SPLIT_W2_FP4 = 5, SPLIT_MAX = 8;
+constexpr int SPLIT_DD = 2, SPLIT_W2 = 5, SPLIT_MAX = 8;
 constexpr int GEMV_MAX_ROWS = 16;
 
 struct LayerPlan {
@@ -45,10 +45,13 @@ struct lfm3_ctx {
   int32_t* row_pos = nullptr;
   unsigned long long* amax = nullptr;
   float* x_res = nullptr;
+  float* x_res2 = nullptr;  // decode: the residual stream ping-pongs between x_res and x_res2
   bf16* xn = nullptr;
   bf16* big = nullptr;
   bf16* y = nullptr;
   float* part = nullptr;
+  float* part2 = nullptr;   // decode: FFN down-projection partials
+  float* part3 = nullptr;   // decode: q|k|v|gate projection
   bf16* q = nullptr;
   float* gate = nullptr;
   bf16* sk = nullptr;
@@ -113,11 +116,14 @@ size_t layout(lfm3_ctx* c, char* base) {
   c->row_pos = reinterpret_cast<int32_t*>(take(4 * R));
   c->amax = reinterpret_cast<unsigned long long*>(take(8 * R));
   c->x_res = reinterpret_cast<float*>(take(4 * R * D));
+  c->x_res2 = reinterpret_cast<float*>(take(4 * (size_t)g.max_batch * D));
   c->xn = reinterpret_cast<bf16*>(take(2 * R * D));
   c->big = reinterpret_cast<bf16*>(take(2 * R * F));
   c->y = reinterpret_cast<bf16*>(take(2 * R * D));
   // fp32 projection outputs: the conv in_proj [R][3D], qkvg [R][3088], or decode K-split partials
   c->part = reinterpret_cast<float*>(take(4 * std::max(R * 3 * D, (size_t)SPLIT_MAX * g.max_batch * NQKVG)));
+  c->part2 = reinterpret_cast<float*>(take(4 * (size_t)SPLIT_MAX * g.max_batch * D));
+  c->part3 = reinterpret_cast<float*>(take(4 * (size_t)g.max_batch * NQKVG));
   c->q = reinterpret_cast<bf16*>(take(2 * R * HQ * HD));
   c->gate = reinterpret_cast<float*>(take(4 * R * HQ));
   c->sk = reinterpret_cast<bf16*>(take(2 * (size_t)HKV * c->scratch_rows * HD));
@@ -217,11 +223,6 @@ struct Bracket {
   }
 };
 
-double gemv_bytes(const GemvArgs& a, int nvfp4) {
-  const double w = nvfp4 ? (double)a.N * a.K / 2 + (double)a.N * a.K / 16 : 2.0 * a.N * a.K;
-  return w + 2.0 * a.rows * a.K + 4.0 * a.rows * a.N;
-}
-double gemv_flops(const GemvArgs& a) { return 2.0 * a.rows * a.N * a.K; }
 double gemm_flops(const GemmPlan& p, int M) {
   return 2.0 * M * (double)p.N * p.K * (p.epi == GEMM_SWIGLU ? 2 : 1);
 }
@@ -230,9 +231,13 @@ double gemm_bytes(const GemmPlan& p, int M) {
   return 2.0 * nw * p.N * (double)p.K + 2.0 * M * p.K + (p.epi == GEMM_F32 ? 4.0 : 2.0) * M * p.N;
 }
 
-cudaError_t run_gemv(lfm3_ctx* c, int epi, int fp4, const GemvArgs& a, cudaStream_t s) {
-  Bracket b(c, s, gemv_bytes(a, fp4), gemv_flops(a));
-  return gemv(epi, fp4, a, s);
+cudaError_t run_ws(lfm3_ctx* c, int epi, int fp4, const WsArgs& a, cudaStream_t s) {
+  const double mats = (a.w3 || a.codes3) ? 2.0 : 1.0;
+  const double rows = epi == GEMV_CONV ? 3.0 * D : (double)a.N;
+  const double w = fp4 ? rows * a.K / 2 + rows * a.K / 16 : 2.0 * rows * a.K;
+  const double bytes = mats * w + 2.0 * a.rows * a.K + 4.0 * a.rows * a.N;
+  Bracket b(c, s, bytes, 2.0 * a.rows * rows * a.K * mats);
+  return wstream(epi, fp4, a, s);
 }
 cudaError_t run_gemm(lfm3_ctx* c, const GemmPlan& p, int M, cudaStream_t s) {
   Bracket b(c, s, gemm_bytes(p, M), gemm_flops(p, M));
@@ -372,7 +377,7 @@ extern "C" lfm3_status lfm3_create(const lfm3_config* cfg, const lfm3_weights* w
   }
   c->max_pos = cfg->max_pages_per_stream * PAGE;
   c->R = std::max(cfg->max_chunk, cfg->max_batch);
-  c->max_splits = std::max((c->max_pos + 255) / 256, 4);
+  c->max_splits = std::max((c->max_pos + DEC_KEYS_FULL - 1) / DEC_KEYS_FULL, WIN / DEC_KEYS_RING);
   c->scratch_rows = WIN + cfg->max_chunk;
   c->ws_bytes = layout(c, nullptr);
   *workspace_bytes = c->ws_bytes;
@@ -387,7 +392,7 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
   if (bytes < ctx->ws_bytes)
     return fail(ctx, LFM3_E_ARG, "workspace of %zu bytes is smaller than the %zu required", bytes, ctx->ws_bytes);
   if (!tma_init()) return fail(ctx, LFM3_E_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  CK(gemv_init());
+  CK(wstream_init());
   CK(gemm_init());
   CK(attn_init());
   layout(ctx, reinterpret_cast<char*>(d_ws));
@@ -512,16 +517,18 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
     }
     const bool head = last && g.has_head && (d_logits || d_argmax);
     if (head) {
-      GemvArgs a{};
+      WsArgs a{};
       a.w = ctx->embed;
+      a.pro = WS_PRO_LOAD;
       a.x = ctx->xn + (size_t)(nc - 1) * D;
       a.K = D;
       a.N = g.vocab;
       a.rows = 1;
       a.splits = 1;
-      a.part = d_logits;
+      a.logits = d_logits;
       a.amax = ctx->amax;
-      CK(run_gemv(ctx, GEMV_HEAD, 0, a, s));
+      a.err = ctx->err;
+      CK(run_ws(ctx, GEMV_HEAD, 0, a, s));
     }
     CK(finish_step(st->seq_len, ctx->row_slot, nc, nc, slot, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
   }
@@ -533,12 +540,11 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
 namespace {
 
 // Every launch of one decode step, in order, on stream s.
-lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* d_slots,
+lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* d_slots,
                            const int32_t* d_tokens, const void* d_embeds, float* d_logits, int32_t* d_argmax,
                            float* d_hidden, int splits_full, float* attn_part, cudaStream_t s) {
   const lfm3_config& g = ctx->cfg;
   const float eps = g.eps;
-  const bool gv = nb <= GEMV_MAX_ROWS;
   const bool fp4 = g.ffn_format == LFM3_FFN_NVFP4;
   CK(setup_rows(0, 0, d_slots, st->seq_len, nb, ctx->row_slot, ctx->row_pos, ctx->amax, s));
   const Rows rows{ctx->row_slot, ctx->row_pos, nb};
@@ -550,21 +556,8 @@ lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const in
     const Views v = views(ctx, st, l);
     int np = 1;
     long pstride = 0;
-    GemvArgs a{};
-    a.rows = nb;
-    a.row_slot = ctx->row_slot;
-    a.max_streams = g.max_streams;
     if (g.layer_type[l] == LFM3_LAYER_CONV) {
-      if (gv) {
-        a.w = B(W.in_proj); a.x = ctx->xn; a.K = D; a.N = 3 * D; a.splits = 1;
-        a.conv_w = B(W.conv); a.conv_state = v.conv_layer; a.y = ctx->y;
-        CK(run_gemv(ctx, GEMV_CONV, 0, a, s));
-        GemvArgs o{};
-        o.w = B(W.out_proj); o.x = ctx->y; o.K = D; o.N = D; o.rows = nb; o.splits = SPLIT_DD; o.part = ctx->part;
-        CK(run_gemv(ctx, GEMV_PARTIAL, 0, o, s));
-        np = SPLIT_DD;
-        pstride = (long)nb * D;
-      } else {
+      {
         CK(run_gemm(ctx, P.in_proj, nb, s));
         CK(conv_decode(ctx->part, B(W.conv), v.conv_layer, ctx->row_slot, nb, ctx->y, s));
         CK(run_gemm(ctx, P.out_proj, nb, s));
@@ -573,12 +566,7 @@ lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const in
       const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
       int nq = 1;
       long qstride = 0;
-      if (gv) {
-        a.w = B(W.qkvg); a.x = ctx->xn; a.K = D; a.N = NQKVG; a.splits = SPLIT_QKVG; a.part = ctx->part;
-        CK(run_gemv(ctx, GEMV_PARTIAL, 0, a, s));
-        nq = SPLIT_QKVG;
-        qstride = (long)nb * NQKVG;
-      } else {
+      {
         CK(run_gemm(ctx, P.qkvg, nb, s));
       }
       KvWrite kw{};
@@ -591,43 +579,16 @@ lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const in
       const int k = full ? 0 : 1;
       CK(qk_norm_rope_kv(ctx->part, nq, qstride, B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], rows,
                          eps, ctx->q, ctx->gate, kw, s));
-      CK(attn_decode(ctx->q, rows, attn_layer(ctx, st, l, v), full ? splits_full : WIN / 64, attn_part, ctx->gate,
+      CK(attn_decode(ctx->q, rows, attn_layer(ctx, st, l, v), full ? splits_full : WIN / DEC_KEYS_RING, attn_part, ctx->gate,
                      ctx->y, s));
-      if (gv) {
-        GemvArgs o{};
-        o.w = B(W.o_proj); o.x = ctx->y; o.K = HQ * HD; o.N = D; o.rows = nb; o.splits = SPLIT_DD; o.part = ctx->part;
-        CK(run_gemv(ctx, GEMV_PARTIAL, 0, o, s));
-        np = SPLIT_DD;
-        pstride = (long)nb * D;
-      } else {
+      {
         CK(run_gemm(ctx, P.o_proj, nb, s));
       }
     }
     CK(resid_norm(ctx->x_res, ctx->part, np, pstride, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nb, eps, nullptr, s));
     np = 1;
     pstride = 0;
-    if (gv) {
-      GemvArgs f{};
-      f.rows = nb; f.x = ctx->xn; f.K = D; f.N = F; f.splits = 1; f.out = ctx->big;
-      if (fp4) {
-        f.codes = W.w1_codes; f.scales = W.w1_scales; f.codes3 = W.w3_codes; f.scales3 = W.w3_scales;
-        f.tscale = W.w13_scale;
-      } else {
-        f.w = B(W.w1); f.w3 = B(W.w3);
-      }
-      CK(run_gemv(ctx, GEMV_SWIGLU, fp4, f, s));
-      GemvArgs d{};
-      d.rows = nb; d.x = ctx->big; d.K = F; d.N = D; d.part = ctx->part;
-      d.splits = fp4 ? SPLIT_W2_FP4 : SPLIT_W2;
-      if (fp4) {
-        d.codes = W.w2_codes; d.scales = W.w2_scales; d.tscale = W.w2_scale;
-      } else {
-        d.w = B(W.w2);
-      }
-      CK(run_gemv(ctx, GEMV_PARTIAL, fp4, d, s));
-      np = d.splits;
-      pstride = (long)nb * D;
-    } else {
+    {
       lfm3_status fs = ffn_gemm(ctx, l, nb, s);
       if (fs != LFM3_OK) return fs;
     }
@@ -638,20 +599,169 @@ lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const in
   const bool head = g.has_head && (d_logits || d_argmax);
   if (head) {
     for (int b0 = 0; b0 < nb; b0 += GEMV_MAX_ROWS) {
-      GemvArgs a{};
+      WsArgs a{};
       a.w = ctx->embed;
+      a.pro = WS_PRO_LOAD;
       a.x = ctx->xn + (size_t)b0 * D;
       a.K = D;
       a.N = g.vocab;
       a.rows = std::min(GEMV_MAX_ROWS, nb - b0);
       a.splits = 1;
-      a.part = d_logits ? d_logits + (size_t)b0 * g.vocab : nullptr;
+      a.logits = d_logits ? d_logits + (size_t)b0 * g.vocab : nullptr;
       a.amax = ctx->amax + b0;
-      CK(run_gemv(ctx, GEMV_HEAD, 0, a, s));
+      a.err = ctx->err;
+      CK(run_ws(ctx, GEMV_HEAD, 0, a, s));
     }
   }
   CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
   return LFM3_OK;
+}
+
+// Decode for up to 16 streams: the weight-streaming kernel, whose prologue also applies the
+// previous projection's residual add + post-norm and this projection's input norm.
+lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* d_slots,
+                                  const int32_t* d_tokens, const void* d_embeds, float* d_logits, int32_t* d_argmax,
+                                  float* d_hidden, int splits_full, float* attn_part, cudaStream_t s) {
+  const lfm3_config& g = ctx->cfg;
+  const float eps = g.eps;
+  const bool fp4 = g.ffn_format == LFM3_FFN_NVFP4;
+  CK(setup_rows(0, 0, d_slots, st->seq_len, nb, ctx->row_slot, ctx->row_pos, ctx->amax, s));
+  const Rows rows{ctx->row_slot, ctx->row_pos, nb};
+  CK(embed_rows(d_tokens, ctx->embed, B(d_embeds), nb, ctx->x_res, d_hidden, s));
+  float* cur = ctx->x_res;
+  float* nxt = ctx->x_res2;
+  // partial sums still to be added into the residual (with their post-norm gain)
+  const float* pend = nullptr;
+  int pend_n = 0;
+  const bf16* pend_g = nullptr;
+  auto base = [&](WsArgs& a, int K, int N, int splits) {
+    a.rows = nb;
+    a.K = K;
+    a.N = N;
+    a.splits = splits;
+    a.err = ctx->err;
+    a.eps = eps;
+  };
+  auto norm_in = [&](WsArgs& a, const bf16* g_next, float* dump) {
+    a.pro = WS_PRO_NORM;
+    a.x_in = cur;
+    a.x_out = nxt;
+    a.parts = pend;
+    a.n_parts = pend_n;
+    a.part_stride = (long)nb * D;
+    a.g_post = pend_g;
+    a.g_next = g_next;
+    a.dump = dump;
+  };
+  auto advance = [&]() { std::swap(cur, nxt); };
+  for (int l = 0; l < g.n_layers; ++l) {
+    const lfm3_layer_weights& W = ctx->L[l];
+    const Views v = views(ctx, st, l);
+    float* dump_l = (d_hidden && l > 0) ? d_hidden + (size_t)l * nb * D : nullptr;
+    if (g.layer_type[l] == LFM3_LAYER_CONV) {
+      WsArgs c{};
+      base(c, D, 3 * D, 1);
+      c.w = B(W.in_proj);
+      c.conv_w = B(W.conv);
+      c.conv_state = v.conv_layer;
+      c.row_slot = ctx->row_slot;
+      c.y = ctx->y;
+      norm_in(c, B(W.op_norm), dump_l);
+      CK(run_ws(ctx, GEMV_CONV, 0, c, s));
+      advance();
+      WsArgs o{};
+      base(o, D, D, SPLIT_DD);
+      o.pro = WS_PRO_LOAD;
+      o.x = ctx->y;
+      o.w = B(W.out_proj);
+      o.part_out = ctx->part;
+      CK(run_ws(ctx, GEMV_PARTIAL, 0, o, s));
+    } else {
+      const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
+      WsArgs q{};
+      base(q, D, NQKVG, 1);
+      q.w = B(W.qkvg);
+      q.part_out = ctx->part3;
+      norm_in(q, B(W.op_norm), dump_l);
+      CK(run_ws(ctx, GEMV_PARTIAL, 0, q, s));
+      advance();
+      KvWrite kw{};
+      kw.mode = full ? KV_PAGES : KV_RING;
+      kw.k = full ? v.kv_k : v.ring_k;
+      kw.v = full ? v.kv_v : v.ring_v;
+      kw.page_table = st->page_table;
+      kw.max_pages = g.max_pages_per_stream;
+      kw.max_streams = g.max_streams;
+      const int k = full ? 0 : 1;
+      CK(qk_norm_rope_kv(ctx->part3, 1, 0, B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], rows, eps,
+                         ctx->q, ctx->gate, kw, s));
+      CK(attn_decode(ctx->q, rows, attn_layer(ctx, st, l, v), full ? splits_full : WIN / DEC_KEYS_RING, attn_part,
+                     ctx->gate, ctx->y, s));
+      WsArgs o{};
+      base(o, HQ * HD, D, SPLIT_DD);
+      o.pro = WS_PRO_LOAD;
+      o.x = ctx->y;
+      o.w = B(W.o_proj);
+      o.part_out = ctx->part;
+      CK(run_ws(ctx, GEMV_PARTIAL, 0, o, s));
+    }
+    pend = ctx->part;
+    pend_n = SPLIT_DD;
+    pend_g = B(W.post_op_norm);
+    WsArgs f{};
+    base(f, D, F, 1);
+    f.out = ctx->big;
+    if (fp4) {
+      f.codes = W.w1_codes; f.scales = W.w1_scales; f.codes3 = W.w3_codes; f.scales3 = W.w3_scales;
+      f.tscale = W.w13_scale;
+    } else {
+      f.w = B(W.w1);
+      f.w3 = B(W.w3);
+    }
+    norm_in(f, B(W.ffn_norm), nullptr);
+    CK(run_ws(ctx, GEMV_SWIGLU, fp4, f, s));
+    advance();
+    WsArgs d{};
+    base(d, F, D, SPLIT_W2);
+    d.pro = WS_PRO_LOAD;
+    d.x = ctx->big;
+    d.part_out = ctx->part2;
+    if (fp4) {
+      d.codes = W.w2_codes; d.scales = W.w2_scales; d.tscale = W.w2_scale;
+    } else {
+      d.w = B(W.w2);
+    }
+    CK(run_ws(ctx, GEMV_PARTIAL, fp4, d, s));
+    pend = ctx->part2;
+    pend_n = SPLIT_W2;
+    pend_g = B(W.post_ffn_norm);
+  }
+  float* dump_last = d_hidden ? d_hidden + (size_t)g.n_layers * nb * D : nullptr;
+  const bool head = g.has_head && (d_logits || d_argmax);
+  if (head) {
+    WsArgs h{};
+    base(h, D, g.vocab, 1);
+    h.w = ctx->embed;
+    h.logits = d_logits;
+    h.amax = ctx->amax;
+    norm_in(h, ctx->final_norm, dump_last);
+    CK(run_ws(ctx, GEMV_HEAD, 0, h, s));
+    advance();
+  } else if (dump_last) {
+    CK(resid_norm(cur, pend, pend_n, (long)nb * D, pend_g, nullptr, nullptr, nb, eps, dump_last, s));
+  }
+  CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
+  return LFM3_OK;
+}
+
+lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* d_slots,
+                           const int32_t* d_tokens, const void* d_embeds, float* d_logits, int32_t* d_argmax,
+                           float* d_hidden, int splits_full, float* attn_part, cudaStream_t s) {
+  if (nb <= GEMV_MAX_ROWS)
+    return enqueue_decode_stream(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                                 splits_full, attn_part, s);
+  return enqueue_decode_large(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden, splits_full,
+                              attn_part, s);
 }
 
 }  // namespace
@@ -683,7 +793,7 @@ lfm3_status validate_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const i
     maxpos = std::max(maxpos, (int)st->h_seq_len[s]);
   }
   int splits_full = 1;
-  while (splits_full < maxpos / 256 + 1) splits_full *= 2;
+  while (splits_full < maxpos / DEC_KEYS_FULL + 1) splits_full *= 2;
   *splits_out = std::min(splits_full, ctx->max_splits);
   return LFM3_OK;
 }
@@ -758,7 +868,7 @@ extern "C" lfm3_status lfm3_decode_step_noalloc(lfm3_ctx* ctx, const lfm3_state*
   float* scratch = nullptr;
   size_t cap = 0;
   CK(attn_static_scratch(&scratch, &cap));
-  const size_t need = (size_t)nb * HQ * std::max(splits_full, WIN / 64) * (HD + 2);
+  const size_t need = (size_t)nb * HQ * std::max(splits_full, WIN / DEC_KEYS_RING) * (HD + 2);
   if (need > cap)
     return fail(ctx, LFM3_E_CAPACITY,
                 "lfm3_decode_step_noalloc: %d streams x %d key splits need %zu bytes of attention scratch, more "

@@ -180,9 +180,9 @@ lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int n_streams,
  *   results go to a fixed 4 MiB array inside the library's own device image instead of the
  *   workspace, and the step is launched kernel by kernel (no captured graph).
  *   Limit: n_streams x 16 heads x splits x 130 floats must fit in the 4 MiB, where splits is
- *   max(4, the smallest power of two >= (longest context / 256) + 1); larger calls are refused
- *   with LFM3_E_CAPACITY and a message giving both sizes. One stream fits up to 126 splits
- *   (the whole 32k context); 64 streams fit 7 (contexts below 1792).
+ *   max(4, the smallest power of two >= (longest context / 128) + 1); larger calls are refused
+ *   with LFM3_E_CAPACITY and a message giving both sizes. One stream fits any context below
+ *   32768 positions; 64 streams fit contexts below 384.
  *   Nothing in the array has to start at zero: every call writes all the partials it reads.
  *   The array is one per GPU for the whole process and every call shares it, so calls that can
  *   overlap on the GPU (different streams, different contexts) race on it; serialise them.

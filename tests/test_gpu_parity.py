@@ -254,7 +254,9 @@ def test_graph_replay_equals_direct_launches_and_profile_counts(lib, slice3, mon
             p = m.profile_read()
             m.profile(False)
             # conv layer: in_proj+conv, out_proj, w1|w3, w2; attention layers: qkvg, o_proj, w1|w3, w2
-            assert p["launches"] == 12 and p["ms"] > 0 and p["bytes"] > 3 * 127e6
+            wbytes = 2 * (3 * 2048 * 2048 + 2048 * 2048 + 2 * 3088 * 2048 + 2 * 2048 * 2048 + 3 * 3 * 7680 * 2048)
+            assert p["launches"] == 12 and p["ms"] > 0
+            assert wbytes < p["bytes"] < wbytes * 1.01
     for a, b in zip(runs[0][0], runs[1][0]):
         assert torch.equal(a, b)
     for i in (1, 2, 3):

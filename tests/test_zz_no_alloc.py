@@ -92,7 +92,8 @@ def test_noalloc_decode_with_head_and_size_refusal(mods):
         _, ln, an = _call(L, m, b, L.lib().lfm3_decode_step_noalloc, [0], tokens=tok[t:t + 1], with_head=True)
         assert float((ln - lr).abs().max()) <= LOGIT_ABS
         assert torch.equal(ln, lr) and torch.equal(an, ar)
-    # 64 streams at a 2048-token context need 16 x 64 x 16 x 130 floats: more than the fixed array
+    # 64 streams at a 2048-token context need 64 x 16 heads x 32 splits x 130 floats (17 MB):
+    # more than the fixed array
     st.h_seq_len[:] = 2048
     st.seq_len.fill_(2048)
     before = st.h_seq_len.copy()
