@@ -19,8 +19,15 @@
 // (x' = x + g_post * RMS(sum parts)), normalises (bf16(g_next * RMS(x'))) and keeps its K range
 // in shared memory; block (0, 0) writes x' to the other residual buffer (and the hidden dump), so
 // no block ever reads a residual another block is rewriting.
-// NVFP4 weights (E2M1 codes + E4M3 block scales) are expanded in registers to exact bf16 values;
-// the fp32 tensor scale multiplies the finished sums.
+// NVFP4 weights (E2M1 codes + E4M3 block scales) are expanded to exact bf16 values through a
+// byte -> bf16x2 table in shared memory (one copy per bank, so lookups never conflict) and a bf16
+// multiply by the block scale (exact: at most 6 significant bits); the fp32 tensor scale
+// multiplies the finished sums.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdlib>
+
 #include "kernels.cuh"
 
 namespace lfm3 {
@@ -37,17 +44,25 @@ template <int EPI, bool FP4>
 struct WsGeom {
   static constexpr int NRT = WsRows<EPI>::NRT;
   static constexpr int RPT = 16 * NRT;                        // weight rows per tile
-  static constexpr int KB = FP4 ? 128 : 32;                   // K per lane step
+  static constexpr int BR = EPI == GEMV_SWIGLU ? 8 : 16;      // rows per copy request (w1 | w3 halves)
+  static constexpr int NREQ = RPT / BR;                       // copy requests per stage
+  static constexpr int KB = FP4 ? 128 : 32;                   // K per lane step (64 bytes of a row)
   static constexpr int KCH = FP4 ? 512 : (NRT == 3 ? 256 : 512);  // K per stage
-  static constexpr int ROWB = FP4 ? KCH / 2 : KCH * 2;        // weight bytes per row per stage
-  static constexpr int RS = ROWB + 64;                        // padded row stride in shared memory
+  static constexpr int NKB = KCH / KB;                        // 64-byte blocks per row per stage
+  static constexpr int REQB = 64 * BR * NKB;                  // bytes of one request: [block][row][64 B]
+  static constexpr int ROWB = 64 * NKB;                       // weight bytes per row per stage
   static constexpr int SCB = FP4 ? KCH / 16 : 0;              // scale bytes per row per stage
-  static constexpr int STAGES = FP4 ? 8 : 4;
-  static constexpr int STAGE_BYTES = RPT * RS + RPT * SCB;
-  static constexpr int TX_BYTES = RPT * (ROWB + SCB);
+  static constexpr int STAGES = FP4 ? 12 : (NRT == 3 ? 3 : 6);  // default ring depth (runtime: a.stages)
+  static constexpr int STAGE_BYTES = RPT * ROWB + RPT * SCB;
+  static constexpr int TX_BYTES = STAGE_BYTES;
   static constexpr int STEPS = KCH / KB;                      // lane steps per stage
-  static constexpr int STEPB = 64;                            // bytes of a row per lane step
 };
+
+// Byte offset, inside a stage, of the 16 bytes lane chunk t reads from row r at step j.
+template <class G>
+DEVI int ws_woff(int r, int j, int t) {
+  return (r / G::BR) * G::REQB + j * (G::BR * 64) + (r % G::BR) * 64 + t * 16;
+}
 
 // Row of tile `tile`, sub-tile rt, fragment row g (0..15); `which` selects w3 for SwiGLU.
 template <int EPI>
@@ -63,19 +78,14 @@ DEVI int ws_row(int tile, int rt, int g, int& which) {
   }
 }
 
-// E2M1 magnitude (3 bits) -> bf16 high and low bytes, as byte-permute tables (0 .. 6).
-constexpr uint32_t WS_HI_LO = 0x3F3F3F00u, WS_HI_HI = 0x40404040u;
-constexpr uint32_t WS_LO_LO = 0xC0800000u, WS_LO_HI = 0xC0804000u;
+constexpr int WS_LUT_BYTES = 256 * 32 * 4;
 
-DEVI void ws_e2m1x4(uint32_t w, uint32_t& o01, uint32_t& o23) {
-  const uint32_t sel = w & 0x7777u;
-  const uint32_t hi = __byte_perm(WS_HI_LO, WS_HI_HI, sel);
-  const uint32_t lo = __byte_perm(WS_LO_LO, WS_LO_HI, sel);
-  o01 = __byte_perm(lo, hi, 0x5140);
-  o23 = __byte_perm(lo, hi, 0x7362);
-  const uint32_t s = w & 0x8888u;
-  o01 |= ((s << 12) & 0x8000u) | ((s << 24) & 0x80000000u);
-  o23 |= ((s << 4) & 0x8000u) | ((s << 16) & 0x80000000u);
+// E2M1 code (bit 3 sign, bits 2..1 exponent with bias 1, bit 0 mantissa) -> bf16 bits, exact:
+// 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives.
+DEVI uint32_t e2m1_bf16_bits(uint32_t c) {
+  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+  const uint32_t mag = e == 0 ? (m ? 0x3F00u : 0u) : (((e + 126u) << 7) | (m << 6));
+  return mag | ((c & 8u) << 12);
 }
 
 DEVI uint32_t ws_e4m3x2(uint32_t b) {
@@ -92,21 +102,49 @@ DEVI uint32_t ws_hmul2(uint32_t a, uint32_t b) {
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
+DEVI void ws_tma3(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+DEVI void ws_tma2(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
 DEVI void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(WS_CW * 32) : "memory"); }
 
-template <int NT>
-DEVI size_t ws_x_bytes(int Kc) { return (size_t)NT * 8 * (Kc + 32) * 2; }
+// Activations in shared memory: a 128-byte zero block (the MMA columns of absent streams read
+// it), then one row per stream of the block's K range, 64-byte skewed against bank conflicts.
+__host__ __device__ inline size_t ws_x_bytes(int rows, int Kc) { return 128 + (size_t)rows * (Kc + 32) * 2; }
+// Stages start on a 1024-byte boundary after the activations (and the NVFP4 table).
+__host__ __device__ inline size_t ws_stage_base(int rows, int Kc, bool fp4) {
+  return (ws_x_bytes(rows, Kc) + (fp4 ? 256 * 32 * 4 : 0) + 1023) / 1024 * 1024;
+}
 
 template <int EPI, int NT, bool FP4>
-__global__ void __launch_bounds__(WS_THREADS) k_wstream(const WsArgs a) {
+__global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ CUtensorMap tw,
+                                                        const __grid_constant__ CUtensorMap tw3,
+                                                        const __grid_constant__ CUtensorMap tsc,
+                                                        const __grid_constant__ CUtensorMap tsc3, const WsArgs a) {
   using G = WsGeom<EPI, FP4>;
   constexpr int NRT = G::NRT;
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int Kc = a.K / a.splits;
   const int XS = Kc + 32;  // activations row stride (elements): 64-byte skew against bank conflicts
-  bf16* xs = reinterpret_cast<bf16*>(smem);
-  unsigned char* stages = smem + ws_x_bytes<NT>(Kc);
-  float* red = reinterpret_cast<float*>(stages + (size_t)G::STAGES * G::STAGE_BYTES);
+  const bf16* xzero = reinterpret_cast<const bf16*>(smem);
+  bf16* xs = reinterpret_cast<bf16*>(smem + 128);
+  // NVFP4: byte (two E2M1 codes) -> bf16x2, 256 entries x 32 copies (one per bank)
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + ws_x_bytes(a.rows, Kc));
+  unsigned char* stages = smem + ws_stage_base(a.rows, Kc, FP4);
+  const int NS = a.stages;  // ring depth chosen by the launcher
+  float* red = reinterpret_cast<float*>(stages + (size_t)NS * G::STAGE_BYTES);
   float* res = red + WS_CW * NRT * NT * 128;
   uint64_t* bars = reinterpret_cast<uint64_t*>(res + NRT * 16 * NT * 8);
   __shared__ float redn[WS_CW];
@@ -116,10 +154,10 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const WsArgs a) {
   const int kcta = blockIdx.y * Kc;
   const int nch = Kc / G::KCH;
   const int ntiles = (EPI == GEMV_SWIGLU) ? a.N / 8 : (EPI == GEMV_CONV ? D / 16 : a.N / 16);
-  const uint32_t full0 = su32(bars), empty0 = su32(bars + G::STAGES);
+  const uint32_t full0 = su32(bars), empty0 = su32(bars + NS);
 
   if (tid == 0) {
-    for (int s = 0; s < G::STAGES; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, WS_CW);
     }
@@ -134,27 +172,24 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const WsArgs a) {
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       for (int ch = 0; ch < nch && ok; ++ch, ++it) {
-        const int s = it % G::STAGES;
-        const uint32_t ph = (it / G::STAGES) & 1;
+        const int s = it % NS;
+        const uint32_t ph = (it / NS) & 1;
         if (lane == 0) ok = mbar_wait(empty0 + 8 * s, ph ^ 1, a.err);
         ok = __shfl_sync(0xffffffffu, ok, 0) && !*(volatile int*)&abort_flag;
         if (!ok) break;
-        if (lane == 0) mbar_expect_tx(full0 + 8 * s, G::TX_BYTES);
-        __syncwarp();
-        unsigned char* st = stages + (size_t)s * G::STAGE_BYTES;
-        const int k0 = kcta + ch * G::KCH;
-        for (int r = lane; r < G::RPT; r += 32) {
-          int which;
-          const int row = ws_row<EPI>(tile, r / 16, r % 16, which);
-          if constexpr (FP4) {
-            const uint8_t* cs = which ? a.codes3 : a.codes;
-            const uint8_t* ss = which ? a.scales3 : a.scales;
-            bulk_g2s(su32(st + r * G::RS), cs + (size_t)row * (a.K / 2) + k0 / 2, G::ROWB, full0 + 8 * s);
-            bulk_g2s(su32(st + G::RPT * G::RS + r * G::SCB), ss + (size_t)row * (a.K / 16) + k0 / 16, G::SCB,
-                     full0 + 8 * s);
-          } else {
-            const bf16* wm = which ? a.w3 : a.w;
-            bulk_g2s(su32(st + r * G::RS), wm + (size_t)row * a.K + k0, G::ROWB, full0 + 8 * s);
+        if (lane == 0) {
+          mbar_expect_tx(full0 + 8 * s, G::TX_BYTES);
+          unsigned char* st = stages + (size_t)s * G::STAGE_BYTES;
+          const int k0 = kcta + ch * G::KCH;
+#pragma unroll
+          for (int q = 0; q < G::NREQ; ++q) {
+            int which;
+            const int row = ws_row<EPI>(tile, (q * G::BR) / 16, (q * G::BR) % 16, which);
+            const CUtensorMap* m = which ? &tw3 : &tw;
+            ws_tma3(su32(st + q * G::REQB), m, 0, row, k0 / G::KB, full0 + 8 * s);
+            if constexpr (FP4)
+              ws_tma2(su32(st + G::RPT * G::ROWB + q * G::BR * G::SCB), which ? &tsc3 : &tsc, k0 / 16, row,
+                      full0 + 8 * s);
           }
         }
       }
@@ -163,9 +198,9 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const WsArgs a) {
     pdl_launch_dependents();
     if (!ok) {
       // drain: copies already issued land before the block exits (bounded)
-      for (int k = 0; k < G::STAGES && k < it; ++k) {
+      for (int k = 0; k < NS && k < it; ++k) {
         const int i = it - 1 - k;
-        if (lane == 0) mbar_wait(full0 + 8 * (i % G::STAGES), (i / G::STAGES) & 1, a.err);
+        if (lane == 0) mbar_wait(full0 + 8 * (i % NS), (i / NS) & 1, a.err);
       }
     }
     return;
@@ -175,23 +210,23 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const WsArgs a) {
   pdl_wait();
   pdl_launch_dependents();
   const int ct = tid;  // 0..127
+  if (ct < 8) reinterpret_cast<uint4*>(smem)[ct] = make_uint4(0, 0, 0, 0);
+  if constexpr (FP4) {
+    for (int i = ct; i < 256 * 32; i += WS_CW * 32) {
+      const uint32_t v = (uint32_t)i >> 5;
+      lut[i] = e2m1_bf16_bits(v & 15u) | (e2m1_bf16_bits(v >> 4) << 16);
+    }
+  }
   if (a.pro == WS_PRO_LOAD) {
     const int chunks = Kc / 8;
-    for (int idx = ct; idx < NT * 8 * chunks; idx += WS_CW * 32) {
+    for (int idx = ct; idx < a.rows * chunks; idx += WS_CW * 32) {
       const int b = idx / chunks, c = idx - b * chunks;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (b < a.rows) v = ldg16(a.x + (size_t)b * a.K + kcta + c * 8);
-      *reinterpret_cast<uint4*>(xs + (size_t)b * XS + c * 8) = v;
+      *reinterpret_cast<uint4*>(xs + (size_t)b * XS + c * 8) = ldg16(a.x + (size_t)b * a.K + kcta + c * 8);
     }
   } else {
     // residual + post-norm of the previous projection, then this projection's input norm
     const bool writer = blockIdx.x == 0 && blockIdx.y == 0;
-    for (int b = 0; b < NT * 8; ++b) {
-      if (b >= a.rows) {
-        for (int c = ct; c < Kc / 8; c += WS_CW * 32)
-          *reinterpret_cast<uint4*>(xs + (size_t)b * XS + c * 8) = make_uint4(0, 0, 0, 0);
-        continue;
-      }
+    for (int b = 0; b < a.rows; ++b) {
       float x[16];
       const float* xin = a.x_in + (size_t)b * D + ct * 16;
 #pragma unroll
@@ -272,8 +307,8 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const WsArgs a) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[rt][nt][j] = 0.f;
     for (int ch = 0; ch < nch; ++ch, ++it) {
-      const int s = it % G::STAGES;
-      const uint32_t ph = (it / G::STAGES) & 1;
+      const int s = it % NS;
+      const uint32_t ph = (it / NS) & 1;
       // after any bounded wait gives up, every warp keeps walking the same loop (so all of them
       // reach every consumer barrier) but waits for nothing and computes nothing
       if (ok && *(volatile int*)&abort_flag) ok = false;
@@ -293,36 +328,39 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const WsArgs a) {
           const int kx = ch * G::KCH + j * G::KB;  // K offset of this step in the block's range
 #pragma unroll
           for (int rt = 0; rt < NRT; ++rt) {
-            const uint4 wa = *reinterpret_cast<const uint4*>(st + (rt * 16 + g) * G::RS + j * G::STEPB + t * 16);
-            const uint4 wb = *reinterpret_cast<const uint4*>(st + (rt * 16 + g + 8) * G::RS + j * G::STEPB + t * 16);
+            const uint4 wa = *reinterpret_cast<const uint4*>(st + ws_woff<G>(rt * 16 + g, j, t));
+            const uint4 wb = *reinterpret_cast<const uint4*>(st + ws_woff<G>(rt * 16 + g + 8, j, t));
             if constexpr (!FP4) {
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
-                const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)(nt * 8 + g) * XS + kx + 8 * t);
+                const int sr = nt * 8 + g;
+                const uint4 xv = *reinterpret_cast<const uint4*>(sr < a.rows ? xs + (size_t)sr * XS + kx + 8 * t : xzero);
                 mma_bf16_16816(acc[rt][nt], wa.x, wb.x, wa.y, wb.y, xv.x, xv.y);
                 mma_bf16_16816(acc[rt][nt], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
               }
             } else {
-              const unsigned char* sc = st + G::RPT * G::RS;
+              const unsigned char* sc = st + G::RPT * G::ROWB;  // scales: [request][row][SCB]
               const uint32_t sa = *reinterpret_cast<const uint16_t*>(sc + (rt * 16 + g) * G::SCB + j * 8 + 2 * t);
               const uint32_t sb = *reinterpret_cast<const uint16_t*>(sc + (rt * 16 + g + 8) * G::SCB + j * 8 + 2 * t);
               const uint32_t s0a = ws_e4m3x2(sa & 0xFF), s1a = ws_e4m3x2(sa >> 8);
               const uint32_t s0b = ws_e4m3x2(sb & 0xFF), s1b = ws_e4m3x2(sb >> 8);
               const uint32_t wA[4] = {wa.x, wa.y, wa.z, wa.w};
               const uint32_t wB[4] = {wb.x, wb.y, wb.z, wb.w};
+              const uint32_t* tab = lut + lane;  // this lane's copy of the table
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                uint32_t a01, a23, a45, a67, b01, b23, b45, b67;
-                ws_e2m1x4(wA[q], a01, a23);
-                ws_e2m1x4(wA[q] >> 16, a45, a67);
-                ws_e2m1x4(wB[q], b01, b23);
-                ws_e2m1x4(wB[q] >> 16, b45, b67);
+                uint32_t a01 = tab[(wA[q] & 0xFFu) << 5], a23 = tab[((wA[q] >> 8) & 0xFFu) << 5];
+                uint32_t a45 = tab[((wA[q] >> 16) & 0xFFu) << 5], a67 = tab[(wA[q] >> 24) << 5];
+                uint32_t b01 = tab[(wB[q] & 0xFFu) << 5], b23 = tab[((wB[q] >> 8) & 0xFFu) << 5];
+                uint32_t b45 = tab[((wB[q] >> 16) & 0xFFu) << 5], b67 = tab[(wB[q] >> 24) << 5];
                 const uint32_t sA = q < 2 ? s0a : s1a, sB = q < 2 ? s0b : s1b;
                 a01 = ws_hmul2(a01, sA); a23 = ws_hmul2(a23, sA); a45 = ws_hmul2(a45, sA); a67 = ws_hmul2(a67, sA);
                 b01 = ws_hmul2(b01, sB); b23 = ws_hmul2(b23, sB); b45 = ws_hmul2(b45, sB); b67 = ws_hmul2(b67, sB);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                  const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)(nt * 8 + g) * XS + kx + 32 * t + 8 * q);
+                  const int sr = nt * 8 + g;
+                  const uint4 xv = *reinterpret_cast<const uint4*>(sr < a.rows ? xs + (size_t)sr * XS + kx + 32 * t + 8 * q
+                                                                               : xzero);
                   mma_bf16_16816(acc[rt][nt], a01, b01, a23, b23, xv.x, xv.y);
                   mma_bf16_16816(acc[rt][nt], a45, b45, a67, b67, xv.z, xv.w);
                 }
@@ -407,45 +445,92 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const WsArgs a) {
 }
 
 template <int EPI, bool FP4>
-size_t ws_smem(int NT, int Kc) {
+size_t ws_smem(int NT, int rows, int Kc, int stages) {
   using G = WsGeom<EPI, FP4>;
-  const size_t x = (size_t)NT * 8 * (Kc + 32) * 2;
-  return x + (size_t)G::STAGES * G::STAGE_BYTES + (size_t)WS_CW * G::NRT * NT * 128 * 4 +
-         (size_t)G::NRT * 16 * NT * 8 * 4 + 2 * G::STAGES * 8;
+  const size_t x = ws_stage_base(rows, Kc, FP4);
+  return 1024 + x + (size_t)stages * G::STAGE_BYTES + (size_t)WS_CW * G::NRT * NT * 128 * 4 +
+         (size_t)G::NRT * 16 * NT * 8 * 4 + 2 * stages * 8;
 }
 
 static int g_num_sms = 0;
+static int g_ws_bps = 2;     // blocks per SM (LFM3_WS_BLOCKS_PER_SM)
+static int g_ws_stages = 0;  // ring depth override (LFM3_WS_STAGES); 0 = the per-shape default
 
 template <int EPI, bool FP4>
-static cudaError_t launch_ws(const WsArgs& a, cudaStream_t s) {
+static cudaError_t launch_ws(const WsMaps& mp, const WsArgs& a, cudaStream_t s) {
   using G = WsGeom<EPI, FP4>;
   const int Kc = a.K / a.splits;
   if (Kc % G::KCH || a.K % a.splits) return cudaErrorInvalidValue;
   const int ntiles = (EPI == GEMV_SWIGLU) ? a.N / 8 : (EPI == GEMV_CONV ? D / 16 : a.N / 16);
   const int NT = a.rows <= 8 ? 1 : 2;
-  const size_t smem = ws_smem<EPI, FP4>(NT, Kc);
+  WsArgs b = a;
+  b.stages = g_ws_stages > 0 ? g_ws_stages : G::STAGES;
+  const size_t smem = ws_smem<EPI, FP4>(NT, a.rows, Kc, b.stages);
   if (smem > (size_t)WS_SMEM_MAX) return cudaErrorInvalidValue;
-  // blocks per K range: about two per SM in all, spread evenly over the tiles
-  const int per_sm = smem <= 110 * 1024 ? 2 : 1;
-  int gx = std::max(1, per_sm * g_num_sms / a.splits);
+  // blocks per K range: g_ws_bps blocks per SM in all, spread evenly over the tiles
+  int gx = std::max(1, g_ws_bps * g_num_sms / a.splits);
   gx = std::min(gx, ntiles);
   const int per = (ntiles + gx - 1) / gx;
   gx = (ntiles + per - 1) / per;
   dim3 grid(gx, a.splits);
-  if (NT == 1) return launch(k_wstream<EPI, 1, FP4>, grid, dim3(WS_THREADS), smem, s, a);
-  return launch(k_wstream<EPI, 2, FP4>, grid, dim3(WS_THREADS), smem, s, a);
+  if (NT == 1) return launch(k_wstream<EPI, 1, FP4>, grid, dim3(WS_THREADS), smem, s, mp.w, mp.w3, mp.s, mp.s3, b);
+  return launch(k_wstream<EPI, 2, FP4>, grid, dim3(WS_THREADS), smem, s, mp.w, mp.w3, mp.s, mp.s3, b);
 }
 
-cudaError_t wstream(int epi, int nvfp4, const WsArgs& a, cudaStream_t s) {
+cudaError_t wstream(int epi, int nvfp4, const WsMaps& mp, const WsArgs& a, cudaStream_t s) {
   if (a.rows > 16 || a.rows < 1) return cudaErrorInvalidValue;
   switch (epi) {
-    case GEMV_PARTIAL: return nvfp4 ? launch_ws<GEMV_PARTIAL, true>(a, s) : launch_ws<GEMV_PARTIAL, false>(a, s);
-    case GEMV_SWIGLU: return nvfp4 ? launch_ws<GEMV_SWIGLU, true>(a, s) : launch_ws<GEMV_SWIGLU, false>(a, s);
-    case GEMV_CONV: return launch_ws<GEMV_CONV, false>(a, s);
-    case GEMV_HEAD: return launch_ws<GEMV_HEAD, false>(a, s);
+    case GEMV_PARTIAL: return nvfp4 ? launch_ws<GEMV_PARTIAL, true>(mp, a, s) : launch_ws<GEMV_PARTIAL, false>(mp, a, s);
+    case GEMV_SWIGLU: return nvfp4 ? launch_ws<GEMV_SWIGLU, true>(mp, a, s) : launch_ws<GEMV_SWIGLU, false>(mp, a, s);
+    case GEMV_CONV: return launch_ws<GEMV_CONV, false>(mp, a, s);
+    case GEMV_HEAD: return launch_ws<GEMV_HEAD, false>(mp, a, s);
   }
   return cudaErrorInvalidValue;
 }
+
+// Weight maps: a bf16 matrix [N][K] seen as {32 elements, N rows, K/32 blocks} (an NVFP4 code
+// matrix [N][K/2] as {64 bytes, N rows, K/128 blocks}), so that one box {., br rows, stage K}
+// lands as [block][row][64 B] - rows 64 B apart, which the lane pattern reads without bank
+// conflicts; NVFP4 scales [N][K/16] as a plain 2-D box {K-chunk/16, br}.
+static PFN_cuTensorMapEncodeTiled_v12000 p_enc_ws = nullptr;
+
+static bool ws_encoder() {
+  if (p_enc_ws) return true;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return false;
+  p_enc_ws = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return true;
+}
+
+bool make_ws_map(CUtensorMap* m, const void* w, int N, int K, int fp4, int br, int kch) {
+  if (!ws_encoder()) return false;
+  const int eb = fp4 ? 64 : 32;        // elements per 64-byte block (bytes of codes, or bf16)
+  const int kpb = fp4 ? 128 : 32;      // K per block
+  cuuint64_t dims[3] = {(cuuint64_t)eb, (cuuint64_t)N, (cuuint64_t)(K / kpb)};
+  cuuint64_t strides[2] = {(cuuint64_t)(fp4 ? K / 2 : K * 2), 64};
+  cuuint32_t box[3] = {(cuuint32_t)eb, (cuuint32_t)br, (cuuint32_t)(kch / kpb)};
+  cuuint32_t es[3] = {1, 1, 1};
+  return p_enc_ws(m, fp4 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(w), dims,
+                  strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_ws_scale_map(CUtensorMap* m, const void* sc, int N, int K, int br, int kch) {
+  if (!ws_encoder()) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N};
+  cuuint64_t strides[1] = {(cuuint64_t)(K / 16)};
+  cuuint32_t box[2] = {(cuuint32_t)(kch / 16), (cuuint32_t)br};
+  cuuint32_t es[2] = {1, 1};
+  return p_enc_ws(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(sc), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int ws_kch(int epi, int fp4) { return fp4 ? 512 : (epi == GEMV_CONV ? 256 : 512); }
+int ws_br(int epi) { return epi == GEMV_SWIGLU ? 8 : 16; }
 
 template <int EPI, bool FP4>
 static cudaError_t ws_attr() {
@@ -456,6 +541,8 @@ static cudaError_t ws_attr() {
 }
 
 cudaError_t wstream_init() {
+  if (const char* v = getenv("LFM3_WS_BLOCKS_PER_SM")) g_ws_bps = std::max(1, atoi(v));
+  if (const char* v = getenv("LFM3_WS_STAGES")) g_ws_stages = std::max(2, std::min(16, atoi(v)));
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

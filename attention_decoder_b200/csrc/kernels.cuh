@@ -104,8 +104,16 @@ struct WsArgs {
   const bf16* conv_w; bf16* conv_state; const int32_t* row_slot; bf16* y;  // CONV
   unsigned long long* amax; float* logits;         // HEAD (logits may be null)
   int* err;
+  int stages;                                      // set by the launcher
 };
-cudaError_t wstream(int epi, int nvfp4, const WsArgs& a, cudaStream_t s);
+struct WsMaps {
+  CUtensorMap w, w3, s, s3;  // weights (SwiGLU: w1, w3) or NVFP4 codes; NVFP4 scales
+};
+bool make_ws_map(CUtensorMap* m, const void* w, int N, int K, int fp4, int br, int kch);
+bool make_ws_scale_map(CUtensorMap* m, const void* sc, int N, int K, int br, int kch);
+int ws_kch(int epi, int fp4);
+int ws_br(int epi);
+cudaError_t wstream(int epi, int nvfp4, const WsMaps& mp, const WsArgs& a, cudaStream_t s);
 cudaError_t wstream_init();
 
 // ---------------------------------------------------------------- attention
@@ -126,6 +134,21 @@ cudaError_t attn_init();
 cudaError_t attn_static_scratch(float** ptr, size_t* nfloats);
 cudaError_t attn_prefill(const bf16* q, int n, int p0, int slot, AttnLayer L, const bf16* sk, const bf16* sv,
                          int scratch_rows, const float* gate, bf16* y, cudaStream_t s);
+
+// Prefill attention on tcgen05: maps over q [rows][16][128] and K/V stores viewed as [rows][128].
+struct AttnTcArgs {
+  int n, p0, slot, full, row0;
+  const int32_t* page_table;
+  int max_pages, scratch_rows;
+  const float* gate;
+  bf16* y;
+  int* err;
+};
+cudaError_t attn_tc_init();
+bool make_tmap_q(CUtensorMap* m, const void* q, uint64_t rows);
+bool make_tmap_kv(CUtensorMap* m, const void* base, uint64_t rows);
+cudaError_t attn_prefill_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnTcArgs& a,
+                            cudaStream_t s);
 
 // ---------------------------------------------------------------- tensor-core GEMM (prefill)
 enum GemmEpi { GEMM_F32 = 0, GEMM_BF16 = 1, GEMM_SWIGLU = 2 };

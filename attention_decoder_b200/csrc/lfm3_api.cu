@@ -22,7 +22,8 @@ constexpr int SPLIT_DD = 2, SPLIT_W2 = 5, SPLIT_MAX = 8;
 constexpr int GEMV_MAX_ROWS = 16;
 
 struct LayerPlan {
-  GemmPlan in_proj, out_proj, qkvg, o_proj, w13, w2;
+  GemmPlan in_proj, out_proj, qkvg, o_proj, w13, w2;   // prefill (tensor-core GEMM)
+  WsMaps ws_in, ws_out, ws_qkvg, ws_o, ws_w13, ws_w2;  // decode (weight streaming)
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -62,6 +63,9 @@ struct lfm3_ctx {
   bf16* deq = nullptr;
   std::vector<LayerPlan> plans;
   GemmPlan deq_w13, deq_w2;  // NVFP4: maps over the dequantised weights (b, b3)
+  CUtensorMap tm_q, tm_sk, tm_sv;  // prefill attention: q rows, sliding scratch K / V
+  WsMaps ws_head;                  // decode: tied head
+  bool attn_tc = true;             // prefill attention on tcgen05 (LFM3_ATTN_MMA=1: warp MMA)
   std::string msg;
   int launches = 0;
   // decode-step CUDA graphs, keyed by batch, split count and every device pointer the step reads
@@ -231,13 +235,13 @@ double gemm_bytes(const GemmPlan& p, int M) {
   return 2.0 * nw * p.N * (double)p.K + 2.0 * M * p.K + (p.epi == GEMM_F32 ? 4.0 : 2.0) * M * p.N;
 }
 
-cudaError_t run_ws(lfm3_ctx* c, int epi, int fp4, const WsArgs& a, cudaStream_t s) {
+cudaError_t run_ws(lfm3_ctx* c, int epi, int fp4, const WsMaps& mp, const WsArgs& a, cudaStream_t s) {
   const double mats = (a.w3 || a.codes3) ? 2.0 : 1.0;
   const double rows = epi == GEMV_CONV ? 3.0 * D : (double)a.N;
   const double w = fp4 ? rows * a.K / 2 + rows * a.K / 16 : 2.0 * rows * a.K;
   const double bytes = mats * w + 2.0 * a.rows * a.K + 4.0 * a.rows * a.N;
   Bracket b(c, s, bytes, 2.0 * a.rows * rows * a.K * mats);
-  return wstream(epi, fp4, a, s);
+  return wstream(epi, fp4, mp, a, s);
 }
 cudaError_t run_gemm(lfm3_ctx* c, const GemmPlan& p, int M, cudaStream_t s) {
   Bracket b(c, s, gemm_bytes(p, M), gemm_flops(p, M));
@@ -395,6 +399,7 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
   CK(wstream_init());
   CK(gemm_init());
   CK(attn_init());
+  CK(attn_tc_init());
   layout(ctx, reinterpret_cast<char*>(d_ws));
   const lfm3_config& g = ctx->cfg;
   const int R = ctx->R;
@@ -435,6 +440,49 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
     }
     if (!ok) return fail(ctx, LFM3_E_CUDA, "layer %d: tensor map encoding failed", l);
   }
+  // decode weight-streaming maps
+  for (int l = 0; l < g.n_layers; ++l) {
+    const lfm3_layer_weights& W = ctx->L[l];
+    LayerPlan& P = ctx->plans[l];
+    bool ok = true;
+    auto bf = [&](CUtensorMap* m, const void* w, int N, int K, int epi) {
+      ok &= make_ws_map(m, w, N, K, 0, ws_br(epi), ws_kch(epi, 0));
+    };
+    if (g.layer_type[l] == LFM3_LAYER_CONV) {
+      bf(&P.ws_in.w, W.in_proj, 3 * D, D, GEMV_CONV);
+      bf(&P.ws_out.w, W.out_proj, D, D, GEMV_PARTIAL);
+      P.ws_in.w3 = P.ws_in.s = P.ws_in.s3 = P.ws_in.w;
+      P.ws_out.w3 = P.ws_out.s = P.ws_out.s3 = P.ws_out.w;
+    } else {
+      bf(&P.ws_qkvg.w, W.qkvg, NQKVG, D, GEMV_PARTIAL);
+      bf(&P.ws_o.w, W.o_proj, D, HQ * HD, GEMV_PARTIAL);
+      P.ws_qkvg.w3 = P.ws_qkvg.s = P.ws_qkvg.s3 = P.ws_qkvg.w;
+      P.ws_o.w3 = P.ws_o.s = P.ws_o.s3 = P.ws_o.w;
+    }
+    if (g.ffn_format == LFM3_FFN_NVFP4) {
+      const int kch = ws_kch(GEMV_PARTIAL, 1);
+      ok &= make_ws_map(&P.ws_w13.w, W.w1_codes, F, D, 1, ws_br(GEMV_SWIGLU), kch);
+      ok &= make_ws_map(&P.ws_w13.w3, W.w3_codes, F, D, 1, ws_br(GEMV_SWIGLU), kch);
+      ok &= make_ws_scale_map(&P.ws_w13.s, W.w1_scales, F, D, ws_br(GEMV_SWIGLU), kch);
+      ok &= make_ws_scale_map(&P.ws_w13.s3, W.w3_scales, F, D, ws_br(GEMV_SWIGLU), kch);
+      ok &= make_ws_map(&P.ws_w2.w, W.w2_codes, D, F, 1, ws_br(GEMV_PARTIAL), kch);
+      ok &= make_ws_scale_map(&P.ws_w2.s, W.w2_scales, D, F, ws_br(GEMV_PARTIAL), kch);
+      P.ws_w2.w3 = P.ws_w2.w;
+      P.ws_w2.s3 = P.ws_w2.s;
+    } else {
+      bf(&P.ws_w13.w, W.w1, F, D, GEMV_SWIGLU);
+      bf(&P.ws_w13.w3, W.w3, F, D, GEMV_SWIGLU);
+      bf(&P.ws_w2.w, W.w2, D, F, GEMV_PARTIAL);
+      P.ws_w13.s = P.ws_w13.s3 = P.ws_w13.w;
+      P.ws_w2.w3 = P.ws_w2.s = P.ws_w2.s3 = P.ws_w2.w;
+    }
+    if (!ok) return fail(ctx, LFM3_E_CUDA, "layer %d: weight-streaming tensor map encoding failed", l);
+  }
+  if (g.has_head) {
+    if (!make_ws_map(&ctx->ws_head.w, ctx->embed, g.vocab, D, 0, ws_br(GEMV_HEAD), ws_kch(GEMV_HEAD, 0)))
+      return fail(ctx, LFM3_E_CUDA, "head weight-streaming tensor map encoding failed");
+    ctx->ws_head.w3 = ctx->ws_head.s = ctx->ws_head.s3 = ctx->ws_head.w;
+  }
   if (g.ffn_format == LFM3_FFN_NVFP4) {
     bool ok = plan_gemm(&ctx->deq_w13, GEMM_SWIGLU, ctx->xn, R, ctx->deq, ctx->deq + (size_t)F * D, F, D, ctx->big, F, 1.f);
     ok &= plan_gemm(&ctx->deq_w2, GEMM_F32, ctx->big, R, ctx->deq, nullptr, D, F, ctx->part, D, 1.f);
@@ -442,6 +490,11 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
   }
   CK(cudaDeviceSynchronize());
   ctx->graphs_on = getenv("LFM3_NO_GRAPH") == nullptr;
+  ctx->attn_tc = getenv("LFM3_ATTN_MMA") == nullptr;
+  if (!make_tmap_q(&ctx->tm_q, ctx->q, (uint64_t)R) ||
+      !make_tmap_kv(&ctx->tm_sk, ctx->sk, (uint64_t)HKV * ctx->scratch_rows) ||
+      !make_tmap_kv(&ctx->tm_sv, ctx->sv, (uint64_t)HKV * ctx->scratch_rows))
+    return fail(ctx, LFM3_E_CUDA, "attention tensor map encoding failed");
   ctx->bound = true;
   ctx->msg.clear();
   return LFM3_OK;
@@ -502,8 +555,30 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
         const int k = full ? 0 : 1;
         CK(qk_norm_rope_kv(ctx->part, 1, 0, B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], rows, eps,
                            ctx->q, ctx->gate, kw, s));
-        CK(attn_prefill(ctx->q, nc, p0, slot, attn_layer(ctx, st, l, v), ctx->sk, ctx->sv, ctx->scratch_rows,
-                        ctx->gate, ctx->y, s));
+        if (ctx->attn_tc) {
+          CUtensorMap tk, tv;
+          if (full) {
+            const uint64_t rows = (uint64_t)g.n_pages * HKV * PAGE;
+            if (!make_tmap_kv(&tk, v.kv_k, rows) || !make_tmap_kv(&tv, v.kv_v, rows))
+              return fail(ctx, LFM3_E_CUDA, "layer %d: K/V pool tensor map encoding failed", l);
+          }
+          AttnTcArgs ta{};
+          ta.n = nc;
+          ta.p0 = p0;
+          ta.slot = slot;
+          ta.full = full;
+          ta.row0 = 0;
+          ta.page_table = st->page_table;
+          ta.max_pages = g.max_pages_per_stream;
+          ta.scratch_rows = ctx->scratch_rows;
+          ta.gate = ctx->gate;
+          ta.y = ctx->y;
+          ta.err = ctx->err;
+          CK(attn_prefill_tc(ctx->tm_q, full ? tk : ctx->tm_sk, full ? tv : ctx->tm_sv, ta, s));
+        } else {
+          CK(attn_prefill(ctx->q, nc, p0, slot, attn_layer(ctx, st, l, v), ctx->sk, ctx->sv, ctx->scratch_rows,
+                          ctx->gate, ctx->y, s));
+        }
         if (!full)
           CK(scratch_to_ring(ctx->sk, ctx->sv, ctx->scratch_rows, nc, p0, v.ring_k, v.ring_v, slot, g.max_streams, s));
         CK(run_gemm(ctx, P.o_proj, nc, s));
@@ -528,7 +603,7 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
       a.logits = d_logits;
       a.amax = ctx->amax;
       a.err = ctx->err;
-      CK(run_ws(ctx, GEMV_HEAD, 0, a, s));
+      CK(run_ws(ctx, GEMV_HEAD, 0, ctx->ws_head, a, s));
     }
     CK(finish_step(st->seq_len, ctx->row_slot, nc, nc, slot, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
   }
@@ -610,7 +685,7 @@ lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, co
       a.logits = d_logits ? d_logits + (size_t)b0 * g.vocab : nullptr;
       a.amax = ctx->amax + b0;
       a.err = ctx->err;
-      CK(run_ws(ctx, GEMV_HEAD, 0, a, s));
+      CK(run_ws(ctx, GEMV_HEAD, 0, ctx->ws_head, a, s));
     }
   }
   CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
@@ -667,7 +742,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       c.row_slot = ctx->row_slot;
       c.y = ctx->y;
       norm_in(c, B(W.op_norm), dump_l);
-      CK(run_ws(ctx, GEMV_CONV, 0, c, s));
+      CK(run_ws(ctx, GEMV_CONV, 0, ctx->plans[l].ws_in, c, s));
       advance();
       WsArgs o{};
       base(o, D, D, SPLIT_DD);
@@ -675,7 +750,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       o.x = ctx->y;
       o.w = B(W.out_proj);
       o.part_out = ctx->part;
-      CK(run_ws(ctx, GEMV_PARTIAL, 0, o, s));
+      CK(run_ws(ctx, GEMV_PARTIAL, 0, ctx->plans[l].ws_out, o, s));
     } else {
       const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
       WsArgs q{};
@@ -683,7 +758,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       q.w = B(W.qkvg);
       q.part_out = ctx->part3;
       norm_in(q, B(W.op_norm), dump_l);
-      CK(run_ws(ctx, GEMV_PARTIAL, 0, q, s));
+      CK(run_ws(ctx, GEMV_PARTIAL, 0, ctx->plans[l].ws_qkvg, q, s));
       advance();
       KvWrite kw{};
       kw.mode = full ? KV_PAGES : KV_RING;
@@ -703,7 +778,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       o.x = ctx->y;
       o.w = B(W.o_proj);
       o.part_out = ctx->part;
-      CK(run_ws(ctx, GEMV_PARTIAL, 0, o, s));
+      CK(run_ws(ctx, GEMV_PARTIAL, 0, ctx->plans[l].ws_o, o, s));
     }
     pend = ctx->part;
     pend_n = SPLIT_DD;
@@ -719,7 +794,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       f.w3 = B(W.w3);
     }
     norm_in(f, B(W.ffn_norm), nullptr);
-    CK(run_ws(ctx, GEMV_SWIGLU, fp4, f, s));
+    CK(run_ws(ctx, GEMV_SWIGLU, fp4, ctx->plans[l].ws_w13, f, s));
     advance();
     WsArgs d{};
     base(d, F, D, SPLIT_W2);
@@ -731,7 +806,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
     } else {
       d.w = B(W.w2);
     }
-    CK(run_ws(ctx, GEMV_PARTIAL, fp4, d, s));
+    CK(run_ws(ctx, GEMV_PARTIAL, fp4, ctx->plans[l].ws_w2, d, s));
     pend = ctx->part2;
     pend_n = SPLIT_W2;
     pend_g = B(W.post_ffn_norm);
@@ -745,7 +820,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
     h.logits = d_logits;
     h.amax = ctx->amax;
     norm_in(h, ctx->final_norm, dump_last);
-    CK(run_ws(ctx, GEMV_HEAD, 0, h, s));
+    CK(run_ws(ctx, GEMV_HEAD, 0, ctx->ws_head, h, s));
     advance();
   } else if (dump_last) {
     CK(resid_norm(cur, pend, pend_n, (long)nb * D, pend_g, nullptr, nullptr, nb, eps, dump_last, s));

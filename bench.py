@@ -218,6 +218,8 @@ def run_ours(args):
         o = model.prefill(st, 0, tokens=prompt)
         return st, o
 
+    if args.only == "prefill":
+        return run_prefill_only(args, world, m, g, stream, clocks, Wm)
     st, o = fresh_state(m)
     bufs = {"argmax": o["argmax"].clone(), "logits": torch.empty(1, g.vocab, device="cuda")}
     slots_d = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -269,7 +271,7 @@ def run_ours(args):
     e2e_ms = max_over_ranks(world, e0.elapsed_time(e1))
 
     # prefill 8k (chunks of 2048) over shuffled pages
-    if not args.no_extra:
+    if not args.no_extra and args.only is None:
         n8 = 8192
         mp = Lfm3Model(make_weights(g, 0), max_streams=1, max_pages_per_stream=n8 // 64, max_batch=1)
         pt = page_permutation(1, "pages8k", n8 // 64).reshape(1, -1)
@@ -300,7 +302,7 @@ def run_ours(args):
     torch.cuda.empty_cache()
 
     # ---------------- NVFP4 FFN model: decode at 1 / 8 streams (2048 ctx) and 64 streams
-    if not args.no_extra:
+    if not args.no_extra and args.only is None:
         Wq = make_weights(g, 0, ffn="nvfp4")
         S = 64
         ctx64 = context_lengths(1, "ctx64", S, 256, 8192)
@@ -381,6 +383,35 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_prefill_only(args, world, m, g, stream, clocks, Wm):
+    """Profiling leg: the 8192-token prompt pass (chunks of 2048, shuffled pages), timed."""
+    import torch
+    from lfm3_inputs import make_tokens, page_permutation
+    del m
+    torch.cuda.empty_cache()
+    from attention_decoder_b200.model import Lfm3Model
+    from lfm3_inputs import make_weights
+    n8 = 8192
+    mp = Lfm3Model(make_weights(g, 0), max_streams=1, max_pages_per_stream=n8 // 64, max_batch=1)
+    pt = page_permutation(1, "pages8k", n8 // 64).reshape(1, -1)
+    tok8 = torch.from_numpy(make_tokens(1, "prompt8k", n8, g.vocab)).cuda()
+    st = mp.new_state(page_table=pt)
+
+    def pstep():
+        st.h_seq_len[:] = 0
+        st.seq_len.zero_()
+        mp.prefill(st, 0, tokens=tok8)
+
+    for _ in range(Wm):
+        pstep()
+    K = max(1, args.steps)
+    ms = timed(world, pstep, K, stream)
+    clk = clocks.stop()
+    if int(os.environ.get("RANK", "0")) == 0:
+        print(json.dumps({"profiling_case": "prefill 8k", "ms": ms / K, "tok_s": n8 * K / (ms / 1e3),
+                          "launches_per_prefill": mp.last_launch_count(), "clocks": clk}), flush=True)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -410,6 +441,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="headline decode only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--small", action="store_true", help="4-layer profiling case (not a bench line)")
+    ap.add_argument("--only", choices=["decode", "prefill"], default=None,
+                    help="profiling: run only the bf16 decode or only the 8k prefill leg")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
