@@ -116,6 +116,56 @@ int ws_br(int epi);
 cudaError_t wstream(int epi, int nvfp4, const WsMaps& mp, const WsArgs& a, cudaStream_t s);
 cudaError_t wstream_init();
 
+// ---------------------------------------------------------------- persistent decode step
+constexpr int MK_MAX_NB = 4;   // streams one persistent step serves
+constexpr int MK_MAPS = 8;     // weight tensor maps per layer (the head's map follows the last layer)
+constexpr int MK_TRACE_PHASES = 256;  // phase stamps kept per block when profiling
+constexpr int MK_TRACE_BLOCKS = 160;
+constexpr int MK_TRACE_WORDS = 8;     // per phase: start, finish, data wait, last copy, prologue done, first copy
+struct MkLayer {
+  int type, kidx;                  // LFM3 layer type; index among the layers of that type
+  const bf16 *op_norm, *post_op_norm, *ffn_norm, *post_ffn_norm;
+  const bf16 *conv_w, *q_norm, *k_norm;
+  float w13_scale, w2_scale;       // NVFP4 tensor scales
+};
+// Fixed at bind: model, weight maps (device arrays) and workspace buffers.
+struct MkModel {
+  int n_layers, has_head, fp4, vocab, max_pages, max_streams, n_pages, nslot;
+  int pf;                          // stages prefetched into L2 ahead of the shared-memory loads
+  float eps;
+  const MkLayer* layers;
+  const CUtensorMap* maps;         // [n_layers * MK_MAPS + 1]
+  const bf16* embed;
+  const bf16* final_norm;
+  const float* rope_cos[2];
+  const float* rope_sin[2];
+  float *x_res, *x_res2, *part, *part2, *part3;
+  bf16 *y, *u;
+  unsigned long long* amax;
+  unsigned* sync;                  // [0] grid barrier, [1] exit count, [16..] attention merge counts
+  int* err;
+  unsigned long long* trace;       // null, or [block][MK_TRACE_PHASES][MK_TRACE_WORDS] stamps (ns)
+};
+// Per step.
+struct MkStep {
+  int nb;
+  const int32_t* slots;
+  const int32_t* tokens;
+  const bf16* embeds;
+  float* logits;
+  int32_t* argmax_out;
+  float* hidden;
+  int32_t* seq_len;
+  const int32_t* page_table;
+  bf16 *conv_state, *kv_k, *kv_v, *ring_k, *ring_v;
+  float* attn_part;
+  int attn_splits;                 // split stride of attn_part
+};
+cudaError_t mk_init();
+int mk_grid();  // blocks of one persistent launch (the SM count)
+// kv_maps: full-layer K, V pools and sliding-layer K, V rings, each viewed as [rows][128] bf16.
+cudaError_t decode_mk(const CUtensorMap* kv_maps, const MkModel& m, const MkStep& s, cudaStream_t st);
+
 // ---------------------------------------------------------------- attention
 constexpr int DEC_KEYS_FULL = 128;  // keys per decode split on full layers
 constexpr int DEC_KEYS_RING = 64;   // ring slots per decode split on sliding layers

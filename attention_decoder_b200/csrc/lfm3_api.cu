@@ -66,6 +66,16 @@ struct lfm3_ctx {
   CUtensorMap tm_q, tm_sk, tm_sv;  // prefill attention: q rows, sliding scratch K / V
   WsMaps ws_head;                  // decode: tied head
   bool attn_tc = true;             // prefill attention on tcgen05 (LFM3_ATTN_MMA=1: warp MMA)
+  // persistent decode step (up to MK_MAX_NB streams; opt-in with LFM3_PERSISTENT=1)
+  MkLayer* mk_layers = nullptr;    // workspace: per-layer table
+  CUtensorMap* mk_maps = nullptr;  // workspace: weight maps
+  unsigned* mk_sync = nullptr;     // workspace: barrier and merge counters
+  unsigned long long* mk_trace = nullptr;  // workspace: phase stamps while profiling
+  int mk_last_phases = 0;          // phases of the last persistent step, if it was stamped
+  int mk_last_head = 0;
+  MkModel mk{};
+  bool mk_on = false;
+  double mk_wbytes = 0;            // weight bytes one step streams
   std::string msg;
   int launches = 0;
   // decode-step CUDA graphs, keyed by batch, split count and every device pointer the step reads
@@ -127,7 +137,7 @@ size_t layout(lfm3_ctx* c, char* base) {
   // fp32 projection outputs: the conv in_proj [R][3D], qkvg [R][3088], or decode K-split partials
   c->part = reinterpret_cast<float*>(take(4 * std::max(R * 3 * D, (size_t)SPLIT_MAX * g.max_batch * NQKVG)));
   c->part2 = reinterpret_cast<float*>(take(4 * (size_t)SPLIT_MAX * g.max_batch * D));
-  c->part3 = reinterpret_cast<float*>(take(4 * (size_t)g.max_batch * NQKVG));
+  c->part3 = reinterpret_cast<float*>(take(4 * (size_t)2 * g.max_batch * NQKVG));  // two K halves (persistent step)
   c->q = reinterpret_cast<bf16*>(take(2 * R * HQ * HD));
   c->gate = reinterpret_cast<float*>(take(4 * R * HQ));
   c->sk = reinterpret_cast<bf16*>(take(2 * (size_t)HKV * c->scratch_rows * HD));
@@ -138,6 +148,10 @@ size_t layout(lfm3_ctx* c, char* base) {
     c->rope_sin[k] = reinterpret_cast<float*>(take(4 * (size_t)c->max_pos * (HD / 2)));
   }
   c->deq = g.ffn_format == LFM3_FFN_NVFP4 ? reinterpret_cast<bf16*>(take(2 * (size_t)2 * F * D)) : nullptr;
+  c->mk_layers = reinterpret_cast<MkLayer*>(take(sizeof(MkLayer) * (size_t)g.n_layers));
+  c->mk_maps = reinterpret_cast<CUtensorMap*>(take(sizeof(CUtensorMap) * ((size_t)g.n_layers * MK_MAPS + 1)));
+  c->mk_sync = reinterpret_cast<unsigned*>(take(256));
+  c->mk_trace = reinterpret_cast<unsigned long long*>(take(8 * (size_t)MK_TRACE_WORDS * MK_TRACE_BLOCKS * MK_TRACE_PHASES));
   return align_up(off, 256);
 }
 
@@ -354,6 +368,152 @@ lfm3_status ffn_gemm(lfm3_ctx* ctx, int l, int n, cudaStream_t s) {
   return LFM3_OK;
 }
 
+// Persistent decode step: per-layer table and weight maps in the workspace, counters zeroed.
+lfm3_status bind_persistent(lfm3_ctx* ctx) {
+  const lfm3_config& g = ctx->cfg;
+  const bool fp4 = g.ffn_format == LFM3_FFN_NVFP4;
+  std::vector<MkLayer> layers(g.n_layers);
+  std::vector<CUtensorMap> maps((size_t)g.n_layers * MK_MAPS + 1);
+  std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
+  double wbytes = 0;
+  for (int l = 0; l < g.n_layers; ++l) {
+    const lfm3_layer_weights& W = ctx->L[l];
+    MkLayer& M = layers[l];
+    M = MkLayer{};
+    M.type = g.layer_type[l];
+    M.kidx = ctx->kidx[l];
+    M.op_norm = B(W.op_norm);
+    M.post_op_norm = B(W.post_op_norm);
+    M.ffn_norm = B(W.ffn_norm);
+    M.post_ffn_norm = B(W.post_ffn_norm);
+    M.conv_w = B(W.conv);
+    M.q_norm = B(W.q_norm);
+    M.k_norm = B(W.k_norm);
+    M.w13_scale = W.w13_scale;
+    M.w2_scale = W.w2_scale;
+    CUtensorMap* lm = maps.data() + (size_t)l * MK_MAPS;
+    bool ok = true;
+    if (M.type == LFM3_LAYER_CONV) {
+      ok &= make_ws_map(lm + 0, W.in_proj, 3 * D, D, 0, 16, 256);
+      ok &= make_ws_map(lm + 1, W.out_proj, D, D, 0, 16, 1024);
+      wbytes += 2.0 * 4 * D * D;
+    } else {
+      ok &= make_ws_map(lm + 0, W.qkvg, NQKVG, D, 0, 16, 1024);
+      ok &= make_ws_map(lm + 1, W.o_proj, D, HQ * HD, 0, 16, 1024);
+      wbytes += 2.0 * (NQKVG + D) * D;
+    }
+    if (fp4) {
+      ok &= make_ws_map(lm + 2, W.w1_codes, F, D, 1, 8, 2048);
+      ok &= make_ws_map(lm + 3, W.w3_codes, F, D, 1, 8, 2048);
+      ok &= make_ws_map(lm + 4, W.w2_codes, D, F, 1, 16, 2560);
+      ok &= make_ws_scale_map(lm + 5, W.w1_scales, F, D, 8, 2048);
+      ok &= make_ws_scale_map(lm + 6, W.w3_scales, F, D, 8, 2048);
+      ok &= make_ws_scale_map(lm + 7, W.w2_scales, D, F, 16, 2560);
+      wbytes += 3.0 * ((double)F * D / 2 + (double)F * D / 16);
+    } else {
+      ok &= make_ws_map(lm + 2, W.w1, F, D, 0, 8, 1024);
+      ok &= make_ws_map(lm + 3, W.w3, F, D, 0, 8, 1024);
+      ok &= make_ws_map(lm + 4, W.w2, D, F, 0, 16, 960);
+      wbytes += 2.0 * 3 * F * D;
+    }
+    if (!ok) return fail(ctx, LFM3_E_CUDA, "layer %d: persistent-step tensor map encoding failed", l);
+  }
+  if (g.has_head) {
+    if (!make_ws_map(maps.data() + (size_t)g.n_layers * MK_MAPS, ctx->embed, g.vocab, D, 0, 16, 1024))
+      return fail(ctx, LFM3_E_CUDA, "persistent-step head tensor map encoding failed");
+  }
+  CK(cudaMemcpy(ctx->mk_layers, layers.data(), layers.size() * sizeof(MkLayer), cudaMemcpyHostToDevice));
+  CK(cudaMemcpy(ctx->mk_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
+  CK(cudaMemset(ctx->mk_sync, 0, 256));
+  MkModel& m = ctx->mk;
+  m = MkModel{};
+  m.n_layers = g.n_layers;
+  m.has_head = g.has_head;
+  m.fp4 = fp4;
+  m.vocab = g.vocab;
+  m.max_pages = g.max_pages_per_stream;
+  m.max_streams = g.max_streams;
+  m.n_pages = g.n_pages;
+  m.eps = g.eps;
+  m.pf = 12;
+  if (const char* v = getenv("LFM3_MK_PREFETCH")) m.pf = std::max(0, std::min(64, atoi(v)));
+  m.layers = ctx->mk_layers;
+  m.maps = ctx->mk_maps;
+  m.embed = ctx->embed;
+  m.final_norm = ctx->final_norm;
+  for (int k = 0; k < 2; ++k) {
+    m.rope_cos[k] = ctx->rope_cos[k];
+    m.rope_sin[k] = ctx->rope_sin[k];
+  }
+  m.x_res = ctx->x_res;
+  m.x_res2 = ctx->x_res2;
+  m.part = ctx->part;
+  m.part2 = ctx->part2;
+  m.part3 = ctx->part3;
+  m.y = ctx->y;
+  m.u = ctx->big;
+  m.amax = ctx->amax;
+  m.sync = ctx->mk_sync;
+  m.err = ctx->err;
+  ctx->mk_wbytes = wbytes;
+  return LFM3_OK;
+}
+
+bool use_persistent(const lfm3_ctx* ctx, int nb) { return ctx->mk_on && nb <= MK_MAX_NB; }
+
+// One decode step as a single persistent launch (see k_decode_mk.cu).
+lfm3_status enqueue_decode_mk(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* h_slots,
+                              const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds, float* d_logits,
+                              int32_t* d_argmax, float* d_hidden, int splits_full, float* attn_part, cudaStream_t s) {
+  const lfm3_config& g = ctx->cfg;
+  CUtensorMap kv[4];
+  const void* dummy = ctx->rope_cos[0];  // any mapped buffer of >= 64 rows of 256 bytes; never read
+  const uint64_t full_rows = (uint64_t)ctx->n_full * g.n_pages * HKV * PAGE;
+  const uint64_t ring_rows = (uint64_t)ctx->n_sliding * g.max_streams * HKV * WIN;
+  bool ok = true;
+  ok &= make_tmap_kv(&kv[0], ctx->n_full ? st->kv_k : dummy, ctx->n_full ? full_rows : 64);
+  ok &= make_tmap_kv(&kv[1], ctx->n_full ? st->kv_v : dummy, ctx->n_full ? full_rows : 64);
+  ok &= make_tmap_kv(&kv[2], ctx->n_sliding ? st->ring_k : dummy, ctx->n_sliding ? ring_rows : 64);
+  ok &= make_tmap_kv(&kv[3], ctx->n_sliding ? st->ring_v : dummy, ctx->n_sliding ? ring_rows : 64);
+  if (!ok) return fail(ctx, LFM3_E_CUDA, "key/value tensor map encoding failed");
+  MkStep S{};
+  S.nb = nb;
+  S.slots = d_slots;
+  S.tokens = g.has_head ? d_tokens : nullptr;
+  S.embeds = B(d_embeds);
+  S.logits = d_logits;
+  S.argmax_out = d_argmax;
+  S.hidden = d_hidden;
+  S.seq_len = st->seq_len;
+  S.page_table = st->page_table;
+  S.conv_state = reinterpret_cast<bf16*>(st->conv_state);
+  S.kv_k = reinterpret_cast<bf16*>(st->kv_k);
+  S.kv_v = reinterpret_cast<bf16*>(st->kv_v);
+  S.ring_k = reinterpret_cast<bf16*>(st->ring_k);
+  S.ring_v = reinterpret_cast<bf16*>(st->ring_v);
+  S.attn_part = attn_part;
+  S.attn_splits = std::max(splits_full, WIN / DEC_KEYS_RING);
+  // algorithmic bytes of the step: every weight once, plus the cached keys and values read
+  double kvb = 0;
+  for (int b = 0; b < nb; ++b) {
+    const double pos = (double)st->h_seq_len[h_slots[b]];
+    kvb += 2.0 * 2 * HKV * HD * (ctx->n_full * (pos + 1) + ctx->n_sliding * std::min(pos + 1, (double)WIN));
+  }
+  const double head = (g.has_head && (d_logits || d_argmax)) ? 2.0 * g.vocab * D : 0.0;
+  MkModel mm = ctx->mk;
+  mm.trace = ctx->prof ? ctx->mk_trace : nullptr;
+  ctx->mk_last_phases = 0;
+  if (ctx->prof) {
+    for (int l = 0; l < g.n_layers; ++l) ctx->mk_last_phases += g.layer_type[l] == LFM3_LAYER_CONV ? 4 : 5;
+    ctx->mk_last_head = head > 0;
+    ctx->mk_last_phases += ctx->mk_last_head;
+  }
+  if (mm.trace) CK(cudaMemsetAsync(ctx->mk_trace, 0, 8 * (size_t)MK_TRACE_WORDS * MK_TRACE_BLOCKS * MK_TRACE_PHASES, s));
+  Bracket br(ctx, s, ctx->mk_wbytes + head + kvb, 0.0);
+  CK(decode_mk(kv, mm, S, s));
+  return LFM3_OK;
+}
+
 }  // namespace
 
 // ======================================================================================== ABI
@@ -400,6 +560,7 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
   CK(gemm_init());
   CK(attn_init());
   CK(attn_tc_init());
+  CK(mk_init());
   layout(ctx, reinterpret_cast<char*>(d_ws));
   const lfm3_config& g = ctx->cfg;
   const int R = ctx->R;
@@ -488,8 +649,13 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
     ok &= plan_gemm(&ctx->deq_w2, GEMM_F32, ctx->big, R, ctx->deq, nullptr, D, F, ctx->part, D, 1.f);
     if (!ok) return fail(ctx, LFM3_E_CUDA, "NVFP4 tensor map encoding failed");
   }
+  {
+    lfm3_status ms = bind_persistent(ctx);
+    if (ms != LFM3_OK) return ms;
+  }
   CK(cudaDeviceSynchronize());
   ctx->graphs_on = getenv("LFM3_NO_GRAPH") == nullptr;
+  ctx->mk_on = getenv("LFM3_PERSISTENT") != nullptr;
   ctx->attn_tc = getenv("LFM3_ATTN_MMA") == nullptr;
   if (!make_tmap_q(&ctx->tm_q, ctx->q, (uint64_t)R) ||
       !make_tmap_kv(&ctx->tm_sk, ctx->sk, (uint64_t)HKV * ctx->scratch_rows) ||
@@ -885,7 +1051,12 @@ extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int
   if (vs != LFM3_OK) return vs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   g_launches = 0;
-  if (!ctx->graphs_on || ctx->prof) {
+  if (use_persistent(ctx, nb)) {
+    lfm3_status es = enqueue_decode_mk(ctx, st, nb, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax,
+                                       d_hidden, splits_full, ctx->attn_part, s);
+    if (es != LFM3_OK) return es;
+    ctx->launches = g_launches;
+  } else if (!ctx->graphs_on || ctx->prof) {
     lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
                                     splits_full, ctx->attn_part, s);
     if (es != LFM3_OK) return es;
@@ -951,8 +1122,12 @@ extern "C" lfm3_status lfm3_decode_step_noalloc(lfm3_ctx* ctx, const lfm3_state*
                 nb, splits_full, need * sizeof(float), cap * sizeof(float));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   g_launches = 0;
-  lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
-                                  splits_full, scratch, s);
+  lfm3_status es =
+      use_persistent(ctx, nb)
+          ? enqueue_decode_mk(ctx, st, nb, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                              splits_full, scratch, s)
+          : enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden, splits_full,
+                           scratch, s);
   if (es != LFM3_OK) return es;
   ctx->launches = g_launches;
   for (int b = 0; b < nb; ++b) st->h_seq_len[h_slots[b]] += 1;
@@ -967,6 +1142,7 @@ extern "C" lfm3_status lfm3_check_device_errors(lfm3_ctx* ctx, void* stream) {
   CK(cudaMemcpy(&e, ctx->err, sizeof e, cudaMemcpyDeviceToHost));
   if (e) {
     CK(cudaMemset(ctx->err, 0, sizeof e));
+    CK(cudaMemset(ctx->mk_sync, 0, 256));  // a persistent step that gave up left its counters mid-way
     return fail(ctx, LFM3_E_TIMEOUT, "a device-side bounded wait gave up (status %d)", e);
   }
   return LFM3_OK;
@@ -1005,6 +1181,77 @@ extern "C" lfm3_status lfm3_profile_read(lfm3_ctx* ctx, int* launches, double* m
   const int over = ctx->ev_overflow;
   ctx->ev_used = ctx->ev_overflow = 0;
   if (over) return fail(ctx, LFM3_E_CAPACITY, "%d launches ran unbracketed (capacity exceeded)", over);
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_profile_phases(lfm3_ctx* ctx, void* stream, int cap, int* n_phases, int* kind,
+                                           double* span_us, double* work_us, double* work_max_us, double* wait_us,
+                                           double* lead_us, double* prologue_us, double* ahead_us) {
+  if (!ctx || !n_phases) return LFM3_E_ARG;
+  *n_phases = 0;
+  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
+  if (!ctx->prof || ctx->mk_last_phases == 0)
+    return fail(ctx, LFM3_E_STATE, "no stamped persistent decode step (profiling off, or another path ran)");
+  const int G = mk_grid();
+  if (G > MK_TRACE_BLOCKS) return fail(ctx, LFM3_E_UNSUPPORTED, "%d blocks exceed the stamp table", G);
+  CK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  std::vector<unsigned long long> t((size_t)G * MK_TRACE_PHASES * MK_TRACE_WORDS);
+  CK(cudaMemcpy(t.data(), ctx->mk_trace, t.size() * 8, cudaMemcpyDeviceToHost));
+  const lfm3_config& g = ctx->cfg;
+  std::vector<int> kinds;
+  for (int l = 0; l < g.n_layers; ++l) {
+    if (g.layer_type[l] == LFM3_LAYER_CONV) kinds.insert(kinds.end(), {0, 3, 4, 5});
+    else kinds.insert(kinds.end(), {1, 2, 3, 4, 5});
+  }
+  if (ctx->mk_last_head) kinds.push_back(6);
+  const int n = std::min({(int)kinds.size(), cap, MK_TRACE_PHASES});
+  for (int p = 0; p < n; ++p) {
+    unsigned long long lo = ~0ull, hi = 0;
+    double sum = 0, mx = 0, wsum = 0, lsum = 0, psum = 0, asum = 0;
+    int ln = 0, an = 0;
+    for (int b = 0; b < G; ++b) {
+      const unsigned long long* r = t.data() + ((size_t)b * MK_TRACE_PHASES + p) * MK_TRACE_WORDS;
+      const unsigned long long a = r[0], e = r[1];
+      lo = std::min(lo, a);
+      hi = std::max(hi, e);
+      const double w = e > a ? (e - a) * 1e-3 : 0.0;
+      sum += w;
+      mx = std::max(mx, w);
+      wsum += r[2] * 1e-3;
+      if (r[3] && e > r[3]) {
+        lsum += (e - r[3]) * 1e-3;
+        ++ln;
+      }
+      if (r[4] > a) psum += (r[4] - a) * 1e-3;
+      if (r[5]) {
+        asum += ((double)a - (double)r[5]) * 1e-3;
+        ++an;
+      }
+    }
+    if (prologue_us) prologue_us[p] = psum / G;
+    if (ahead_us) ahead_us[p] = an ? asum / an : 0.0;
+    if (wait_us) wait_us[p] = wsum / G;
+    if (lead_us) lead_us[p] = ln ? lsum / ln : 0.0;
+    if (kind) kind[p] = kinds[p];
+    if (span_us) span_us[p] = hi > lo ? (hi - lo) * 1e-3 : 0.0;
+    if (work_us) work_us[p] = sum / G;
+    if (work_max_us) work_max_us[p] = mx;
+  }
+  *n_phases = n;
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_profile_stamps(lfm3_ctx* ctx, void* stream, uint64_t* out, size_t cap, int* n_blocks) {
+  if (!ctx || !out || !n_blocks) return LFM3_E_ARG;
+  *n_blocks = 0;
+  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
+  if (!ctx->prof || ctx->mk_last_phases == 0)
+    return fail(ctx, LFM3_E_STATE, "no stamped persistent decode step (profiling off, or another path ran)");
+  const int G = std::min(mk_grid(), MK_TRACE_BLOCKS);
+  CK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  const size_t n = std::min(cap, (size_t)G * MK_TRACE_PHASES * MK_TRACE_WORDS);
+  CK(cudaMemcpy(out, ctx->mk_trace, n * 8, cudaMemcpyDeviceToHost));
+  *n_blocks = G;
   return LFM3_OK;
 }
 

@@ -348,6 +348,10 @@ def run_ours(args):
         del mq, stq
     clk = clocks.stop()
 
+    if launches_per_step == 1:
+        kkey, kname = "k_decode_mk", "k_decode_mk (persistent decode step: every weight + cached K/V once)"
+    else:
+        kkey, kname = "k_wstream", "k_wstream (decode weight-streaming projections)"
     tok_s_rank = res["decode_b1"]["tok_s"]
     value = world * tok_s_rank
     hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -359,11 +363,11 @@ def run_ours(args):
                                 "(prefilled), tied 128000 head") if not args.small else
                                "profiling case: 4-layer LFM3 slice + head, bf16 decode, 256-token context",
                    "streams_per_gpu": 1, "context": ctx0,
-                   "l2": "no flush: each step streams 3.46 GB of weights, > 126 MB L2",
+                   "l2": "no flush: each step streams %.2f GB of weights and K/V, > 126 MB L2" % (step_bytes / 1e9),
                    "parallelism": "replicas" if world > 1 else "single GPU"},
-        "roofline": {"bound": "hbm", "kernel": "k_gemv (decode weight-streaming projections)",
+        "roofline": {"bound": "hbm", "kernel": kname,
                      "achieved": round(gemv_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gemv_gbs / hbm, 4),
-                     "peak_kind": pk_kind, "traffic": traffic_record("k_gemv"),
+                     "peak_kind": pk_kind, "traffic": traffic_record(kkey),
                      "bytes_per_step": round(step_bytes), "kernel_launches_timed": prof["launches"]},
         "e2e": {"value": round(world * K / (e2e_ms / 1e3), 2), "unit": "tok/s", "h2d_bytes_per_step": 4,
                 "d2h_bytes_per_step": 4},

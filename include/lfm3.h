@@ -210,6 +210,29 @@ lfm3_status lfm3_profile_enable(lfm3_ctx* ctx, int on, int capacity);
  * excess launches ran unbracketed). */
 lfm3_status lfm3_profile_read(lfm3_ctx* ctx, int* launches, double* ms, double* bytes, double* flops);
 
+/* Phase timing of the persistent decode step (the one-launch step lfm3_decode_step uses for up
+ * to 4 streams). While profiling is enabled each block of that launch stamps the device clock
+ * (ns) when it starts a phase and when it has finished its share of it, into the workspace.
+ * After a decode step, this synchronises the stream and, for each phase p < *n_phases (at most
+ * `cap`), writes: kind[p] (0 conv in_proj+conv, 1 q|k|v|gate, 2 attention, 3 out/o_proj,
+ * 4 w1|w3, 5 w2, 6 head), span_us[p] (first start to last finish over the blocks), work_us[p]
+ * (mean over blocks of finish - start), work_max_us[p], wait_us[p] (mean over blocks of the
+ * time the first consumer warp waited for streamed data) and lead_us[p] (mean over blocks of
+ * the time from the block's last copy issue in the phase to its finish), prologue_us[p] (mean
+ * time spent on the phase's input step before its units) and ahead_us[p] (mean over blocks of
+ * how long before the phase started the block's first copy for it was issued). Any output array
+ * may be NULL. Returns LFM3_E_STATE if profiling is off or the last decode step did not run as
+ * one persistent launch. */
+lfm3_status lfm3_profile_phases(lfm3_ctx* ctx, void* stream, int cap, int* n_phases, int* kind, double* span_us,
+                                double* work_us, double* work_max_us, double* wait_us, double* lead_us,
+                                double* prologue_us, double* ahead_us);
+
+/* The raw stamps behind lfm3_profile_phases: synchronises the stream and copies up to `cap`
+ * uint64 words laid out [block][256 phases][8] (device clock, ns; 0 = not stamped): phase
+ * start, finish, first warp's data wait, last copy issued, input step done, first copy issued,
+ * sandwich loads in, sandwich done. *n_blocks receives the number of blocks. */
+lfm3_status lfm3_profile_stamps(lfm3_ctx* ctx, void* stream, uint64_t* out, size_t cap, int* n_blocks);
+
 /* Number of kernels the last prefill/decode call enqueued. */
 int lfm3_last_launch_count(const lfm3_ctx* ctx);
 
