@@ -186,6 +186,212 @@ cudaError_t attn_decode(const bf16* q, Rows rows, AttnLayer L, int splits, float
   return launch(k_attn_merge, dim3(rows.n, HQ), dim3(HD), 0, s, part, splits, gate, y);
 }
 
+// ------------------------------------------------------------------------------------------ decode, one kernel
+// Decode attention of one layer in one launch, from the raw q|k|v|gate projection (fp32, one row
+// per stream): block (split, kv head, stream) normalises and rotates its four query heads and
+// the head's new key (RMS over the head, gain, rotary pairs (i, i + 64), bf16) and rounds the
+// new value; it scores its key range with the new key and value standing in for the current
+// position's cache row, which the block holding that position also writes. The cached rows are
+// staged before the block waits for the projection kernel (they do not depend on it). The last
+// block of a (stream, kv head) to finish - counted with an atomic - merges the splits, applies
+// the sigmoid gate and writes the bf16 output, then resets the count for the next layer.
+__global__ void __launch_bounds__(128) k_attn_decode_fused(const float* __restrict__ qkvg, Rows rows, AttnLayer L,
+                                                           AttnDecodeArgs A, int splits, float* __restrict__ part,
+                                                           bf16* __restrict__ y) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  bf16* ks = reinterpret_cast<bf16*>(dsm);
+  bf16* vs = ks + DEC_SPLIT * HD;
+  __shared__ float qs[GQA][HD];
+  __shared__ float kn[HD], vn[HD];
+  __shared__ float sc[GQA][DEC_SPLIT];
+  __shared__ float ored[2][GQA][HD];
+  __shared__ float ml[GQA][2];
+  __shared__ float red[GQA + 1][4];
+  __shared__ int last;
+  const int sp = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int slot = rows.slot[b], pos = rows.pos[b];
+  const int span = L.full ? DEC_SPLIT : DEC_SPLIT_RING;
+  const int nkeys = L.full ? pos + 1 : min(pos + 1, WIN);  // ring: slots 0..nkeys-1 are live
+  const int cur = L.full ? pos : pos % WIN;                 // index of the current position's key
+  const int j0 = sp * span, j1 = min(nkeys, j0 + span), cnt = j1 - j0;
+  auto row_ptr = [&](const bf16* base, int j) -> const bf16* {
+    if (L.full) {
+      const int page = L.page_table[(size_t)slot * L.max_pages + j / PAGE];
+      return base + (((size_t)page * HKV + kvh) * PAGE + j % PAGE) * HD;
+    }
+    return base + (((size_t)slot * HKV + kvh) * WIN + j) * HD;
+  };
+  // ---- stage the cached keys / values of the split (all but the current position)
+  for (int e = tid; e < max(cnt, 0) * 16; e += blockDim.x) {
+    const int r = e >> 4, c = e & 15;
+    if (j0 + r == cur) continue;
+    const uint32_t kd = (uint32_t)__cvta_generic_to_shared(ks + krot(r, c));
+    const uint32_t vd = (uint32_t)__cvta_generic_to_shared(vs + r * HD + c * 8);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(kd), "l"(row_ptr(L.k, j0 + r) + c * 8));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vd), "l"(row_ptr(L.v, j0 + r) + c * 8));
+  }
+  asm volatile("cp.async.commit_group;");
+  // gains and rotary coefficients of this thread's dimension d = tid are weights too
+  const int d = tid, pd = d < 64 ? d + 64 : d - 64, ir = d & 63;
+  const float gq = bf2f(A.q_norm[d]), gk = bf2f(A.k_norm[d]);
+  const float cr = A.rope_cos[(size_t)pos * (HD / 2) + ir], sr = A.rope_sin[(size_t)pos * (HD / 2) + ir];
+  pdl_wait();
+  pdl_launch_dependents();
+  // ---- queries and the new key / value: thread = dimension d of each of the 4 heads
+  const float* raw = qkvg + (size_t)b * NQKVG;
+  float qv[GQA], s2[GQA + 1];
+#pragma unroll
+  for (int hh = 0; hh < GQA; ++hh) {
+    qv[hh] = raw[(kvh * GQA + hh) * HD + d];
+    s2[hh] = warp_sum(qv[hh] * qv[hh]);
+  }
+  const float kv = raw[HQ * HD + kvh * HD + d];
+  const float vv = raw[HQ * HD + HKV * HD + kvh * HD + d];
+  s2[GQA] = warp_sum(kv * kv);
+  if (lane == 0)
+#pragma unroll
+    for (int hh = 0; hh <= GQA; ++hh) red[hh][warp] = s2[hh];
+  __syncthreads();
+#pragma unroll
+  for (int hh = 0; hh < GQA; ++hh) {
+    const float inv = rsqrtf((red[hh][0] + red[hh][1] + red[hh][2] + red[hh][3]) * (1.0f / HD) + A.eps);
+    qs[hh][d] = gq * (qv[hh] * inv);
+  }
+  kn[d] = gk * (kv * rsqrtf((red[GQA][0] + red[GQA][1] + red[GQA][2] + red[GQA][3]) * (1.0f / HD) + A.eps));
+  vn[d] = round_bf(vv);
+  __syncthreads();
+  const float scale = rsqrtf((float)HD);
+  float qr[GQA];
+#pragma unroll
+  for (int hh = 0; hh < GQA; ++hh) qr[hh] = d < 64 ? qs[hh][d] * cr - qs[hh][pd] * sr : qs[hh][d] * cr + qs[hh][pd] * sr;
+  const float kr = d < 64 ? kn[d] * cr - kn[pd] * sr : kn[d] * cr + kn[pd] * sr;
+  __syncthreads();
+#pragma unroll
+  for (int hh = 0; hh < GQA; ++hh) qs[hh][d] = round_bf(qr[hh]) * scale;
+  kn[d] = round_bf(kr);
+  const bool has_cur = cur >= j0 && cur < j1;
+  if (has_cur) {  // the new key and value into the cache (bf16, as every later step reads them)
+    bf16* kd = const_cast<bf16*>(row_ptr(L.k, cur));
+    bf16* vd = const_cast<bf16*>(row_ptr(L.v, cur));
+    kd[d] = f2bf(kn[d]);
+    vd[d] = f2bf(vn[d]);
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  float* out = part + (((size_t)b * HQ + kvh * GQA) * splits + sp) * (HD + 2);
+  if (cnt > 0) {
+    // scores: one key per thread (span <= 128)
+    if (tid < cnt) {
+      float s[GQA] = {0.f, 0.f, 0.f, 0.f};
+      if (j0 + tid == cur) {
+        for (int c = 0; c < HD; ++c)
+#pragma unroll
+          for (int hh = 0; hh < GQA; ++hh) s[hh] += qs[hh][c] * kn[c];
+      } else {
+#pragma unroll 4
+        for (int c = 0; c < 16; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(ks + krot(tid, c));
+          const float k8[8] = {bflo(w.x), bfhi(w.x), bflo(w.y), bfhi(w.y), bflo(w.z), bfhi(w.z), bflo(w.w), bfhi(w.w)};
+#pragma unroll
+          for (int hh = 0; hh < GQA; ++hh)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s[hh] += qs[hh][c * 8 + e] * k8[e];
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < GQA; ++hh) sc[hh][tid] = s[hh];
+    }
+    __syncthreads();
+    {
+      const int hh = warp;
+      float mx = -INFINITY;
+      for (int j = lane; j < cnt; j += 32) mx = fmaxf(mx, sc[hh][j]);
+      mx = warp_max(mx);
+      float l = 0.f;
+      for (int j = lane; j < cnt; j += 32) {
+        const float p = __expf(sc[hh][j] - mx);
+        sc[hh][j] = p;
+        l += p;
+      }
+      l = warp_sum(l);
+      if (lane == 0) { ml[hh][0] = mx; ml[hh][1] = l; }
+    }
+    __syncthreads();
+    {
+      const int par = tid >> 6, dp = (tid & 63) * 2;
+      float o[GQA][2] = {};
+#pragma unroll 4
+      for (int j = par; j < cnt; j += 2) {
+        float v0, v1;
+        if (j0 + j == cur) {
+          v0 = vn[dp];
+          v1 = vn[dp + 1];
+        } else {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(vs + j * HD + dp);
+          v0 = bflo(w);
+          v1 = bfhi(w);
+        }
+#pragma unroll
+        for (int hh = 0; hh < GQA; ++hh) {
+          const float p = sc[hh][j];
+          o[hh][0] += p * v0;
+          o[hh][1] += p * v1;
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < GQA; ++hh) { ored[par][hh][dp] = o[hh][0]; ored[par][hh][dp + 1] = o[hh][1]; }
+    }
+    __syncthreads();
+    for (int e = tid; e < GQA * HD; e += blockDim.x) {
+      const int hh = e / HD, dd = e % HD;
+      out[(size_t)hh * splits * (HD + 2) + dd] = ored[0][hh][dd] + ored[1][hh][dd];
+    }
+    if (tid < GQA) {
+      out[(size_t)tid * splits * (HD + 2) + HD] = ml[tid][0];
+      out[(size_t)tid * splits * (HD + 2) + HD + 1] = ml[tid][1];
+    }
+  } else {  // empty split
+    for (int e = tid; e < GQA * (HD + 2); e += blockDim.x) {
+      const int hh = e / (HD + 2), k = e % (HD + 2);
+      out[(size_t)hh * splits * (HD + 2) + k] = (k == HD) ? -INFINITY : 0.f;
+    }
+  }
+  // ---- the last block of (stream, kv head) merges the splits and applies the gates
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    unsigned* ctr = A.counters + b * HKV + kvh;
+    last = atomicAdd(ctr, 1u) == (unsigned)(splits - 1);
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int hh = 0; hh < GQA; ++hh) {
+    const float* pp = part + ((size_t)b * HQ + kvh * GQA + hh) * splits * (HD + 2);
+    float M = -INFINITY, l = 0.f, o = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float* q = pp + (size_t)s * (HD + 2);
+      const float ms = __ldcg(q + HD), ls = __ldcg(q + HD + 1), os = __ldcg(q + d);
+      if (ms == -INFINITY) continue;
+      const float Mn = fmaxf(M, ms);
+      const float fo = __expf(M - Mn), fs = __expf(ms - Mn);
+      l = l * fo + ls * fs;
+      o = o * fo + os * fs;
+      M = Mn;
+    }
+    const float gt = sigmoidf_(raw[HQ * HD + 2 * HKV * HD + kvh * GQA + hh]);
+    y[(size_t)b * HQ * HD + (kvh * GQA + hh) * HD + d] = f2bf(gt * (o / l));
+  }
+  if (tid == 0) A.counters[b * HKV + kvh] = 0u;
+}
+
+cudaError_t attn_decode_fused(const float* qkvg, Rows rows, AttnLayer L, const AttnDecodeArgs& A, int splits,
+                              float* part, bf16* y, cudaStream_t s) {
+  return launch(k_attn_decode_fused, dim3(splits, HKV, rows.n), dim3(128), DEC_SMEM, s, qkvg, rows, L, A, splits, part,
+                y);
+}
+
 // ------------------------------------------------------------------------------------------ prefill
 constexpr int PA_ROWS = 32;        // query rows per block
 constexpr int PA_KT = 64;          // keys per tile
@@ -413,6 +619,8 @@ cudaError_t attn_prefill(const bf16* q, int n, int p0, int slot, AttnLayer L, co
 
 cudaError_t attn_init() {
   cudaError_t e = cudaFuncSetAttribute(k_attn_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_attn_decode_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(k_attn_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, 4 * PA_TILE_BYTES);
 }

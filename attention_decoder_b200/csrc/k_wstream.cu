@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
   float* red = reinterpret_cast<float*>(stages + (size_t)NS * G::STAGE_BYTES);
   float* res = red + WS_CW * NRT * NT * 128;
   uint64_t* bars = reinterpret_cast<uint64_t*>(res + NRT * 16 * NT * 8);
-  __shared__ float redn[WS_CW];
+  __shared__ __align__(16) float redn[WS_CW * 4];
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -207,9 +207,24 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
   }
 
   // -------------------------------------------------------------- consumers: prologue
+  const int ct = tid;  // 0..127
+  // the norm gains are weights: requested before waiting for the previous kernel
+  float gp[16], gn[16];
+  if (a.pro == WS_PRO_NORM) {
+    const int c0 = ct * 16;
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+    const uint4 p0 = a.n_parts > 0 ? ldg16(a.g_post + c0) : z4, p1 = a.n_parts > 0 ? ldg16(a.g_post + c0 + 8) : z4;
+    const uint4 n0 = ldg16(a.g_next + c0), n1 = ldg16(a.g_next + c0 + 8);
+    const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    const uint32_t nw[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      gp[2 * j] = bflo(pw[j]); gp[2 * j + 1] = bfhi(pw[j]);
+      gn[2 * j] = bflo(nw[j]); gn[2 * j + 1] = bfhi(nw[j]);
+    }
+  }
   pdl_wait();
   pdl_launch_dependents();
-  const int ct = tid;  // 0..127
   if (ct < 8) reinterpret_cast<uint4*>(smem)[ct] = make_uint4(0, 0, 0, 0);
   if constexpr (FP4) {
     for (int i = ct; i < 256 * 32; i += WS_CW * 32) {
@@ -224,71 +239,73 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
       *reinterpret_cast<uint4*>(xs + (size_t)b * XS + c * 8) = ldg16(a.x + (size_t)b * a.K + kcta + c * 8);
     }
   } else {
-    // residual + post-norm of the previous projection, then this projection's input norm
+    // residual + post-norm of the previous projection, then this projection's input norm. The
+    // gains are requested first (HBM round trips), then each stream's residual and partials; one
+    // reduction per stream gives both norms: with a = RMS^-1 of the partials' sum m and the post
+    // gain g, x' = x + a g m and sum(x'^2) = sum(x^2) + 2a sum(g x m) + a^2 sum(g^2 m^2).
     const bool writer = blockIdx.x == 0 && blockIdx.y == 0;
+    const int c0 = ct * 16;
     for (int b = 0; b < a.rows; ++b) {
-      float x[16];
-      const float* xin = a.x_in + (size_t)b * D + ct * 16;
+      float x[16], m[16];
+      const float* xin = a.x_in + (size_t)b * D + c0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float4 v = reinterpret_cast<const float4*>(xin)[q];
         x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
       }
-      if (a.n_parts > 0) {
-        float m[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) m[j] = 0.f;
-        for (int s = 0; s < a.n_parts; ++s) {
-          const float* p = a.parts + s * a.part_stride + (size_t)b * D + ct * 16;
+      for (int j = 0; j < 16; ++j) m[j] = 0.f;
+      for (int s = 0; s < a.n_parts; ++s) {
+        const float* p = a.parts + s * a.part_stride + (size_t)b * D + c0;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + q);
-            m[4 * q] += v.x; m[4 * q + 1] += v.y; m[4 * q + 2] += v.z; m[4 * q + 3] += v.w;
-          }
+        for (int q = 0; q < 4; ++q) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + q);
+          m[4 * q] += v.x; m[4 * q + 1] += v.y; m[4 * q + 2] += v.z; m[4 * q + 3] += v.w;
         }
-        float ss = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) ss += m[j] * m[j];
-        ss = warp_sum(ss);
-        if (lane == 0) redn[warp] = ss;
-        consumers_sync();
-        ss = redn[0] + redn[1] + redn[2] + redn[3];
-        consumers_sync();
-        const float inv = rsqrtf(ss * (1.0f / D) + a.eps);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) x[j] += bf2f(a.g_post[ct * 16 + j]) * (m[j] * inv);
       }
+      float q4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float gm = gp[j] * m[j];
+        q4[0] += m[j] * m[j];
+        q4[1] += x[j] * x[j];
+        q4[2] += x[j] * gm;
+        q4[3] += gm * gm;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) q4[c] = warp_sum(q4[c]);
+      if (lane == 0) *reinterpret_cast<float4*>(redn + 4 * warp) = make_float4(q4[0], q4[1], q4[2], q4[3]);
+      consumers_sync();
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int w = 0; w < WS_CW; ++w)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) t[c] += redn[4 * w + c];
+      const float al = a.n_parts > 0 ? rsqrtf(t[0] * (1.0f / D) + a.eps) : 0.f;
+      const float inv = rsqrtf(fmaxf(t[1] + 2.f * al * t[2] + al * al * t[3], 0.f) * (1.0f / D) + a.eps);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x[j] += al * (gp[j] * m[j]);
       if (writer) {
-        float* xo = a.x_out + (size_t)b * D + ct * 16;
+        float* xo = a.x_out + (size_t)b * D + c0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) reinterpret_cast<float4*>(xo)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
         if (a.dump) {
-          float* dd = a.dump + (size_t)b * D + ct * 16;
+          float* dd = a.dump + (size_t)b * D + c0;
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             reinterpret_cast<float4*>(dd)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
         }
       }
-      float ss = 0.f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) ss += x[j] * x[j];
-      ss = warp_sum(ss);
-      if (lane == 0) redn[warp] = ss;
-      consumers_sync();
-      ss = redn[0] + redn[1] + redn[2] + redn[3];
-      consumers_sync();
-      const float inv = rsqrtf(ss * (1.0f / D) + a.eps);
       // this thread's 16 columns go to shared memory if they are in the block's K range
-      const int c0 = ct * 16;
       if (c0 >= kcta && c0 < kcta + Kc) {
         uint32_t w[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          w[j] = pack_bf2(bf2f(a.g_next[c0 + 2 * j]) * (x[2 * j] * inv), bf2f(a.g_next[c0 + 2 * j + 1]) * (x[2 * j + 1] * inv));
+        for (int j = 0; j < 8; ++j) w[j] = pack_bf2(gn[2 * j] * (x[2 * j] * inv), gn[2 * j + 1] * (x[2 * j + 1] * inv));
         uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)b * XS + (c0 - kcta));
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
+      consumers_sync();  // redn is reused by the next stream
     }
   }
   consumers_sync();

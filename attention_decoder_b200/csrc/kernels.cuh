@@ -179,6 +179,17 @@ cudaError_t attn_decode(const bf16* q, Rows rows, AttnLayer L, int splits, float
                         bf16* y, cudaStream_t s);
 // Prefill attention for the n rows of one slot starting at position p0.
 //  full: keys through the page table; sliding: keys in scratch [HKV][scratch_rows][HD], index i <-> p0-WIN+i
+// Decode attention in one launch from the raw q|k|v|gate rows (see k_attn_decode_fused).
+struct AttnDecodeArgs {
+  const bf16* q_norm;
+  const bf16* k_norm;
+  const float* rope_cos;   // [pos][64] of this layer kind
+  const float* rope_sin;
+  float eps;
+  unsigned* counters;      // [streams][HKV], zero between calls
+};
+cudaError_t attn_decode_fused(const float* qkvg, Rows rows, AttnLayer L, const AttnDecodeArgs& A, int splits,
+                              float* part, bf16* y, cudaStream_t s);
 cudaError_t attn_init();
 // Device address and size (floats) of the library's fixed attention scratch on the current device.
 cudaError_t attn_static_scratch(float** ptr, size_t* nfloats);

@@ -70,6 +70,7 @@ struct lfm3_ctx {
   MkLayer* mk_layers = nullptr;    // workspace: per-layer table
   CUtensorMap* mk_maps = nullptr;  // workspace: weight maps
   unsigned* mk_sync = nullptr;     // workspace: barrier and merge counters
+  unsigned* attn_cnt = nullptr;    // workspace: decode attention split counts [max_batch][n_kv]
   unsigned long long* mk_trace = nullptr;  // workspace: phase stamps while profiling
   int mk_last_phases = 0;          // phases of the last persistent step, if it was stamped
   int mk_last_head = 0;
@@ -151,6 +152,7 @@ size_t layout(lfm3_ctx* c, char* base) {
   c->mk_layers = reinterpret_cast<MkLayer*>(take(sizeof(MkLayer) * (size_t)g.n_layers));
   c->mk_maps = reinterpret_cast<CUtensorMap*>(take(sizeof(CUtensorMap) * ((size_t)g.n_layers * MK_MAPS + 1)));
   c->mk_sync = reinterpret_cast<unsigned*>(take(256));
+  c->attn_cnt = reinterpret_cast<unsigned*>(take(4 * (size_t)g.max_batch * HKV));
   c->mk_trace = reinterpret_cast<unsigned long long*>(take(8 * (size_t)MK_TRACE_WORDS * MK_TRACE_BLOCKS * MK_TRACE_PHASES));
   return align_up(off, 256);
 }
@@ -425,6 +427,7 @@ lfm3_status bind_persistent(lfm3_ctx* ctx) {
   CK(cudaMemcpy(ctx->mk_layers, layers.data(), layers.size() * sizeof(MkLayer), cudaMemcpyHostToDevice));
   CK(cudaMemcpy(ctx->mk_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
   CK(cudaMemset(ctx->mk_sync, 0, 256));
+  CK(cudaMemset(ctx->attn_cnt, 0, 4 * (size_t)g.max_batch * HKV));
   MkModel& m = ctx->mk;
   m = MkModel{};
   m.n_layers = g.n_layers;
@@ -926,18 +929,10 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       norm_in(q, B(W.op_norm), dump_l);
       CK(run_ws(ctx, GEMV_PARTIAL, 0, ctx->plans[l].ws_qkvg, q, s));
       advance();
-      KvWrite kw{};
-      kw.mode = full ? KV_PAGES : KV_RING;
-      kw.k = full ? v.kv_k : v.ring_k;
-      kw.v = full ? v.kv_v : v.ring_v;
-      kw.page_table = st->page_table;
-      kw.max_pages = g.max_pages_per_stream;
-      kw.max_streams = g.max_streams;
       const int k = full ? 0 : 1;
-      CK(qk_norm_rope_kv(ctx->part3, 1, 0, B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], rows, eps,
-                         ctx->q, ctx->gate, kw, s));
-      CK(attn_decode(ctx->q, rows, attn_layer(ctx, st, l, v), full ? splits_full : WIN / DEC_KEYS_RING, attn_part,
-                     ctx->gate, ctx->y, s));
+      AttnDecodeArgs A{B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], eps, ctx->attn_cnt};
+      CK(attn_decode_fused(ctx->part3, rows, attn_layer(ctx, st, l, v), A, full ? splits_full : WIN / DEC_KEYS_RING,
+                           attn_part, ctx->y, s));
       WsArgs o{};
       base(o, HQ * HD, D, SPLIT_DD);
       o.pro = WS_PRO_LOAD;
