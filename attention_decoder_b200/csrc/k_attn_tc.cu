@@ -4,7 +4,8 @@
 // rows are (row r, head j) with m = 4 r + j. Keys come in tiles of 128 (two 64-position pages of
 // a full layer, or 128 consecutive rows of a sliding layer's chunk scratch), K and V by TMA into a
 // two-stage ring. Per tile:
-//   warp 1 (one lane):  S = Q K^T      (tcgen05.mma kind::f16, 128 x 128 x 128, fp32 in TMEM)
+//   warp 1 (one lane):  S = Q K^T      (tcgen05.mma kind::f16, 128 x 128 x 128, fp32 in TMEM; two S
+//                       buffers, so the next tile's scores are computed during this tile's softmax)
 //   warps 2..5:         each thread owns one TMEM lane (= one row): read S, mask (causal, the
 //                       256-key window on sliding layers, written keys only), online softmax in
 //                       fp32 (exp2 with the 1/sqrt(128) scale folded in), write P as bf16 into a
@@ -111,7 +112,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   unsigned char* ps = vs + 2 * AT_KV_BYTES;                   // [2 key blocks][128 rows][128 B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(ps + AT_P_BYTES);
   const uint32_t q_full = su32(bars), kv_full0 = su32(bars + 1), kv_empty0 = su32(bars + 3);
-  const uint32_t s_full = su32(bars + 5), p_full = su32(bars + 6), o_done = su32(bars + 7);
+  // S is double-buffered in TMEM (columns 0..127 and 128..255, one full barrier each) so the next
+  // tile's Q K^T runs while the softmax works on this one; O lives in columns 256..383
+  const uint32_t s_full0 = su32(bars + 5), p_full = su32(bars + 6), o_done = su32(bars + 7);
+  const uint32_t s_full1 = su32(bars + 9);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -133,19 +137,20 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       mbar_init(kv_full0 + 8 * s, 1);
       mbar_init(kv_empty0 + 8 * s, 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(s_full0, 1);
+    mbar_init(s_full1, 1);
     mbar_init(p_full, 4);
     mbar_init(o_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)), "r"(256));
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)), "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   at_fence_before();
   __syncthreads();
   at_fence_after();
-  const uint32_t tmem = *tmem_slot;  // S: columns 0..127, O: columns 128..255
+  const uint32_t tmem = *tmem_slot;  // S: columns 0..127 / 128..255 by tile parity, O: 256..383
   pdl_wait();
   pdl_launch_dependents();
 
@@ -192,26 +197,35 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       constexpr uint32_t idesc_o = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(HD >> 3) << 17) |
                                    ((uint32_t)(AT_M >> 4) << 24);
       bool ok = mbar_wait(q_full, 0, a.err);
-      for (int j = 0; j < ntiles && ok; ++j) {
+      const uint32_t qb = su32(qs);
+      auto issue_s = [&](int j) -> bool {  // S(j) = Q K(j)^T into S buffer j & 1
         const int st = j & 1;
-        if (!mbar_wait(kv_full0 + 8 * st, (j >> 1) & 1, a.err)) break;
+        if (!mbar_wait(kv_full0 + 8 * st, (j >> 1) & 1, a.err)) return false;
         at_fence_after();
-        const uint32_t qb = su32(qs), kb = su32(ks + st * AT_KV_BYTES), vb = su32(vs + st * AT_KV_BYTES);
+        const uint32_t kb = su32(ks + st * AT_KV_BYTES);
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           const uint32_t off = (k >> 2) * (AT_Q_BYTES / 2) + (k & 3) * 32;
           const uint32_t koff_b = (k >> 2) * (AT_KV_BYTES / 2) + (k & 3) * 32;
-          at_mma(tmem, at_desc_k(qb + off), at_desc_k(kb + koff_b), idesc_s, k != 0);
+          at_mma(tmem + (uint32_t)st * 128, at_desc_k(qb + off), at_desc_k(kb + koff_b), idesc_s, k != 0);
         }
-        at_commit(s_full);
+        at_commit(st ? s_full1 : s_full0);
+        return true;
+      };
+      if (ok && ntiles > 0) ok = issue_s(0);
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int st = j & 1;
+        // the next tile's scores go into the other S buffer, whose last reader (the softmax of
+        // tile j - 1) finished before its P was handed over below
+        if (j + 1 < ntiles && !issue_s(j + 1)) break;
         if (!mbar_wait(p_full, j & 1, a.err)) break;
         at_fence_after();
-        const uint32_t pb = su32(ps);
+        const uint32_t pb = su32(ps), vb = su32(vs + st * AT_KV_BYTES);
 #pragma unroll
         for (int k = 0; k < AT_KT / 16; ++k) {
           const uint32_t poff = (k >> 2) * (AT_P_BYTES / 2) + (k & 3) * 32;   // P: K-major (keys)
           const uint32_t voff = k * 2048;                                      // V: 16 keys = 2 atoms
-          at_mma(tmem + 128, at_desc_k(pb + poff), at_desc_mn(vb + voff, AT_KV_BYTES / 2), idesc_o,
+          at_mma(tmem + 256, at_desc_k(pb + poff), at_desc_mn(vb + voff, AT_KV_BYTES / 2), idesc_o,
                  (j | k) != 0);
         }
         at_commit(o_done);
@@ -230,14 +244,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
       const int kt0 = klo + j * AT_KT;
-      if (!mbar_wait(s_full, j & 1, a.err)) { ok = false; break; }
+      if (!mbar_wait((j & 1) ? s_full1 : s_full0, (j >> 1) & 1, a.err)) { ok = false; break; }
       at_fence_after();
+      const uint32_t srow = trow + (uint32_t)(j & 1) * 128;  // this tile's S buffer
       // pass 1: masked row maximum
       float tmax = -INFINITY;
 #pragma unroll 1
       for (int c = 0; c < AT_KT / 32; ++c) {
         float v[32];
-        at_ld32(trow + c * 32, v);
+        at_ld32(srow + c * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int kp = kt0 + c * 32 + i + koff;
@@ -257,10 +272,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 #pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
           float o[32];
-          at_ld32(trow + 128 + c * 32, o);
+          at_ld32(trow + 256 + c * 32, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          at_st32(trow + 128 + c * 32, o);
+          at_st32(trow + 256 + c * 32, o);
         }
       }
       // pass 2: probabilities -> bf16 P tile (row m, 128-byte swizzle)
@@ -268,7 +283,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 #pragma unroll 1
       for (int c = 0; c < AT_KT / 32; ++c) {
         float v[32];
-        at_ld32(trow + c * 32, v);
+        at_ld32(srow + c * 32, v);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -321,7 +336,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
         float o[32];
-        at_ld32(trow + 128 + c * 32, o);
+        at_ld32(trow + 256 + c * 32, o);
         if (live) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
@@ -335,7 +350,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   at_fence_before();
   __syncthreads();
   at_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
 }
 
 constexpr size_t AT_SMEM = 1024 + AT_Q_BYTES + 4 * AT_KV_BYTES + AT_P_BYTES + 256;

@@ -213,36 +213,57 @@ cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot,
 // ------------------------------------------------------------------------------------------
 // Per-head q/k RMSNorm (gain of length 128 shared across heads), rotary on pairs (i, i+64) with
 // a per-position table (zero-tail pairs carry cos 1, sin 0), and placement of k/v.
-// Block = (row, head among q | k | v), 128 threads = head_dim.
-__global__ void __launch_bounds__(128) k_qk_norm_rope_kv(const float* __restrict__ part, int n_part,
+// One warp per (row, head slot): slots 0..15 are q heads, 16..19 k heads, 20..23 v heads. Lane l
+// holds dims l, l + 32, l + 64, l + 96, so each rotary pair (i, i + 64) sits in one lane; the head's
+// RMS is a warp sum. q (and k) are normalised, rotated and rounded to bf16; v is rounded; the gate
+// logits (q slots' lane 0) are summed over the partials.
+__global__ void __launch_bounds__(256) k_qk_norm_rope_kv(const float* __restrict__ part, int n_part,
                                                          long part_stride, const bf16* __restrict__ q_norm,
                                                          const bf16* __restrict__ k_norm,
                                                          const float* __restrict__ rope_cos,
                                                          const float* __restrict__ rope_sin, Rows rows, float eps,
                                                          bf16* __restrict__ q_out, float* __restrict__ gate_out,
                                                          KvWrite kv) {
-  __shared__ float red[4];
-  __shared__ float xs[HD];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x, hh = blockIdx.y * 8 + warp;  // head slot 0..23
+  // gains and rotary rows do not depend on the previous kernel
+  const bool qk = hh < HQ + HKV;
+  float gn[4] = {1.f, 1.f, 1.f, 1.f};
+  if (qk) {
+    const bf16* g = hh < HQ ? q_norm : k_norm;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) gn[k] = bf2f(g[lane + 32 * k]);
+  }
   pdl_wait();
   pdl_launch_dependents();
-  const int r = blockIdx.x, hh = blockIdx.y, i = threadIdx.x;
-  const int col0 = hh * HD;  // q heads, then k heads, then v heads are consecutive in qkvg
-  float x = 0.f;
-  for (int s = 0; s < n_part; ++s) x += part[s * part_stride + (size_t)r * NQKVG + col0 + i];
   const int pos = rows.pos[r];
-  if (hh < HQ + HKV) {
-    const bf16* g = hh < HQ ? q_norm : k_norm;
-    float ss = block_sum<4>(x * x, red);
-    x = bf2f(g[i]) * (x * rsqrtf(ss * (1.0f / HD) + eps));
-    xs[i] = x;
-    __syncthreads();
-    const int j = i & (HD / 2 - 1);
-    const float c = rope_cos[(size_t)pos * (HD / 2) + j], sn = rope_sin[(size_t)pos * (HD / 2) + j];
-    x = i < HD / 2 ? x * c - xs[i + HD / 2] * sn : x * c + xs[i - HD / 2] * sn;
+  const int col0 = hh * HD;  // q heads, then k heads, then v heads are consecutive in qkvg
+  float x[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < n_part; ++s) {
+    const float* p = part + s * part_stride + (size_t)r * NQKVG + col0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] += p[lane + 32 * k];
+  }
+  if (qk) {
+    const float ss = warp_sum(x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3]);
+    const float inv = rsqrtf(ss * (1.0f / HD) + eps);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] = gn[k] * (x[k] * inv);
+    // pairs (d, d + 64): dims lane + 32k for k = 0, 1 with k + 2
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = lane + 32 * k;
+      const float c = rope_cos[(size_t)pos * (HD / 2) + i], sn = rope_sin[(size_t)pos * (HD / 2) + i];
+      const float lo = x[k], hi = x[k + 2];
+      x[k] = lo * c - hi * sn;
+      x[k + 2] = hi * c + lo * sn;
+    }
   }
   if (hh < HQ) {
-    q_out[((size_t)r * HQ + hh) * HD + i] = f2bf(x);
-    if (i == 0) {
+    bf16* qo = q_out + ((size_t)r * HQ + hh) * HD;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) qo[lane + 32 * k] = f2bf(x[k]);
+    if (lane == 0) {
       float gsum = 0.f;
       for (int s = 0; s < n_part; ++s) gsum += part[s * part_stride + (size_t)r * NQKVG + HQ * HD + 2 * HKV * HD + hh];
       gate_out[r * HQ + hh] = gsum;
@@ -263,14 +284,15 @@ __global__ void __launch_bounds__(128) k_qk_norm_rope_kv(const float* __restrict
   } else {
     off = ((size_t)kvh * kv.scratch_rows + WIN + r) * HD;
   }
-  base[off + i] = f2bf(x);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) base[off + lane + 32 * k] = f2bf(x[k]);
 }
 
 cudaError_t qk_norm_rope_kv(const float* part, int n_part, long part_stride, const bf16* q_norm, const bf16* k_norm,
                             const float* rope_cos, const float* rope_sin, Rows rows, float eps, bf16* q_out,
                             float* gate_out, KvWrite kv, cudaStream_t s) {
-  return launch(k_qk_norm_rope_kv, dim3(rows.n, HQ + 2 * HKV), dim3(HD), 0, s, part, n_part, part_stride, q_norm,
-                k_norm, rope_cos, rope_sin, rows, eps, q_out, gate_out, kv);
+  return launch(k_qk_norm_rope_kv, dim3(rows.n, (HQ + 2 * HKV) / 8), dim3(256), 0, s, part, n_part, part_stride,
+                q_norm, k_norm, rope_cos, rope_sin, rows, eps, q_out, gate_out, kv);
 }
 
 // ------------------------------------------------------------------------------------------

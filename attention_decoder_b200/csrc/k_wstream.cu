@@ -52,7 +52,7 @@ struct WsGeom {
   static constexpr int REQB = 64 * BR * NKB;                  // bytes of one request: [block][row][64 B]
   static constexpr int ROWB = 64 * NKB;                       // weight bytes per row per stage
   static constexpr int SCB = FP4 ? KCH / 16 : 0;              // scale bytes per row per stage
-  static constexpr int STAGES = FP4 ? 12 : (NRT == 3 ? 3 : 6);  // default ring depth (runtime: a.stages)
+  static constexpr int STAGES = FP4 ? 12 : 5;  // default ring depth (runtime: a.stages); swept on B200
   static constexpr int STAGE_BYTES = RPT * ROWB + RPT * SCB;
   static constexpr int TX_BYTES = STAGE_BYTES;
   static constexpr int STEPS = KCH / KB;                      // lane steps per stage
