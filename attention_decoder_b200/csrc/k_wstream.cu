@@ -32,7 +32,8 @@
 
 namespace lfm3 {
 
-constexpr int WS_CW = 4;                    // consumer warps
+constexpr int WS_CW = 8;                    // consumer warps
+constexpr int WS_EPT = D / (WS_CW * 32);      // residual elements per consumer thread in the prologue
 // Largest dynamic shared memory a launch asks for (in_proj + conv with 16 streams: ~192 KB).
 constexpr int WS_SMEM_MAX = 200 * 1024;
 constexpr int WS_THREADS = 32 * (WS_CW + 1);
@@ -209,18 +210,19 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
   // -------------------------------------------------------------- consumers: prologue
   const int ct = tid;  // 0..127
   // the norm gains are weights: requested before waiting for the previous kernel
-  float gp[16], gn[16];
+  float gp[WS_EPT], gn[WS_EPT];
   if (a.pro == WS_PRO_NORM) {
-    const int c0 = ct * 16;
+    const int c0 = ct * WS_EPT;
     const uint4 z4 = make_uint4(0, 0, 0, 0);
-    const uint4 p0 = a.n_parts > 0 ? ldg16(a.g_post + c0) : z4, p1 = a.n_parts > 0 ? ldg16(a.g_post + c0 + 8) : z4;
-    const uint4 n0 = ldg16(a.g_next + c0), n1 = ldg16(a.g_next + c0 + 8);
-    const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-    const uint32_t nw[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      gp[2 * j] = bflo(pw[j]); gp[2 * j + 1] = bfhi(pw[j]);
-      gn[2 * j] = bflo(nw[j]); gn[2 * j + 1] = bfhi(nw[j]);
+    for (int h = 0; h < WS_EPT / 8; ++h) {
+      const uint4 pw = a.n_parts > 0 ? ldg16(a.g_post + c0 + 8 * h) : z4, nw = ldg16(a.g_next + c0 + 8 * h);
+      const uint32_t pv[4] = {pw.x, pw.y, pw.z, pw.w}, nv[4] = {nw.x, nw.y, nw.z, nw.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        gp[8 * h + 2 * j] = bflo(pv[j]); gp[8 * h + 2 * j + 1] = bfhi(pv[j]);
+        gn[8 * h + 2 * j] = bflo(nv[j]); gn[8 * h + 2 * j + 1] = bfhi(nv[j]);
+      }
     }
   }
   pdl_wait();
@@ -244,28 +246,28 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
     // reduction per stream gives both norms: with a = RMS^-1 of the partials' sum m and the post
     // gain g, x' = x + a g m and sum(x'^2) = sum(x^2) + 2a sum(g x m) + a^2 sum(g^2 m^2).
     const bool writer = blockIdx.x == 0 && blockIdx.y == 0;
-    const int c0 = ct * 16;
+    const int c0 = ct * WS_EPT;
     for (int b = 0; b < a.rows; ++b) {
-      float x[16], m[16];
+      float x[WS_EPT], m[WS_EPT];
       const float* xin = a.x_in + (size_t)b * D + c0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < WS_EPT / 4; ++q) {
         const float4 v = reinterpret_cast<const float4*>(xin)[q];
         x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
       }
 #pragma unroll
-      for (int j = 0; j < 16; ++j) m[j] = 0.f;
+      for (int j = 0; j < WS_EPT; ++j) m[j] = 0.f;
       for (int s = 0; s < a.n_parts; ++s) {
         const float* p = a.parts + s * a.part_stride + (size_t)b * D + c0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < WS_EPT / 4; ++q) {
           const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + q);
           m[4 * q] += v.x; m[4 * q + 1] += v.y; m[4 * q + 2] += v.z; m[4 * q + 3] += v.w;
         }
       }
       float q4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < WS_EPT; ++j) {
         const float gm = gp[j] * m[j];
         q4[0] += m[j] * m[j];
         q4[1] += x[j] * x[j];
@@ -284,26 +286,30 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
       const float al = a.n_parts > 0 ? rsqrtf(t[0] * (1.0f / D) + a.eps) : 0.f;
       const float inv = rsqrtf(fmaxf(t[1] + 2.f * al * t[2] + al * al * t[3], 0.f) * (1.0f / D) + a.eps);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] += al * (gp[j] * m[j]);
+      for (int j = 0; j < WS_EPT; ++j) x[j] += al * (gp[j] * m[j]);
       if (writer) {
         float* xo = a.x_out + (size_t)b * D + c0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) reinterpret_cast<float4*>(xo)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+        for (int q = 0; q < WS_EPT / 4; ++q) reinterpret_cast<float4*>(xo)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
         if (a.dump) {
           float* dd = a.dump + (size_t)b * D + c0;
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
+          for (int q = 0; q < WS_EPT / 4; ++q)
             reinterpret_cast<float4*>(dd)[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
         }
       }
-      // this thread's 16 columns go to shared memory if they are in the block's K range
+      // this thread's columns go to shared memory if they are in the block's K range
       if (c0 >= kcta && c0 < kcta + Kc) {
-        uint32_t w[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) w[j] = pack_bf2(gn[2 * j] * (x[2 * j] * inv), gn[2 * j + 1] * (x[2 * j + 1] * inv));
-        uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)b * XS + (c0 - kcta));
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        for (int h = 0; h < WS_EPT / 8; ++h) {
+          uint32_t w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int e = 8 * h + 2 * j;
+            w[j] = pack_bf2(gn[e] * (x[e] * inv), gn[e + 1] * (x[e + 1] * inv));
+          }
+          *reinterpret_cast<uint4*>(xs + (size_t)b * XS + (c0 - kcta) + 8 * h) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
       }
       consumers_sync();  // redn is reused by the next stream
     }
