@@ -222,16 +222,22 @@ __global__ void __launch_bounds__(128) k_attn_decode_fused(const float* __restri
     }
     return base + (((size_t)slot * HKV + kvh) * WIN + j) * HD;
   };
-  // ---- stage the cached keys / values of the split (all but the current position)
-  for (int e = tid; e < max(cnt, 0) * 16; e += blockDim.x) {
-    const int r = e >> 4, c = e & 15;
-    if (j0 + r == cur) continue;
-    const uint32_t kd = (uint32_t)__cvta_generic_to_shared(ks + krot(r, c));
-    const uint32_t vd = (uint32_t)__cvta_generic_to_shared(vs + r * HD + c * 8);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(kd), "l"(row_ptr(L.k, j0 + r) + c * 8));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vd), "l"(row_ptr(L.v, j0 + r) + c * 8));
+  // ---- stage the split's keys / values: whole 64-position blocks, each contiguous in the pool
+  // (a page of one kv head) or the ring, one bulk copy per block for K and one for V. Rows past
+  // the visible keys and the current position's stale row come along and are never used.
+  __shared__ __align__(8) uint64_t kv_bar;
+  const int nblk = cnt > 0 ? (cnt + 63) / 64 : 0;
+  if (tid == 0) {
+    mbar_init(su32(&kv_bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (nblk) {
+      mbar_expect_tx(su32(&kv_bar), (uint32_t)nblk * 2 * 64 * HD * 2);
+      for (int i = 0; i < nblk; ++i) {
+        bulk_g2s(su32(ks + i * 64 * HD), row_ptr(L.k, j0 + 64 * i), 64 * HD * 2, su32(&kv_bar));
+        bulk_g2s(su32(vs + i * 64 * HD), row_ptr(L.v, j0 + 64 * i), 64 * HD * 2, su32(&kv_bar));
+      }
+    }
   }
-  asm volatile("cp.async.commit_group;");
   // gains and rotary coefficients of this thread's dimension d = tid are weights too
   const int d = tid, pd = d < 64 ? d + 64 : d - 64, ir = d & 63;
   const float gq = bf2f(A.q_norm[d]), gk = bf2f(A.k_norm[d]);
@@ -277,8 +283,11 @@ __global__ void __launch_bounds__(128) k_attn_decode_fused(const float* __restri
     kd[d] = f2bf(kn[d]);
     vd[d] = f2bf(vn[d]);
   }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
+  __syncthreads();  // also orders the barrier's initialisation before every thread's wait
+  if (nblk && !mbar_wait(su32(&kv_bar), 0, A.err)) {
+    // a copy that never lands: report through the status word, drop this block's partial
+    asm volatile("" ::: "memory");
+  }
   float* out = part + (((size_t)b * HQ + kvh * GQA) * splits + sp) * (HD + 2);
   if (cnt > 0) {
     // scores: one key per thread (span <= 128)
@@ -291,12 +300,15 @@ __global__ void __launch_bounds__(128) k_attn_decode_fused(const float* __restri
       } else {
 #pragma unroll 4
         for (int c = 0; c < 16; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(ks + krot(tid, c));
+          // rows are 256 B apart: rotating the chunk order by the key spreads a warp's reads over all
+          // banks (and the q chunks it needs over 8 broadcast groups)
+          const int ch = (c + tid) & 15;
+          const uint4 w = *reinterpret_cast<const uint4*>(ks + tid * HD + ch * 8);
           const float k8[8] = {bflo(w.x), bfhi(w.x), bflo(w.y), bfhi(w.y), bflo(w.z), bfhi(w.z), bflo(w.w), bfhi(w.w)};
 #pragma unroll
           for (int hh = 0; hh < GQA; ++hh)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s[hh] += qs[hh][c * 8 + e] * k8[e];
+            for (int e = 0; e < 8; ++e) s[hh] += qs[hh][ch * 8 + e] * k8[e];
         }
       }
 #pragma unroll

@@ -187,6 +187,7 @@ struct AttnDecodeArgs {
   const float* rope_sin;
   float eps;
   unsigned* counters;      // [streams][HKV], zero between calls
+  int* err;                // status word (a bounded wait that gave up)
 };
 cudaError_t attn_decode_fused(const float* qkvg, Rows rows, AttnLayer L, const AttnDecodeArgs& A, int splits,
                               float* part, bf16* y, cudaStream_t s);

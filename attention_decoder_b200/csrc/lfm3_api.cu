@@ -930,7 +930,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       CK(run_ws(ctx, GEMV_PARTIAL, 0, ctx->plans[l].ws_qkvg, q, s));
       advance();
       const int k = full ? 0 : 1;
-      AttnDecodeArgs A{B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], eps, ctx->attn_cnt};
+      AttnDecodeArgs A{B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], eps, ctx->attn_cnt, ctx->err};
       CK(attn_decode_fused(ctx->part3, rows, attn_layer(ctx, st, l, v), A, full ? splits_full : WIN / DEC_KEYS_RING,
                            attn_part, ctx->y, s));
       WsArgs o{};
