@@ -226,6 +226,7 @@ struct GemmPlan {
 bool tma_init();
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 cudaError_t gemm(const GemmPlan& p, int M, int* err, cudaStream_t s);
+bool gemm_wide(int N);  // 256-column tiles for this output width
 cudaError_t gemm_init();
 // NVFP4 prefill: dequantise a weight to bf16 [N][K] in scratch, then run the bf16 GEMM.
 cudaError_t nvfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, float tscale, int N, int K, bf16* out,
