@@ -119,8 +119,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the last query rows see the most keys: they are dispatched first, so the blocks left for the
+  // final wave are the short ones (causal full layers)
   const int kvh = blockIdx.y;
-  const int rb0 = blockIdx.x * AT_ROWS;
+  const int rb0 = (gridDim.x - 1 - blockIdx.x) * AT_ROWS;
   const int rb1 = min(a.n, rb0 + AT_ROWS) - 1;
   const bool full = a.full;
   const int koff = full ? 0 : a.p0 - WIN;                   // key index -> position
