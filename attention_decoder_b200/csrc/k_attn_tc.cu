@@ -6,13 +6,14 @@
 // two-stage ring. Per tile:
 //   warp 1 (one lane):  S = Q K^T      (tcgen05.mma kind::f16, 128 x 128 x 128, fp32 in TMEM; two S
 //                       buffers, so the next tile's scores are computed during this tile's softmax)
-//   warps 2..5:         each thread owns one TMEM lane (= one row): read S, mask (causal, the
-//                       256-key window on sliding layers, written keys only), online softmax in
-//                       fp32 (exp2 with the 1/sqrt(128) scale folded in), write P as bf16 into a
-//                       128-byte-swizzled shared tile, rescale its O row in TMEM when the running
-//                       maximum grows, zero the V rows of unwritten keys
+//   warps 2..9:         two warps per TMEM lane quarter, so each thread owns one row (TMEM lane)
+//                       and half of its keys: read S, mask (causal, the 256-key window on sliding
+//                       layers, written keys only), online softmax in fp32 (exp2 with the
+//                       1/sqrt(128) scale folded in; the pair shares the row maximum), write P as bf16
+//                       into a 128-byte-swizzled shared tile, rescale its half of the O row in TMEM
+//                       when the running maximum grows, zero the V rows of unwritten keys
 //   warp 1:             O += P V       (V read as an MN-major operand: dims contiguous)
-// After the last tile each row thread divides by the softmax sum, multiplies by the head gate
+// After the last tile the pair adds its two partial softmax sums; each thread divides its half row, multiplies by the head gate
 // sigmoid(g) (coreai-model-zoo "lfm3-1.7b-port", diff table row 4) and stores bf16.
 // Every mbarrier wait is bounded (the device error word is set when one gives up).
 #include <cudaTypedefs.h>
@@ -27,7 +28,7 @@ constexpr int AT_KT = 128;                  // keys per tile
 constexpr uint32_t AT_Q_BYTES = AT_M * HD * 2;      // 32 KB
 constexpr uint32_t AT_KV_BYTES = AT_KT * HD * 2;    // 32 KB per K or V tile
 constexpr uint32_t AT_P_BYTES = AT_M * AT_KT * 2;   // 32 KB
-constexpr int AT_THREADS = 192;
+constexpr int AT_THREADS = 320;  // loader, MMA issuer, 8 softmax / epilogue warps
 
 DEVI void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
   asm volatile(
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
     mbar_init(s_full0, 1);
     mbar_init(s_full1, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(o_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -236,54 +237,72 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- softmax / epilogue
-    const int quarter = warp & 3;
+    // Two warps per TMEM lane quarter: `half` 0 takes keys 0..63 of each tile and dims 0..63 of O,
+    // half 1 keys 64..127 and dims 64..127. The pair shares its rows' maxima and sums through
+    // shared memory at a 64-thread named barrier, where it also agrees on giving up after a wait
+    // that timed out, so both warps always reach the same barriers.
+    const int quarter = warp & 3, half = (warp - 2) >> 2;
     const int m = quarter * 32 + lane;                     // this thread's row
     const int r = rb0 + (m >> 2), h = kvh * GQA + (m & 3);
     const int qp = a.p0 + r;                               // query position
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;
+    float* pair_f = reinterpret_cast<float*>(bars + 16);   // [2 halves][128 rows]
+    int* pair_ok = reinterpret_cast<int*>(pair_f + 256);   // [2 halves][4 quarters]
+    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(3 + quarter) : "memory"); };
     float mrun = -INFINITY, lrun = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
       const int kt0 = klo + j * AT_KT;
-      if (!mbar_wait((j & 1) ? s_full1 : s_full0, (j >> 1) & 1, a.err)) { ok = false; break; }
+      bool got = mbar_wait((j & 1) ? s_full1 : s_full0, (j >> 1) & 1, a.err);
       at_fence_after();
-      const uint32_t srow = trow + (uint32_t)(j & 1) * 128;  // this tile's S buffer
-      // pass 1: masked row maximum
+      const uint32_t srow = trow + (uint32_t)(j & 1) * 128 + half * 64;  // this tile's S, my keys
+      const int kh0 = kt0 + half * 64;
+      // pass 1: masked maximum over my 64 keys
       float tmax = -INFINITY;
+      if (got) {
 #pragma unroll 1
-      for (int c = 0; c < AT_KT / 32; ++c) {
-        float v[32];
-        at_ld32(srow + c * 32, v);
+        for (int c = 0; c < 2; ++c) {
+          float v[32];
+          at_ld32(srow + c * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int kp = kt0 + c * 32 + i + koff;
-          bool vis = kp <= qp && kp >= 0 && (kt0 + c * 32 + i) <= kmax_valid;
-          if (!full) vis = vis && (qp - kp < WIN);
-          if (vis) tmax = fmaxf(tmax, v[i] * sl2);
+          for (int i = 0; i < 32; ++i) {
+            const int kk = kh0 + c * 32 + i, kp = kk + koff;
+            bool vis = kp <= qp && kp >= 0 && kk <= kmax_valid;
+            if (!full) vis = vis && (qp - kp < WIN);
+            if (vis) tmax = fmaxf(tmax, v[i] * sl2);
+          }
         }
       }
+      // the previous P.V must be finished before P is overwritten and O is rescaled
+      if (got && j > 0) got = mbar_wait(o_done, (j - 1) & 1, a.err);
+      pair_f[half * 128 + m] = tmax;
+      if (lane == 0) pair_ok[half * 4 + quarter] = got;
+      pair_sync();
+      ok = pair_ok[quarter] && pair_ok[4 + quarter];
+      tmax = fmaxf(pair_f[m], pair_f[128 + m]);
+      pair_sync();  // pair_f is rewritten below
+      if (!ok) break;
+      at_fence_after();
       const float mnew = fmaxf(mrun, tmax);
       const float mu = mnew == -INFINITY ? 0.f : mnew;
       const float alpha = exp2f(mrun - mu);
-      // the previous P.V must be finished before P is overwritten and O is rescaled
-      if (j > 0 && !mbar_wait(o_done, (j - 1) & 1, a.err)) { ok = false; break; }
-      at_fence_after();
       // tcgen05.ld/st are warp-wide: rescale when any row of the warp needs it (others use 1)
       if (__any_sync(0xffffffffu, j > 0 && alpha < 1.f)) {
 #pragma unroll 1
-        for (int c = 0; c < HD / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           float o[32];
-          at_ld32(trow + 256 + c * 32, o);
+          at_ld32(trow + 256 + half * 64 + c * 32, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          at_st32(trow + 256 + c * 32, o);
+          at_st32(trow + 256 + half * 64 + c * 32, o);
         }
       }
-      // pass 2: probabilities -> bf16 P tile (row m, 128-byte swizzle)
+      // pass 2: probabilities of my keys -> bf16 P (row m, key block `half`, 128-byte swizzle)
       float lsum = 0.f;
+      unsigned char* pb = ps + half * (AT_P_BYTES / 2);
 #pragma unroll 1
-      for (int c = 0; c < AT_KT / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float v[32];
         at_ld32(srow + c * 32, v);
         uint32_t pk[16];
@@ -292,8 +311,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           float pp[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int kk = kt0 + c * 32 + i + e;
-            const int kp = kk + koff;
+            const int kk = kh0 + c * 32 + i + e, kp = kk + koff;
             bool vis = kp <= qp && kp >= 0 && kk <= kmax_valid;
             if (!full) vis = vis && (qp - kp < WIN);
             pp[e] = vis ? exp2f(v[i + e] * sl2 - mu) : 0.f;
@@ -301,18 +319,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           }
           pk[i >> 1] = pack_bf2(pp[0], pp[1]);
         }
-        // keys c*32 .. c*32+31 = key block (c >> 1), 16-byte chunks (c & 1) * 4 .. +3
-        unsigned char* pb = ps + (c >> 1) * (AT_P_BYTES / 2);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(pb + sw_off(m, (c & 1) * 4 + q)) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          *reinterpret_cast<uint4*>(pb + sw_off(m, c * 4 + q)) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
-      lrun = lrun * alpha + lsum;
+      lrun = lrun * alpha + lsum;  // my keys' share; the halves add up at the end
       mrun = mnew;
       // V rows of keys never written (past the chunk) or not loaded (the tile's second page lies
       // past every query of the block): zero them so 0 * V cannot bring in stale values
       const int loaded = (kt0 + 64 <= khi) ? AT_KT : 64;
-      if (kt0 + AT_KT - 1 > kmax_valid || loaded < AT_KT) {
+      if (half == 0 && (kt0 + AT_KT - 1 > kmax_valid || loaded < AT_KT)) {
         const int st = j & 1;
         unsigned char* vd = vs + st * AT_KV_BYTES;
         const int key = m;  // one key row per thread
@@ -329,16 +345,23 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (ok && mbar_wait(o_done, (ntiles - 1) & 1, a.err)) {
+    // the row's softmax sum is the two halves' sums (both kept with the same running maximum)
+    pair_f[half * 128 + m] = lrun;
+    bool fin = ok && mbar_wait(o_done, (ntiles - 1) & 1, a.err);
+    if (lane == 0) pair_ok[half * 4 + quarter] = fin;
+    pair_sync();
+    fin = pair_ok[quarter] && pair_ok[4 + quarter];
+    const float ltot = pair_f[m] + pair_f[128 + m];
+    if (fin) {
       at_fence_after();
       // every lane reads TMEM (warp-wide loads); rows past the chunk do not store
       const bool live = r <= rb1;
-      const float gt = live ? sigmoidf_(a.gate[(size_t)r * HQ + h]) / lrun : 0.f;
-      bf16* dst = a.y + (size_t)(live ? r : 0) * HQ * HD + h * HD;
+      const float gt = live ? sigmoidf_(a.gate[(size_t)r * HQ + h]) / ltot : 0.f;
+      bf16* dst = a.y + (size_t)(live ? r : 0) * HQ * HD + h * HD + half * 64;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float o[32];
-        at_ld32(trow + 256 + c * 32, o);
+        at_ld32(trow + 256 + half * 64 + c * 32, o);
         if (live) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
@@ -355,7 +378,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
 }
 
-constexpr size_t AT_SMEM = 1024 + AT_Q_BYTES + 4 * AT_KV_BYTES + AT_P_BYTES + 256;
+constexpr size_t AT_SMEM = 1024 + AT_Q_BYTES + 4 * AT_KV_BYTES + AT_P_BYTES + 256 + 256 * 4 + 64;  // + pair scratch
 
 cudaError_t attn_tc_init() {
   return cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AT_SMEM);
