@@ -52,6 +52,20 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_out(CUtensorMap* m, void* base, bool fp32, uint64_t rows, uint64_t cols, uint64_t ld) {
+  if (!p_encode) return false;
+  const uint64_t es = fp32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (ld * es) % 16 || cols > ld) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * es};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / es), 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = p_encode(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------- PTX wrappers
 DEVI void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
   asm volatile(
@@ -95,6 +109,47 @@ DEVI void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two 64-column TMEM loads (this thread's lane) behind a single wait, in one statement so that no
+// use of the registers can be scheduled before the wait.
+DEVI void tmem_ld64x2(uint32_t ta, uint32_t tb, float* va, float* vb) {
+  uint32_t r[128];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,"
+      "%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,"
+      "%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%129];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]),
+        "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]),
+        "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]),
+        "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
+        "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]),
+        "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]),
+        "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]),
+        "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]),
+        "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]),
+        "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]),
+        "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]),
+        "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]),
+        "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]),
+        "=r"(r[126]), "=r"(r[127])
+      : "r"(ta), "r"(tb));
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    va[i] = __uint_as_float(r[i]);
+    vb[i] = __uint_as_float(r[64 + i]);
+  }
+}
+
+// SiLU for the GEMM epilogue: the fast division (the argument of the exponential is capped so that
+// the divisor stays finite; silu(x) for x < -80 is 0 at fp32 precision anyway).
+DEVI float silu_fast(float x) { return __fdividef(x, 1.f + __expf(fminf(-x, 80.f))); }
+
 struct GemmArgs {
   int M, N, K, ld;
   void* out;
@@ -110,19 +165,105 @@ struct GemmGeom {
   static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
 };
 
+DEVI void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+DEVI void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+DEVI void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+DEVI void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+DEVI void sts128(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+constexpr uint32_t GM_STG_WARP = 2 * 4096;  // per epilogue warp: two 32-row x 128-byte staging tiles
+constexpr uint32_t GM_STG = 4 * GM_STG_WARP;
+
+// Epilogue of one 128-row x BN-column accumulator, run by each of the 4 epilogue warps on its 32
+// rows [wrow0, wrow0 + 32) (TMEM lanes of its quarter; tbase points at the quarter and the
+// accumulator's first column). Per 128 output bytes of a row (32 fp32 or 64 bf16 columns) the
+// warp stages its 32 rows in shared memory with the 128-byte swizzle and writes them with one TMA
+// tensor store, so each row segment leaves the SM as whole lines; the two staging tiles alternate,
+// and a tile is rewritten only once the store issued from it two steps earlier has read it. Rows
+// past M (the last tile of a ragged chunk) take plain per-thread stores instead; column chunks past
+// N are skipped, and a chunk that straddles N is clipped by the store.
+template <int BN, int EPI>
+DEVI void gemm_epilogue(uint32_t tbase, int wrow0, int n0, const GemmArgs& g, const CUtensorMap* to, uint32_t stg,
+                        int lane) {
+  constexpr int NOUT = EPI == GEMM_SWIGLU ? BN / 2 : BN;
+  constexpr int CPC = EPI == GEMM_F32 ? 32 : 64;  // output columns per 128-byte row segment
+  const int row = wrow0 + lane;
+  const bool staged = wrow0 + 32 <= g.M;
+#pragma unroll 1
+  for (int c = 0; c < NOUT / CPC; ++c) {
+    const int col = n0 + c * CPC;
+    uint32_t w[32];  // this row's 128 output bytes
+    if constexpr (EPI == GEMM_F32) {
+      float v[32];
+      tmem_ld32(tbase + c * 32, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(g.alpha * v[j]);
+    } else if constexpr (EPI == GEMM_BF16) {
+      float v[64];
+      tmem_ld32(tbase + c * 64, v);
+      tmem_ld32(tbase + c * 64 + 32, v + 32);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) w[j] = pack_bf2(g.alpha * v[2 * j], g.alpha * v[2 * j + 1]);
+    } else {  // w1 products in columns [0, BN/2), w3 products in [BN/2, BN)
+      float va[64], vb[64];
+      tmem_ld64x2(tbase + c * 64, tbase + BN / 2 + c * 64, va, vb);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        w[j] = pack_bf2(silu_fast(g.alpha * va[2 * j]) * (g.alpha * vb[2 * j]),
+                        silu_fast(g.alpha * va[2 * j + 1]) * (g.alpha * vb[2 * j + 1]));
+    }
+    if (col >= g.N) continue;  // the same for the whole warp
+    if (staged) {
+      const uint32_t buf = stg + (uint32_t)(c & 1) * 4096;
+      if (lane == 0) bulk_wait_read_1();
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        sts128(buf + lane * 128 + ((q ^ (lane & 7)) << 4), make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(to, buf, col, wrow0);
+        bulk_commit();
+      }
+    } else if (row < g.M) {
+      if constexpr (EPI == GEMM_F32) {
+        float* dst = reinterpret_cast<float*>(g.out) + (size_t)row * g.ld + col;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col + j < g.N) dst[j] = __uint_as_float(w[j]);
+      } else {
+        uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<bf16*>(g.out) + (size_t)row * g.ld + col);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)  // output widths are even
+          if (col + 2 * j < g.N) dst[j] = w[j];
+      }
+    }
+  }
+}
+
 // Persistent: block b takes tiles b, b + gridDim.x, ... (M tiles fastest, so consecutive blocks
 // share a weight tile through L2). TMEM holds two BN-column accumulators: the MMA thread fills
 // one while the epilogue warps drain the other (acc_full / acc_empty barriers).
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtensorMap ta,
                                                  const __grid_constant__ CUtensorMap tb,
-                                                 const __grid_constant__ CUtensorMap tb3, const GemmArgs g) {
+                                                 const __grid_constant__ CUtensorMap tb3,
+                                                 const __grid_constant__ CUtensorMap to, const GemmArgs g) {
   using G = GemmGeom<BN>;
   constexpr int S = G::STAGES;
   constexpr int NOUT = EPI == GEMM_SWIGLU ? BN / 2 : BN;  // output columns per tile
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * G::STAGE);
+  const uint32_t stg0 = su32(smem + S * G::STAGE);  // epilogue staging (GM_STG bytes)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * G::STAGE + GM_STG);
   const uint32_t full0 = su32(bars), empty0 = su32(bars + S);
   const uint32_t accf0 = su32(bars + 2 * S), acce0 = su32(bars + 2 * S + 2);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
@@ -177,8 +318,10 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
           if constexpr (EPI == GEMM_SWIGLU) {
             tma_load_2d(b_s, &tb, kb * GM_BK, n0, full0 + 8 * s);
             tma_load_2d(b_s + G::B_BYTES / 2, &tb3, kb * GM_BK, n0, full0 + 8 * s);
-          } else {
-            tma_load_2d(b_s, &tb, kb * GM_BK, n0, full0 + 8 * s);
+          } else {  // weight boxes are 128 rows: a 256-wide tile takes two
+#pragma unroll
+            for (int h = 0; h < BN / 128; ++h)
+              tma_load_2d(b_s + h * (G::B_BYTES / (BN / 128)), &tb, kb * GM_BK, n0 + 128 * h, full0 + 8 * s);
           }
         }
       }
@@ -187,32 +330,41 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
     if (lane == 0) {
       constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                  ((uint32_t)(GM_BM >> 4) << 24);
-      int it = 0, i = 0, after_fail = 0;
+      // The issue loop is latency-bound when it does more than wait, issue and commit: keep the
+      // k-loop to exactly that (the stage barriers order the copies before the MMAs; the fence is
+      // only needed where TMEM changes hands).
+      const uint32_t smem0 = su32(smem);
+      int it = 0, i = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
         const int buf = i & 1;
-        if (ok && !mbar_wait(acce0 + 8 * buf, ((i >> 1) & 1) ^ 1, g.err)) ok = false;
+        if (!mbar_wait(acce0 + 8 * buf, ((i >> 1) & 1) ^ 1, g.err)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t td = tmem + buf * BN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          // after a failure keep draining (bounded) the stages the producer may still have in
-          // flight - it runs at most S ahead - so no copy lands after the block exits
-          if (!ok && ++after_fail > S) break;
-          const bool got = mbar_wait(full0 + 8 * s, ph, g.err);
-          ok = ok && got;
-          tc_fence_after();
-          if (ok) {
-            const uint64_t ad = sw128_desc(su32(smem + s * G::STAGE));
-            const uint64_t bd = sw128_desc(su32(smem + s * G::STAGE + G::A_BYTES));
-#pragma unroll
-            for (int k = 0; k < GM_BK / 16; ++k) umma_f16(td, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+          if (!mbar_wait(full0 + 8 * s, (it / S) & 1, g.err)) {
+            ok = false;
+            break;
           }
+          const uint32_t sa = smem0 + s * G::STAGE;
+          const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + G::A_BYTES);
+#pragma unroll
+          for (int k = 0; k < GM_BK / 16; ++k) umma_f16(td, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
           umma_commit(empty0 + 8 * s);
         }
-        umma_commit(accf0 + 8 * buf);
-        if (after_fail > S) break;
+        if (ok) umma_commit(accf0 + 8 * buf);
+      }
+      if (!ok) {
+        // a wait gave up: drain (bounded) the stages the producer may still have in flight - it
+        // runs at most S ahead - so that no copy lands after the block exits
+        for (int d = 0; d < S; ++d, ++it) {
+          mbar_wait(full0 + 8 * (it % S), (it / S) & 1, g.err);
+          umma_commit(empty0 + 8 * (it % S));
+        }
       }
     }
   } else {
@@ -222,75 +374,16 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
       const int buf = i & 1;
       const int m0 = (tile % num_m) * GM_BM, n0 = (tile / num_m) * NOUT;
-      const int row = m0 + quarter * 32 + lane;
       ok = mbar_wait(accf0 + 8 * buf, (i >> 1) & 1, g.err);
       tc_fence_after();
       if (!ok) break;
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
-      if constexpr (EPI == GEMM_SWIGLU) {
-        bf16* out = reinterpret_cast<bf16*>(g.out);
-#pragma unroll 1
-        for (int c = 0; c < BN / 64; ++c) {
-          float va[32], vb[32];
-          tmem_ld32(tbase + c * 32, va);
-          tmem_ld32(tbase + BN / 2 + c * 32, vb);
-          if (row < g.M) {
-            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * g.ld + n0 + c * 32);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t w[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = q * 8 + e * 2;
-                w[e] = pack_bf2(siluf_(g.alpha * va[j]) * (g.alpha * vb[j]),
-                                siluf_(g.alpha * va[j + 1]) * (g.alpha * vb[j + 1]));
-              }
-              dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          tmem_ld32(tbase + c * 32, v);
-          const int col = n0 + c * 32;
-          if (row < g.M && col < g.N) {
-            if constexpr (EPI == GEMM_F32) {
-              float* dst = reinterpret_cast<float*>(g.out) + (size_t)row * g.ld + col;
-              if (col + 32 <= g.N) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                  reinterpret_cast<float4*>(dst)[q] = make_float4(g.alpha * v[4 * q], g.alpha * v[4 * q + 1],
-                                                                  g.alpha * v[4 * q + 2], g.alpha * v[4 * q + 3]);
-              } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (j < g.N - col) dst[j] = g.alpha * v[j];
-              }
-            } else {
-              bf16* dst = reinterpret_cast<bf16*>(g.out) + (size_t)row * g.ld + col;
-              if (col + 32 <= g.N) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  uint32_t w[4];
-#pragma unroll
-                  for (int e = 0; e < 4; ++e) w[e] = pack_bf2(g.alpha * v[q * 8 + 2 * e], g.alpha * v[q * 8 + 2 * e + 1]);
-                  reinterpret_cast<uint4*>(dst)[q] = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-              } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (j < g.N - col) dst[j] = f2bf(g.alpha * v[j]);
-              }
-            }
-          }
-        }
-      }
+      gemm_epilogue<BN, EPI>(tbase, m0 + quarter * 32, n0, g, &to, stg0 + quarter * GM_STG_WARP, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce0 + 8 * buf);
     }
+    if (lane == 0) bulk_wait_all();  // the output is written before the block exits
   }
   tc_fence_before();
   __syncthreads();
@@ -298,10 +391,207 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN));
 }
 
+// ---------------------------------------------------------------- 2-SM tiles (prefill, M > 128)
+// A cluster of two CTAs on two SMs computes one 256 x BN tile with tcgen05.mma.cta_group::2
+// (M = 256): CTA rank r holds rows [128 r, 128 r + 128) of the A tile and rows [BN/2 r, BN/2 r +
+// BN/2) of the weight tile (SwiGLU: rank 0 the 128 rows of w1, rank 1 the same rows of w3), and
+// its TMEM receives the accumulator of its own 128 rows over all BN columns. Each SM thus stages
+// half of the weight tile that a 1-SM 128 x BN tile needs. Rank 0 issues every MMA; its full
+// barrier counts the bytes of both CTAs' copies, and each commit arrives on the barrier at the
+// same offset in both CTAs, so each producer and each epilogue waits on its own CTA's barriers.
+// The epilogue warps of both CTAs hand an accumulator back through rank 0's acc_empty barrier.
+DEVI uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+DEVI uint32_t peer_addr(uint32_t saddr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
+  return d;
+}
+DEVI void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Copy into this CTA's shared memory, completing on a barrier that may sit in the peer CTA.
+DEVI void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+DEVI void umma_f16_pair(uint32_t tmem_d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(
+          tmem_d),
+      "l"(ad), "l"(bd), "r"(idesc), "r"(accum));
+}
+// Arrive (once the issued MMAs finish) on the barrier at offset `bar` in both CTAs of the pair.
+DEVI void umma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((unsigned short)3)
+      : "memory");
+}
+DEVI void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
 template <int BN>
-constexpr size_t gemm_smem() { return 1024 + GemmGeom<BN>::STAGES * (size_t)GemmGeom<BN>::STAGE + 256; }
+struct Gemm2Geom {
+  static constexpr int STAGES = 6;
+  static constexpr uint32_t A_BYTES = 128 * GM_BK * 2;       // this CTA's 128 rows of the A tile
+  static constexpr uint32_t B_BYTES = (BN / 2) * GM_BK * 2;  // this CTA's half of the weight rows
+  static constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+};
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1) k_gemm2(const __grid_constant__ CUtensorMap ta,
+                                                  const __grid_constant__ CUtensorMap tb,
+                                                  const __grid_constant__ CUtensorMap tb3,
+                                                 const __grid_constant__ CUtensorMap to, const GemmArgs g) {
+  using G = Gemm2Geom<BN>;
+  constexpr int S = G::STAGES;
+  constexpr int NOUT = EPI == GEMM_SWIGLU ? BN / 2 : BN;
+  static_assert(BN == 256, "each CTA copies one 128-row weight box per stage");
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t stg0 = su32(smem + S * G::STAGE);  // epilogue staging (GM_STG bytes)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * G::STAGE + GM_STG);
+  const uint32_t full0 = su32(bars), empty0 = su32(bars + S);
+  const uint32_t accf0 = su32(bars + 2 * S), acce0 = su32(bars + 2 * S + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_m = (g.M + 2 * GM_BM - 1) / (2 * GM_BM), num_n = (g.N + NOUT - 1) / NOUT;
+  const int ntiles = num_m * num_n;
+  const int nk = g.K / GM_BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf0 + 8 * b, 1);
+      mbar_init(acce0 + 8 * b, 8);  // 4 epilogue warps in each CTA (only rank 0's is waited on)
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&ta)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tb)) : "memory");
+  }
+  if (warp == 1) {  // the same warp in both CTAs allocates the pair's columns
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                 "r"(2 * BN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised before any copy or commit reaches them
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  pdl_wait();
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < ntiles && ok; tile += npairs) {
+        const int m0 = (tile % num_m) * 2 * GM_BM + (int)rank * GM_BM, n0 = (tile / num_m) * NOUT;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait(empty0 + 8 * s, ph ^ 1, g.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_s = su32(smem + s * G::STAGE), b_s = a_s + G::A_BYTES;
+          const uint32_t bar = peer_addr(full0 + 8 * s, 0);
+          if (rank == 0) mbar_expect_tx(full0 + 8 * s, 2 * G::STAGE);
+          tma_load_2d_pair(a_s, &ta, kb * GM_BK, m0, bar);
+          if constexpr (EPI == GEMM_SWIGLU) {
+            tma_load_2d_pair(b_s, rank ? &tb3 : &tb, kb * GM_BK, n0, bar);
+          } else {
+            tma_load_2d_pair(b_s, &tb, kb * GM_BK, n0 + (int)rank * (BN / 2), bar);  // one 128-row box
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                 ((uint32_t)((2 * GM_BM) >> 4) << 24);
+      const uint32_t smem0 = su32(smem);
+      int it = 0, i = 0;
+      bool ok = true;
+      for (int tile = pair; tile < ntiles && ok; tile += npairs, ++i) {
+        const int buf = i & 1;
+        if (!mbar_wait(acce0 + 8 * buf, ((i >> 1) & 1) ^ 1, g.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t td = tmem + buf * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(full0 + 8 * s, (it / S) & 1, g.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = smem0 + s * G::STAGE;
+          const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + G::A_BYTES);
+#pragma unroll
+          for (int k = 0; k < GM_BK / 16; ++k) umma_f16_pair(td, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+          umma_commit_pair(empty0 + 8 * s);
+        }
+        if (ok) umma_commit_pair(accf0 + 8 * buf);
+      }
+      if (!ok) {  // drain (bounded) the stages both producers may still have in flight
+        for (int d = 0; d < S; ++d, ++it) {
+          mbar_wait(full0 + 8 * (it % S), (it / S) & 1, g.err);
+          umma_commit_pair(empty0 + 8 * (it % S));
+        }
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    int i = 0;
+    bool ok = true;
+    for (int tile = pair; tile < ntiles && ok; tile += npairs, ++i) {
+      const int buf = i & 1;
+      const int m0 = (tile % num_m) * 2 * GM_BM + (int)rank * GM_BM, n0 = (tile / num_m) * NOUT;
+      ok = mbar_wait(accf0 + 8 * buf, (i >> 1) & 1, g.err);
+      tc_fence_after();
+      if (!ok) break;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
+      gemm_epilogue<BN, EPI>(tbase, m0 + quarter * 32, n0, g, &to, stg0 + quarter * GM_STG_WARP, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(peer_addr(acce0 + 8 * buf, 0));
+    }
+    if (lane == 0) bulk_wait_all();  // the output is written before the block exits
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();  // no MMA, copy or arrival of either CTA still targets the other
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN));
+}
+
+template <int BN>
+constexpr size_t gemm_smem() { return 1024 + GemmGeom<BN>::STAGES * (size_t)GemmGeom<BN>::STAGE + GM_STG + 256; }
 
 static int g_gemm_sms = 0;
+static int g_gemm_pairs = 0;  // clusters of two that fit on the device at once (paired kernel)
+// Paired (2-SM) tiles from this many rows on, for the FFN projections and the wide or deep ones
+// (measured on 2048-row chunks: w13 92.0 -> 91.6 us, w2 48.8 -> 46.8, in_proj 42.5 -> 40.5; the
+// 2048 x 2048 projections are 1.2 us faster on single-SM tiles); LFM3_GEMM_PAIR_MIN_M overrides.
+static int g_gemm_pair_min_m = 129;
 
 template <int BN, int EPI>
 static cudaError_t launch_gemm(const GemmPlan& p, int M, int* err, cudaStream_t s) {
@@ -311,7 +601,39 @@ static cudaError_t launch_gemm(const GemmPlan& p, int M, int* err, cudaStream_t 
   const int ntile = EPI == GEMM_SWIGLU ? BN / 2 : BN;
   const int tiles = ((p.N + ntile - 1) / ntile) * ((M + GM_BM - 1) / GM_BM);
   dim3 grid(std::min(tiles, g_gemm_sms > 0 ? g_gemm_sms : 148));
-  return launch(k, grid, dim3(192), smem, s, p.a, p.b, EPI == GEMM_SWIGLU ? p.b3 : p.b, g);
+  return launch(k, grid, dim3(192), smem, s, p.a, p.b, EPI == GEMM_SWIGLU ? p.b3 : p.b, p.o, g);
+}
+
+template <int BN>
+constexpr size_t gemm2_smem() { return 1024 + Gemm2Geom<BN>::STAGES * (size_t)Gemm2Geom<BN>::STAGE + GM_STG + 256; }
+
+static cudaLaunchConfig_t pair_config(int pairs, size_t smem, cudaStream_t s, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cfg;
+}
+
+template <int EPI>
+static cudaError_t launch_gemm2(const GemmPlan& p, int M, int* err, cudaStream_t s) {
+  constexpr int BN = 256;
+  constexpr int ntile = EPI == GEMM_SWIGLU ? BN / 2 : BN;
+  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err};
+  const int tiles = ((p.N + ntile - 1) / ntile) * ((M + 2 * GM_BM - 1) / (2 * GM_BM));
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pair_config(std::min(tiles, g_gemm_pairs), gemm2_smem<BN>(), s, attr);
+  ++g_launches;
+  return cudaLaunchKernelEx(&cfg, k_gemm2<BN, EPI>, p.a, p.b, EPI == GEMM_SWIGLU ? p.b3 : p.b, p.o, g);
 }
 
 // Output widths from which a tile is 256 columns wide (fewer, more L2-efficient tiles) rather than
@@ -320,6 +642,7 @@ static int g_gemm_wide_min = 2048;  // measured: 8k prefill 37.8 -> 34.6 ms agai
 
 cudaError_t gemm_init() {
   if (const char* v = getenv("LFM3_GEMM_WIDE_MIN_N")) g_gemm_wide_min = atoi(v);
+  if (const char* v = getenv("LFM3_GEMM_PAIR_MIN_M")) g_gemm_pair_min_m = atoi(v);
   cudaError_t e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -332,13 +655,35 @@ cudaError_t gemm_init() {
     return e;
   if ((e = cudaFuncSetAttribute(k_gemm<256, GEMM_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem<256>())))
     return e;
-  return cudaFuncSetAttribute(k_gemm<256, GEMM_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem<256>());
+  if ((e = cudaFuncSetAttribute(k_gemm<256, GEMM_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem<256>())))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_gemm2<256, GEMM_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm2_smem<256>())))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_gemm2<256, GEMM_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm2_smem<256>())))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_gemm2<256, GEMM_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm2_smem<256>())))
+    return e;
+  // every paired launch is persistent over the clusters that fit at once (one CTA per SM)
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pair_config(g_gemm_sms / 2, gemm2_smem<256>(), 0, attr);
+  cfg.numAttrs = 2;
+  if ((e = cudaOccupancyMaxActiveClusters(&g_gemm_pairs, k_gemm2<256, GEMM_F32>, &cfg)) != cudaSuccess) return e;
+  if (g_gemm_pairs < 1) return cudaErrorInvalidConfiguration;
+  return cudaSuccess;
 }
 
 bool gemm_wide(int N) { return N >= g_gemm_wide_min; }
 
 cudaError_t gemm(const GemmPlan& p, int M, int* err, cudaStream_t s) {
   if (p.K % GM_BK) return cudaErrorInvalidValue;
+  if (M >= g_gemm_pair_min_m && (p.epi == GEMM_SWIGLU || p.N >= 4096 || p.K >= 4096)) {
+    switch (p.epi) {
+      case GEMM_F32: return launch_gemm2<GEMM_F32>(p, M, err, s);
+      case GEMM_BF16: return launch_gemm2<GEMM_BF16>(p, M, err, s);
+      case GEMM_SWIGLU: return launch_gemm2<GEMM_SWIGLU>(p, M, err, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (p.epi) {
     case GEMM_F32: return gemm_wide(p.N) ? launch_gemm<256, GEMM_F32>(p, M, err, s) : launch_gemm<128, GEMM_F32>(p, M, err, s);
     case GEMM_BF16: return gemm_wide(p.N) ? launch_gemm<256, GEMM_BF16>(p, M, err, s) : launch_gemm<128, GEMM_BF16>(p, M, err, s);

@@ -218,6 +218,7 @@ struct GemmPlan {
   CUtensorMap a;      // activations [M][K] bf16, box 64 x 128
   CUtensorMap b;      // weights [N][K] bf16 (SwiGLU: w1)
   CUtensorMap b3;     // SwiGLU: w3
+  CUtensorMap o;      // output [M][ld] (fp32, or bf16), 32-row boxes of 128 bytes for TMA stores
   int epi, M, N, K;
   void* out;          // fp32 or bf16 [M][ld]
   int ld;
@@ -225,6 +226,9 @@ struct GemmPlan {
 };
 bool tma_init();
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Output map of a GEMM: [rows][cols] with row pitch ld elements, fp32 (32-column boxes) or bf16
+// (64-column boxes), 32 rows per box, 128-byte swizzle.
+bool make_tmap_out(CUtensorMap* m, void* base, bool fp32, uint64_t rows, uint64_t cols, uint64_t ld);
 cudaError_t gemm(const GemmPlan& p, int M, int* err, cudaStream_t s);
 bool gemm_wide(int N);  // 256-column tiles for this output width
 cudaError_t gemm_init();

@@ -273,12 +273,12 @@ bool plan_gemm(GemmPlan* p, int epi, const void* a, int a_rows, const void* b, c
   p->out = out;
   p->ld = ld;
   p->alpha = alpha;
-  const uint32_t box_b = (epi == GEMM_SWIGLU) ? 128 : (gemm_wide(N) ? 256 : 128);
+  const uint32_t box_b = 128;  // weight boxes: 128 rows (wide and paired tiles issue several)
   if (!make_tmap_bf16(&p->a, a, a_rows, K, 128)) return false;
   if (!make_tmap_bf16(&p->b, b, N, K, box_b)) return false;
   if (b3 && !make_tmap_bf16(&p->b3, b3, N, K, box_b)) return false;
   if (!b3) p->b3 = p->b;
-  return true;
+  return make_tmap_out(&p->o, out, epi == GEMM_F32, a_rows, N, ld);
 }
 
 // Host check that every position a call writes or reads in slot s, [0, end), has a page.
