@@ -1,19 +1,22 @@
 // Prefill projections on the 5th-generation tensor cores: C[M][N] = alpha * A[M][K] . W[N][K]^T
 // with A the bf16 activations of a prompt chunk and W a bf16 weight, both K-major.
 //
-// Persistent blocks (one per SM, 6 warps) walk 128 x BN output tiles (BN = 128 or 256):
-//   warp 0      TMA producer: 128x64 A box and BNx64 W box per stage (128-byte swizzle), into a
-//               4- or 6-stage ring guarded by full/empty mbarriers;
-//   warp 1      allocates 2 x BN TMEM columns (two accumulators); one elected lane issues
-//               tcgen05.mma (kind::f16, M=128, N=BN, K=16 per instruction, fp32 accumulate in TMEM),
-//               commits each stage back to the producer and each finished accumulator to the
-//               epilogue, and moves on to the next tile in the other accumulator;
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time (warp w reads TMEM lanes
-//               32*(w%4) ..), apply the fused epilogue, store, release the accumulator.
+// Persistent blocks (one per SM, 6 warps) walk output tiles:
+//   warp 0      TMA producer: A and W boxes of 64 K-columns per stage (128-byte swizzle) into a ring
+//               guarded by full/empty mbarriers;
+//   warp 1      allocates two accumulators in TMEM; one elected lane issues tcgen05.mma (kind::f16,
+//               K=16 per instruction, fp32 accumulate), commits each stage back to the producer and
+//               each finished accumulator to the epilogue, and moves on to the next tile in the
+//               other accumulator;
+//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes (warp w reads lanes 32*(w%4) ..), the
+//               fused epilogue, a 128-byte-swizzled staging tile in shared memory and a TMA tensor
+//               store per 32 rows x 128 bytes; then the accumulator is released.
+// k_gemm: one SM per 128 x BN tile (BN = 128 or 256). k_gemm2: a cluster of two SMs per 256 x 256
+// tile (tcgen05 cta_group::2), each SM staging its 128 rows of A and half of the weight rows.
 // Epilogues: fp32 out, bf16 out, and SwiGLU (the tile's 256 columns are 128 rows of w1 and the
 // same 128 rows of w3: u = silu(alpha a) * (alpha b), bf16).
-// Every mbarrier wait is bounded; a wait that gives up sets the device error word and the
-// block runs to completion without further MMAs so that TMEM is always released.
+// Every mbarrier wait is bounded; a wait that gives up sets the device error word, and the MMA
+// thread drains (bounded) the stages still in flight so that TMEM is always released.
 #include <cudaTypedefs.h>
 
 #include <algorithm>

@@ -294,7 +294,13 @@ def run_ours(args):
         pstep()
         pprof = mp.profile_read()
         mp.profile(False)
+        pf = prefill_flops(g, n8)
+        p_tf = pf / (pms / pk_steps / 1e3) / 1e12
         res["prefill_8k"] = {"tok_s": n8 * pk_steps / (pms / 1e3), "ms": pms / pk_steps,
+                             "flops": pf, "tflops": p_tf,
+                             "tc_frac": p_tf / float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
+                             "tc_frac_sustained": p_tf / float(pk.get("bf16_tflops_sustained",
+                                                                      pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))),
                              "gemm_tflops": pprof["flops"] / (pprof["ms"] / 1e3) / 1e12,
                              "gemm_share": pprof["ms"] / (pms / pk_steps)}
         del mp, sts
@@ -385,6 +391,26 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def prefill_flops(g, n):
+    """Algorithmic FLOPs of one n-token prompt pass: every projection GEMM (2 M N K), causal
+    attention (Q K^T and P V over the keys each query sees: all earlier positions on full layers,
+    at most the window on sliding ones) and the head on the last row. The 7-tap convolution and the
+    norms are left out (under 0.01 %)."""
+    from lfm3_inputs.gen import CONV, FULL
+    d, f, hd = g.d_model, g.d_ffn, g.head_dim
+    per_tok = 0
+    for t in g.layer_types:
+        per_tok += 2 * d * f * 3
+        per_tok += 2 * d * 3 * d + 2 * d * d if t == CONV else 2 * d * g.qkvg_rows + 2 * g.n_q * hd * d
+    keys_full = n * (n + 1) // 2
+    keys_win = sum(min(p + 1, g.window) for p in range(n))
+    attn = 0
+    for t in g.layer_types:
+        if t != CONV:
+            attn += 4 * hd * g.n_q * (keys_full if t == FULL else keys_win)
+    return n * per_tok + attn + 2 * d * g.vocab
 
 
 def run_prefill_only(args, world, m, g, stream, clocks, Wm):
