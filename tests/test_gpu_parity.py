@@ -72,6 +72,20 @@ def test_slice3_ragged_chunked_prefill_across_the_window(lib, slice3):
     m.check_device_errors()
 
 
+def test_slice3_300_row_chunk_on_paired_gemm_tiles(lib, slice3):
+    """One 300-row chunk: the 2-SM GEMM tiles cover rows 0..511, so the second tile's upper CTA
+    reads only rows past the chunk (zero-filled) and its lower CTA stores a ragged 32-row group."""
+    g, W, o = slice3
+    x = make_embeds(1, "paired", 300, g.d_model)
+    ref = o.forward_full(x0=f64_rows(x))
+    m = lib(W, max_streams=1, max_pages_per_stream=8, max_chunk=512)
+    st = m.new_state(poison=True)
+    out = m.prefill(st, 0, embeds=bf16_rows(x), hidden=True)
+    torch.cuda.synchronize()
+    assert_hidden(out["hidden"], ref["hidden"], what="300-row chunk")
+    m.check_device_errors()
+
+
 def test_slice3_prompt_equals_one_row_decode_at_cuts(lib, slice3):
     g, W, o = slice3
     x = make_embeds(2, "cuts", 270, g.d_model)
