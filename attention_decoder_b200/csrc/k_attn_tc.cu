@@ -99,6 +99,13 @@ DEVI void at_st32(uint32_t taddr, const float* v) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 2^x with the hardware approximation (relative error about 2^-22; denormal results flush to 0).
+DEVI float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled block of 128-B rows.
 DEVI uint32_t sw_off(int r, int c) { return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)); }
 
@@ -250,6 +257,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     float* pair_f = reinterpret_cast<float*>(bars + 16);   // [2 halves][128 rows]
     int* pair_ok = reinterpret_cast<int*>(pair_f + 256);   // [2 halves][4 quarters]
     auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(3 + quarter) : "memory"); };
+    // Visible keys of this row, as key indices: [vis_lo, vis_hi] (causal, written keys, and on
+    // sliding layers the 256-position window). A half tile all of whose keys are visible to every
+    // row of the block takes the unmasked path (all but the diagonal and window-edge tiles).
+    const int vis_hi = min(qp, kmax_valid + koff) - koff;
+    const int vis_lo = (full ? 0 : max(0, qp - (WIN - 1))) - koff;
+    const int dense_hi = min(qpos_lo, kmax_valid + koff) - koff;
+    const int dense_lo = (full ? 0 : max(0, qpos_hi - (WIN - 1))) - koff;
     float mrun = -INFINITY, lrun = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles && ok; ++j) {
@@ -258,21 +272,25 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       at_fence_after();
       const uint32_t srow = trow + (uint32_t)(j & 1) * 128 + half * 64;  // this tile's S, my keys
       const int kh0 = kt0 + half * 64;
-      // pass 1: masked maximum over my 64 keys
+      const bool dense = kh0 >= dense_lo && kh0 + 63 <= dense_hi;  // the same for the whole block
+      const int ilo = vis_lo - kh0, ihi = vis_hi - kh0;            // visible i in [ilo, ihi]
+      // pass 1: maximum of the raw scores over my visible keys (the scale is positive)
       float tmax = -INFINITY;
       if (got) {
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           float v[32];
           at_ld32(srow + c * 32, v);
+          if (dense) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int kk = kh0 + c * 32 + i, kp = kk + koff;
-            bool vis = kp <= qp && kp >= 0 && kk <= kmax_valid;
-            if (!full) vis = vis && (qp - kp < WIN);
-            if (vis) tmax = fmaxf(tmax, v[i] * sl2);
+            for (int i = 0; i < 32; ++i) tmax = fmaxf(tmax, v[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i >= ilo && c * 32 + i <= ihi) tmax = fmaxf(tmax, v[i]);
           }
         }
+        tmax *= sl2;
       }
       // the previous P.V must be finished before P is overwritten and O is rescaled
       if (got && j > 0) got = mbar_wait(o_done, (j - 1) & 1, a.err);
@@ -311,10 +329,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           float pp[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int kk = kh0 + c * 32 + i + e, kp = kk + koff;
-            bool vis = kp <= qp && kp >= 0 && kk <= kmax_valid;
-            if (!full) vis = vis && (qp - kp < WIN);
-            pp[e] = vis ? exp2f(v[i + e] * sl2 - mu) : 0.f;
+            pp[e] = ex2_approx(fmaf(v[i + e], sl2, -mu));
+            if (!dense && (c * 32 + i + e < ilo || c * 32 + i + e > ihi)) pp[e] = 0.f;
             lsum += pp[e];
           }
           pk[i >> 1] = pack_bf2(pp[0], pp[1]);
