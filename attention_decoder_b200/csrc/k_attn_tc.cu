@@ -302,7 +302,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       pair_sync();  // pair_f is rewritten below
       if (!ok) break;
       at_fence_after();
-      const float mnew = fmaxf(mrun, tmax);
+      // The running maximum moves only when a score exceeds it by more than 8 (in log2 units):
+      // probabilities stay below 2^8, O and the sum keep one common reference, and most tiles
+      // skip the O rescale. The final division by the sum is unchanged.
+      const float mnew = tmax > mrun + 8.f ? tmax : mrun;
       const float mu = mnew == -INFINITY ? 0.f : mnew;
       const float alpha = exp2f(mrun - mu);
       // tcgen05.ld/st are warp-wide: rescale when any row of the warp needs it (others use 1)
