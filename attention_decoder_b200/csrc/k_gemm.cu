@@ -666,12 +666,15 @@ cudaError_t gemm_init() {
     return e;
   if ((e = cudaFuncSetAttribute(k_gemm2<256, GEMM_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm2_smem<256>())))
     return e;
-  // every paired launch is persistent over the clusters that fit at once (one CTA per SM)
+  // every paired launch is persistent over the clusters that fit at once (one CTA per SM); where
+  // no pair can be resident (or the query is refused) the single-SM tiles do all the work
   cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config(g_gemm_sms / 2, gemm2_smem<256>(), 0, attr);
-  cfg.numAttrs = 2;
-  if ((e = cudaOccupancyMaxActiveClusters(&g_gemm_pairs, k_gemm2<256, GEMM_F32>, &cfg)) != cudaSuccess) return e;
-  if (g_gemm_pairs < 1) return cudaErrorInvalidConfiguration;
+  if (cudaOccupancyMaxActiveClusters(&g_gemm_pairs, k_gemm2<256, GEMM_F32>, &cfg) != cudaSuccess || g_gemm_pairs < 1) {
+    (void)cudaGetLastError();
+    g_gemm_pairs = 0;
+    g_gemm_pair_min_m = 1 << 30;
+  }
   return cudaSuccess;
 }
 
