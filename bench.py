@@ -304,10 +304,29 @@ def run_ours(args):
                              "gemm_tflops": pprof["flops"] / (pprof["ms"] / 1e3) / 1e12,
                              "gemm_share": pprof["ms"] / (pms / pk_steps)}
         del mp, sts
+    # prefill 32k (chunks of 2048) over shuffled pages: opt-in (--long)
+    if args.long and args.only is None:
+        n32 = 32768
+        mp = Lfm3Model(make_weights(g, 0), max_streams=1, max_pages_per_stream=n32 // 64, max_batch=1)
+        s32 = mp.new_state(page_table=page_permutation(1, "pages32k", n32 // 64).reshape(1, -1))
+        tok32 = torch.from_numpy(make_tokens(1, "prompt32k", n32, g.vocab)).cuda()
+
+        def lstep():
+            s32.h_seq_len[:] = 0
+            s32.seq_len.zero_()
+            mp.prefill(s32, 0, tokens=tok32)
+
+        lstep()
+        lms = timed(world, lstep, 2, stream)
+        lf = prefill_flops(g, n32)
+        l_tf = lf / (lms / 2 / 1e3) / 1e12
+        res["prefill_32k"] = {"tok_s": n32 * 2 / (lms / 1e3), "ms": lms / 2, "flops": lf, "tflops": l_tf,
+                              "tc_frac": l_tf / float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))}
+        del mp, s32
     del m, st
     torch.cuda.empty_cache()
 
-    # ---------------- NVFP4 FFN model: decode at 1 / 8 streams (2048 ctx) and 64 streams
+    # ---------------- NVFP4 FFN model: decode at 1 / 4 / 8 streams (2048 ctx) and 64 streams
     if not args.no_extra and args.only is None:
         Wq = make_weights(g, 0, ffn="nvfp4")
         S = 64
@@ -320,7 +339,7 @@ def run_ours(args):
         for s in range(8):
             mq.prefill(stq, s, tokens=prompt)
         qb = {}
-        for B in (1, 8):
+        for B in (1, 4, 8):
             sl = torch.arange(B, dtype=torch.int32, device="cuda")
             ob = {"argmax": torch.zeros(B, dtype=torch.int32, device="cuda"),
                   "logits": torch.empty(B, g.vocab, device="cuda")}
@@ -471,6 +490,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="headline decode only")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--small", action="store_true", help="4-layer profiling case (not a bench line)")
+    ap.add_argument("--long", action="store_true", help="also time the 32768-token prefill")
     ap.add_argument("--only", choices=["decode", "prefill"], default=None,
                     help="profiling: run only the bf16 decode or only the 8k prefill leg")
     args = ap.parse_args()
