@@ -32,7 +32,7 @@ norm and rotary, v, the gated attention output and the SwiGLU product. Projectio
 gate logits, norms, softmax and the residual stream are reductions and stay unrounded. With
 ``bf16=False`` (default) nothing is rounded: the plain float64 definition.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 in_proj rows are B, C, x in that order; the conv is causal with tap 6 on the
 current column and zero history at sequence start; no biases; q/k RMSNorm
 before rotary, gains of length head_dim shared by all heads; q head h reads kv

@@ -14,7 +14,7 @@ Element formats (OCP Microscaling Formats spec, v1.0):
   Exponent 0 is subnormal: 2^-6 * m/8. Exponent 15 with mantissa 7 is NaN;
   there is no infinity.
 
-Packing (this build's own choice; the pages do not give it): two codes per byte
+Packing (a layout this library chooses; the pages do not give one): two codes per byte
 along the input dimension, element 2b in the low nibble and 2b+1 in the high
 nibble; scales row-major [rows, cols/16].
 """
