@@ -142,20 +142,23 @@ def dist_setup(args):
     return world, rank, local
 
 
-def barrier(world):
+def barrier(world, cuda=True):
+    """All ranks meet; then (on a GPU) the device is drained."""
     import torch
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
 
 
-def max_over_ranks(world, x):
+def max_over_ranks(world, x, device="cuda"):
+    """The largest of the ranks' values (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
