@@ -19,9 +19,10 @@ the pages fix (``bf16=True``; see lfm3.py):
   NVFP4 dequantisation.
 
 Every function is pinned by the ``-m "not gpu"`` tests (library routines,
-brute force, closed forms, invariants and the pages' own totals). The one
-thing the pages give no worked numbers for - whole-model values - is
-"parity unpinned" beyond those invariants and brute-force pins.
+brute force, closed forms, invariants and the pages' own totals). The pages
+print no worked numbers for a whole forward pass; whole-model values are pinned
+instead against an independent torch assembly of the decoder on a small
+geometry (tests/test_oracle_head_pins.py), beside the invariants above.
 """
 from .lfm3 import Lfm3Oracle, OracleState, rms_norm, rope_inv_freq, apply_rope, round_bf16  # noqa: F401
 from .nvfp4 import e2m1_value, e4m3_value, nvfp4_dequant  # noqa: F401
