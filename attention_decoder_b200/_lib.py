@@ -17,8 +17,8 @@ STATUS = {0: "LFM3_OK", -1: "LFM3_E_ARG", -2: "LFM3_E_CONFIG", -3: "LFM3_E_CAPAC
 
 # exported entry points (every one declared in include/lfm3.h)
 SYMBOLS = ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_decode_step", "lfm3_decode_step_noalloc",
-           "lfm3_check_device_errors",
-           "lfm3_profile_enable", "lfm3_profile_read", "lfm3_profile_phases", "lfm3_profile_stamps",
+           "lfm3_check_device_errors", "lfm3_selftest_wait",
+           "lfm3_profile_enable", "lfm3_profile_read",
            "lfm3_last_launch_count", "lfm3_last_error", "lfm3_free")
 
 
@@ -67,19 +67,18 @@ def lib():
     L.lfm3_decode_step.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, i32p, vp, vp, vp, vp, vp, vp, vp]
     L.lfm3_decode_step_noalloc.argtypes = L.lfm3_decode_step.argtypes
     L.lfm3_check_device_errors.argtypes = [vp, vp]
+    L.lfm3_selftest_wait.argtypes = [vp, C.c_uint, vp]
     L.lfm3_profile_enable.argtypes = [vp, C.c_int, C.c_int]
     dp = C.POINTER(C.c_double)
     L.lfm3_profile_read.argtypes = [vp, C.POINTER(C.c_int), dp, dp, dp]
-    L.lfm3_profile_phases.argtypes = [vp, vp, C.c_int, C.POINTER(C.c_int), C.POINTER(C.c_int), dp, dp, dp, dp, dp, dp, dp]
-    L.lfm3_profile_stamps.argtypes = [vp, vp, C.POINTER(C.c_uint64), C.c_size_t, C.POINTER(C.c_int)]
     L.lfm3_last_launch_count.argtypes = [vp]
     L.lfm3_last_error.argtypes = [vp]
     L.lfm3_last_error.restype = C.c_char_p
     L.lfm3_free.argtypes = [vp]
     L.lfm3_free.restype = None
     for name in ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_decode_step", "lfm3_decode_step_noalloc",
-                 "lfm3_check_device_errors", "lfm3_profile_enable", "lfm3_profile_read", "lfm3_profile_phases",
-                 "lfm3_profile_stamps", "lfm3_last_launch_count"):
+                 "lfm3_check_device_errors", "lfm3_selftest_wait", "lfm3_profile_enable", "lfm3_profile_read",
+                 "lfm3_last_launch_count"):
         getattr(L, name).restype = C.c_int
     _lib = L
     return L
@@ -126,22 +125,16 @@ def lfm3_check_device_errors(ctx, stream):
     return lib().lfm3_check_device_errors(ctx, stream)
 
 
+def lfm3_selftest_wait(ctx, rounds, stream):
+    return lib().lfm3_selftest_wait(ctx, rounds, stream)
+
+
 def lfm3_profile_enable(ctx, on, capacity):
     return lib().lfm3_profile_enable(ctx, on, capacity)
 
 
 def lfm3_profile_read(ctx, launches, ms, nbytes, flops):
     return lib().lfm3_profile_read(ctx, launches, ms, nbytes, flops)
-
-
-def lfm3_profile_phases(ctx, stream, cap, n, kind, span_us, work_us, work_max_us, wait_us, lead_us, prologue_us,
-                        ahead_us):
-    return lib().lfm3_profile_phases(ctx, stream, cap, n, kind, span_us, work_us, work_max_us, wait_us, lead_us,
-                                     prologue_us, ahead_us)
-
-
-def lfm3_profile_stamps(ctx, stream, out, cap, n_blocks):
-    return lib().lfm3_profile_stamps(ctx, stream, out, cap, n_blocks)
 
 
 def lfm3_last_launch_count(ctx):

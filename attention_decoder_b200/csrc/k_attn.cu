@@ -1,640 +1,344 @@
-// GQA attention of the LFM3 decoder (16 q heads over 4 kv heads of 128; coreai-model-zoo note
-// "lfm3-1.7b-port", diff table rows 2 and 4, and "window_size, with no mask input").
+// Decode-time GQA attention of the LFM3 decoder (16 q heads over 4 kv heads of 128;
+// coreai-model-zoo note "lfm3-1.7b-port", diff table rows 2-4, and "window_size, with no mask
+// input").
 //
 // A key at position k is visible to a query at position p iff k <= p and, on sliding layers,
 // p - k < 256. Scores are q.k / sqrt(128), softmax in fp32, and the per-head gate sigmoid(g_h)
-// multiplies each head's output before o_proj (fused into the epilogues here).
+// multiplies each head's output before o_proj (fused into the merge here).
 //
-// Decode: split-KV. Block (split, kv head, stream) stages its key range (up to 128 keys) of K and
-// V in shared memory with asynchronous copies, scores it for the 4 query heads of the group and
-// writes unnormalised (max, sum, o) partials; the merge kernel combines splits, applies the gate
-// and writes bf16 o. Full layers read keys through the page table (64
-// positions per page); sliding layers read the 256-slot ring (slot = position % 256).
-//
-// Prefill: flash attention on the tensor cores (m16n8k16), one block per (32 query rows, kv
-// head): 8 warps = 4 heads x 2 row groups share every K/V tile staged in shared memory.
+// One launch per layer, from the raw q|k|v|gate projection rows (fp32, one row per stream):
+// block (split, kv head, stream) owns 64 keys - one 64-position page of that kv head on full
+// layers, a quarter of the 256-slot ring on sliding layers - so its keys and values are two
+// contiguous 16 KB tiles, copied with two bulk copies before the block waits for the projection
+// kernel (the cache does not depend on it). After the wait the block normalises and rotates its
+// four query heads and the head's new key, rounds them to bf16, writes the new key and value to
+// the cache (the block holding the current position does) and substitutes them for the stale
+// row in its shared copy. Scores: eight warps take 8 keys each; lane l holds dims 4l..4l+3 of
+// the four queries, and one transposing butterfly turns the 32 per-lane partial dots (8 keys x
+// 4 heads) into 32 finished scores, one per lane. Each block writes its unnormalised partial
+// (max, sum, o) per head; the last block of a (stream, kv head) - counted with an atomic -
+// merges the splits with every warp loading a different subset of them, applies the gate and
+// writes the bf16 output.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "kernels.cuh"
 
 namespace lfm3 {
 
-constexpr int DEC_SPLIT = DEC_KEYS_FULL;       // two 64-position pages
-constexpr int DEC_SPLIT_RING = DEC_KEYS_RING;
-constexpr int DEC_SMEM = 2 * DEC_SPLIT * HD * 2;  // K and V tiles, bf16
+constexpr int DA_THREADS = 256;                  // 8 warps
+constexpr int DA_WARPS = DA_THREADS / 32;
+constexpr int DA_TILE = DEC_KEYS * HD * 2;       // bytes of one K or V tile
+constexpr int DA_SMEM = 2 * DA_TILE;             // dynamic shared memory: K and V tiles
+static_assert(DEC_KEYS == PAGE, "a decode split is one page");
+static_assert(DA_WARPS * 8 == DEC_KEYS, "eight keys per warp");
 
-// 16-byte chunk c of key row r in a K tile: rotated by the row so that one key per thread reads
-// distinct banks.
-DEVI int krot(int r, int c) { return r * HD + ((c + r) & 15) * 8; }
+int attn_decode_splits(int max_pos) {
+  int s = WIN / DEC_KEYS;
+  while (s * DEC_KEYS < max_pos) s *= 2;
+  return s;
+}
 
-__global__ void __launch_bounds__(128) k_attn_decode(const bf16* __restrict__ q, Rows rows, AttnLayer L, int splits,
-                                                     float* __restrict__ part) {
-  extern __shared__ __align__(16) unsigned char dsm[];
+// Partials of a step: o [rows][HQ][splits][HD] (float4 aligned), then (max, sum) [rows][HQ][splits][2].
+DEVI size_t da_ml_offset(int nrows, int splits) { return (size_t)nrows * HQ * splits * HD; }
+
+__global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* __restrict__ qkvg, Rows rows,
+                                                                  AttnLayer L, AttnDecodeArgs A, int splits,
+                                                                  float* __restrict__ part, bf16* __restrict__ y) {
+  extern __shared__ __align__(128) unsigned char dsm[];
   bf16* ks = reinterpret_cast<bf16*>(dsm);
-  bf16* vs = ks + DEC_SPLIT * HD;
-  __shared__ float qs[GQA][HD];
-  __shared__ float sc[GQA][DEC_SPLIT];
-  __shared__ float ored[2][GQA][HD];
-  __shared__ float ml[GQA][2];
-  pdl_wait();
-  pdl_launch_dependents();
+  bf16* vs = ks + DEC_KEYS * HD;
+  __shared__ __align__(16) float qs[GQA][HD];
+  __shared__ float kb[HD];
+  __shared__ float sc[GQA][DEC_KEYS];
+  __shared__ __align__(16) float4 pr[DEC_KEYS];          // the 4 heads' probabilities of each key
+  __shared__ __align__(16) float obuf[4][GQA][HD];       // PV of the four key quarters
+  __shared__ float red[GQA + 1][4];
+  __shared__ float lx[GQA];
+  __shared__ __align__(8) uint64_t kv_bar;
+  __shared__ int last;
+
   const int sp = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int slot = rows.slot[b], pos = rows.pos[b];
-  const int span = L.full ? DEC_SPLIT : DEC_SPLIT_RING;
-  const int nkeys = L.full ? pos + 1 : min(pos + 1, WIN);  // ring: slots 0..nkeys-1 are live
-  const int j0 = sp * span, j1 = min(nkeys, j0 + span), cnt = j1 - j0;
-  float* out = part + (((size_t)b * HQ + kvh * GQA) * splits + sp) * (HD + 2);
-  if (cnt <= 0) {  // empty split
-    for (int e = tid; e < GQA * (HD + 2); e += blockDim.x) {
-      const int h = e / (HD + 2), k = e % (HD + 2);
-      out[(size_t)h * splits * (HD + 2) + k] = (k == HD) ? -INFINITY : 0.f;
-    }
+  // rows were set by the first kernel of the step, which has completed (reads go to L2)
+  const int slot = __ldcg(rows.slot + b), pos = __ldcg(rows.pos + b);
+  const int nkeys = L.full ? pos + 1 : min(pos + 1, WIN);
+  const int nact = (nkeys + DEC_KEYS - 1) / DEC_KEYS;  // splits with keys
+  if (sp >= nact) {
+    pdl_wait();
+    pdl_launch_dependents();
     return;
   }
-  // stage the split's keys and values: cnt rows x 16 chunks of 16 B each, all in flight at once
-  auto row_ptr = [&](const bf16* base, int j) -> const bf16* {
-    if (L.full) {
-      const int page = L.page_table[(size_t)slot * L.max_pages + j / PAGE];
-      return base + (((size_t)page * HKV + kvh) * PAGE + j % PAGE) * HD;
-    }
-    return base + (((size_t)slot * HKV + kvh) * WIN + j) * HD;
-  };
-  for (int e = tid; e < cnt * 16; e += blockDim.x) {
-    const int r = e >> 4, c = e & 15;
-    const uint32_t kd = (uint32_t)__cvta_generic_to_shared(ks + krot(r, c));
-    const uint32_t vd = (uint32_t)__cvta_generic_to_shared(vs + r * HD + c * 8);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(kd), "l"(row_ptr(L.k, j0 + r) + c * 8));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vd), "l"(row_ptr(L.v, j0 + r) + c * 8));
-  }
-  asm volatile("cp.async.commit_group;");
-  const float scale = rsqrtf((float)HD);
-  for (int e = tid; e < GQA * HD; e += blockDim.x)
-    qs[e / HD][e % HD] = bf2f(q[((size_t)b * HQ + kvh * GQA + e / HD) * HD + e % HD]) * scale;
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
-  // scores: one key per thread (span <= 128)
-  if (tid < cnt) {
-    float s[GQA] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int c = 0; c < 16; ++c) {
-      const uint4 w = *reinterpret_cast<const uint4*>(ks + krot(tid, c));
-      const float kv[8] = {bflo(w.x), bfhi(w.x), bflo(w.y), bfhi(w.y), bflo(w.z), bfhi(w.z), bflo(w.w), bfhi(w.w)};
-#pragma unroll
-      for (int h = 0; h < GQA; ++h)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s[h] += qs[h][c * 8 + e] * kv[e];
-    }
-#pragma unroll
-    for (int h = 0; h < GQA; ++h) sc[h][tid] = s[h];
-  }
-  __syncthreads();
-  {
-    const int h = warp;
-    float m = -INFINITY;
-    for (int j = lane; j < cnt; j += 32) m = fmaxf(m, sc[h][j]);
-    m = warp_max(m);
-    float l = 0.f;
-    for (int j = lane; j < cnt; j += 32) {
-      const float p = __expf(sc[h][j] - m);
-      sc[h][j] = p;
-      l += p;
-    }
-    l = warp_sum(l);
-    if (lane == 0) { ml[h][0] = m; ml[h][1] = l; }
-  }
-  __syncthreads();
-  {
-    const int par = tid >> 6, dp = (tid & 63) * 2;
-    float o[GQA][2] = {};
-#pragma unroll 4
-    for (int j = par; j < cnt; j += 2) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(vs + j * HD + dp);
-      const float v0 = bflo(w), v1 = bfhi(w);
-#pragma unroll
-      for (int h = 0; h < GQA; ++h) {
-        const float p = sc[h][j];
-        o[h][0] += p * v0;
-        o[h][1] += p * v1;
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < GQA; ++h) { ored[par][h][dp] = o[h][0]; ored[par][h][dp + 1] = o[h][1]; }
-  }
-  __syncthreads();
-  for (int e = tid; e < GQA * HD; e += blockDim.x) {
-    const int h = e / HD, d = e % HD;
-    out[(size_t)h * splits * (HD + 2) + d] = ored[0][h][d] + ored[1][h][d];
-  }
-  if (tid < GQA) {
-    out[(size_t)tid * splits * (HD + 2) + HD] = ml[tid][0];
-    out[(size_t)tid * splits * (HD + 2) + HD + 1] = ml[tid][1];
-  }
-}
-
-// Combine splits, divide, gate: y[b][h*128 + d] = bf16(sigmoid(g[b][h]) * o).
-__global__ void __launch_bounds__(128) k_attn_merge(const float* __restrict__ part, int splits,
-                                                    const float* __restrict__ gate, bf16* __restrict__ y) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int b = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
-  const float* p = part + ((size_t)b * HQ + h) * splits * (HD + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, p[(size_t)s * (HD + 2) + HD]);
-  float l = 0.f, o = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float ms = p[(size_t)s * (HD + 2) + HD];
-    if (ms == -INFINITY) continue;
-    const float f = __expf(ms - M);
-    l += f * p[(size_t)s * (HD + 2) + HD + 1];
-    o += f * p[(size_t)s * (HD + 2) + d];
-  }
-  const float gt = sigmoidf_(gate[b * HQ + h]);
-  y[(size_t)b * HQ * HD + h * HD + d] = f2bf(gt * (o / l));
-}
-
-// Fixed scratch for callers that cannot allocate device memory (lfm3_decode_step_noalloc): 4 MiB
-// of split-KV partials, one copy per GPU that loads the library, kept until the process exits.
-// Host code never names the array directly: the symbol is a host-side stand-in, so its device
-// address is looked up once per device (with that device current) and passed to the kernels.
-constexpr size_t ATTN_STATIC_FLOATS = (size_t(4) << 20) / sizeof(float);
-static __device__ __align__(256) float g_attn_static[ATTN_STATIC_FLOATS];
-
-cudaError_t attn_static_scratch(float** ptr, size_t* nfloats) {
-  static std::mutex mu;
-  static float* addr[128] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_attn_static);
-    if (e != cudaSuccess) return e;
-    addr[dev] = static_cast<float*>(p);
-  }
-  *ptr = addr[dev];
-  *nfloats = ATTN_STATIC_FLOATS;
-  return cudaSuccess;
-}
-
-cudaError_t attn_decode(const bf16* q, Rows rows, AttnLayer L, int splits, float* part, const float* gate, bf16* y,
-                        cudaStream_t s) {
-  cudaError_t e = launch(k_attn_decode, dim3(splits, HKV, rows.n), dim3(128), DEC_SMEM, s, q, rows, L, splits, part);
-  if (e != cudaSuccess) return e;
-  return launch(k_attn_merge, dim3(rows.n, HQ), dim3(HD), 0, s, part, splits, gate, y);
-}
-
-// ------------------------------------------------------------------------------------------ decode, one kernel
-// Decode attention of one layer in one launch, from the raw q|k|v|gate projection (fp32, one row
-// per stream): block (split, kv head, stream) normalises and rotates its four query heads and
-// the head's new key (RMS over the head, gain, rotary pairs (i, i + 64), bf16) and rounds the
-// new value; it scores its key range with the new key and value standing in for the current
-// position's cache row, which the block holding that position also writes. The cached rows are
-// staged before the block waits for the projection kernel (they do not depend on it). The last
-// block of a (stream, kv head) to finish - counted with an atomic - merges the splits, applies
-// the sigmoid gate and writes the bf16 output, then resets the count for the next layer.
-__global__ void __launch_bounds__(128) k_attn_decode_fused(const float* __restrict__ qkvg, Rows rows, AttnLayer L,
-                                                           AttnDecodeArgs A, int splits, float* __restrict__ part,
-                                                           bf16* __restrict__ y) {
-  extern __shared__ __align__(16) unsigned char dsm[];
-  bf16* ks = reinterpret_cast<bf16*>(dsm);
-  bf16* vs = ks + DEC_SPLIT * HD;
-  __shared__ float qs[GQA][HD];
-  __shared__ float kn[HD], vn[HD];
-  __shared__ float sc[GQA][DEC_SPLIT];
-  __shared__ float ored[2][GQA][HD];
-  __shared__ float ml[GQA][2];
-  __shared__ float red[GQA + 1][4];
-  __shared__ int last;
-  const int sp = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int slot = rows.slot[b], pos = rows.pos[b];
-  const int span = L.full ? DEC_SPLIT : DEC_SPLIT_RING;
-  const int nkeys = L.full ? pos + 1 : min(pos + 1, WIN);  // ring: slots 0..nkeys-1 are live
-  const int cur = L.full ? pos : pos % WIN;                 // index of the current position's key
-  const int j0 = sp * span, j1 = min(nkeys, j0 + span), cnt = j1 - j0;
-  auto row_ptr = [&](const bf16* base, int j) -> const bf16* {
-    if (L.full) {
-      const int page = L.page_table[(size_t)slot * L.max_pages + j / PAGE];
-      return base + (((size_t)page * HKV + kvh) * PAGE + j % PAGE) * HD;
-    }
-    return base + (((size_t)slot * HKV + kvh) * WIN + j) * HD;
-  };
-  // ---- stage the split's keys / values: whole 64-position blocks, each contiguous in the pool
-  // (a page of one kv head) or the ring, one bulk copy per block for K and one for V. Rows past
-  // the visible keys and the current position's stale row come along and are never used.
-  __shared__ __align__(8) uint64_t kv_bar;
-  const int nblk = cnt > 0 ? (cnt + 63) / 64 : 0;
+  const int cur = L.full ? pos : pos % WIN;  // key index of the current position
+  const int j0 = sp * DEC_KEYS, cnt = min(nkeys - j0, DEC_KEYS);
+  const size_t tile = L.full ? ((size_t)L.page_table[(size_t)slot * L.max_pages + sp] * HKV + kvh) * PAGE * HD
+                             : (((size_t)slot * HKV + kvh) * WIN + j0) * HD;
   if (tid == 0) {
     mbar_init(su32(&kv_bar), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    if (nblk) {
-      mbar_expect_tx(su32(&kv_bar), (uint32_t)nblk * 2 * 64 * HD * 2);
-      for (int i = 0; i < nblk; ++i) {
-        bulk_g2s(su32(ks + i * 64 * HD), row_ptr(L.k, j0 + 64 * i), 64 * HD * 2, su32(&kv_bar));
-        bulk_g2s(su32(vs + i * 64 * HD), row_ptr(L.v, j0 + 64 * i), 64 * HD * 2, su32(&kv_bar));
-      }
-    }
+    mbar_expect_tx(su32(&kv_bar), DA_SMEM);
+    bulk_g2s(su32(ks), L.k + tile, DA_TILE, su32(&kv_bar));
+    bulk_g2s(su32(vs), L.v + tile, DA_TILE, su32(&kv_bar));
   }
-  // gains and rotary coefficients of this thread's dimension d = tid are weights too
-  const int d = tid, pd = d < 64 ? d + 64 : d - 64, ir = d & 63;
+  // gains and rotary coefficients of dimension d = tid (threads < 128) are weights too
+  const int d = tid & (HD - 1), pd = d < 64 ? d + 64 : d - 64, ir = d & 63;
   const float gq = bf2f(A.q_norm[d]), gk = bf2f(A.k_norm[d]);
   const float cr = A.rope_cos[(size_t)pos * (HD / 2) + ir], sr = A.rope_sin[(size_t)pos * (HD / 2) + ir];
   pdl_wait();
   pdl_launch_dependents();
-  // ---- queries and the new key / value: thread = dimension d of each of the 4 heads
+
+  // ---- queries and the new key / value (threads 0..127: thread = dimension d of each head)
   const float* raw = qkvg + (size_t)b * NQKVG;
-  float qv[GQA], s2[GQA + 1];
+  float qv[GQA], kv = 0.f, vv = 0.f;
+  if (tid < HD) {
+    float s2[GQA + 1];
 #pragma unroll
-  for (int hh = 0; hh < GQA; ++hh) {
-    qv[hh] = raw[(kvh * GQA + hh) * HD + d];
-    s2[hh] = warp_sum(qv[hh] * qv[hh]);
+    for (int hh = 0; hh < GQA; ++hh) {
+      qv[hh] = raw[(kvh * GQA + hh) * HD + d];
+      s2[hh] = warp_sum(qv[hh] * qv[hh]);
+    }
+    kv = raw[HQ * HD + kvh * HD + d];
+    vv = raw[HQ * HD + HKV * HD + kvh * HD + d];
+    s2[GQA] = warp_sum(kv * kv);
+    if (lane == 0)
+#pragma unroll
+      for (int hh = 0; hh <= GQA; ++hh) red[hh][warp] = s2[hh];
   }
-  const float kv = raw[HQ * HD + kvh * HD + d];
-  const float vv = raw[HQ * HD + HKV * HD + kvh * HD + d];
-  s2[GQA] = warp_sum(kv * kv);
-  if (lane == 0)
-#pragma unroll
-    for (int hh = 0; hh <= GQA; ++hh) red[hh][warp] = s2[hh];
   __syncthreads();
+  if (tid < HD) {
 #pragma unroll
-  for (int hh = 0; hh < GQA; ++hh) {
-    const float inv = rsqrtf((red[hh][0] + red[hh][1] + red[hh][2] + red[hh][3]) * (1.0f / HD) + A.eps);
-    qs[hh][d] = gq * (qv[hh] * inv);
+    for (int hh = 0; hh < GQA; ++hh) {
+      const float inv = rsqrtf((red[hh][0] + red[hh][1] + red[hh][2] + red[hh][3]) * (1.0f / HD) + A.eps);
+      qs[hh][d] = gq * (qv[hh] * inv);
+    }
+    kb[d] = gk * (kv * rsqrtf((red[GQA][0] + red[GQA][1] + red[GQA][2] + red[GQA][3]) * (1.0f / HD) + A.eps));
   }
-  kn[d] = gk * (kv * rsqrtf((red[GQA][0] + red[GQA][1] + red[GQA][2] + red[GQA][3]) * (1.0f / HD) + A.eps));
-  vn[d] = round_bf(vv);
+  __syncthreads();
+  // rotary on pairs (i, i + 64); q and k rounded to bf16 (their stored precision)
+  float qr[GQA], kr = 0.f;
+  if (tid < HD) {
+#pragma unroll
+    for (int hh = 0; hh < GQA; ++hh)
+      qr[hh] = round_bf(d < 64 ? qs[hh][d] * cr - qs[hh][pd] * sr : qs[hh][d] * cr + qs[hh][pd] * sr);
+    kr = round_bf(d < 64 ? kb[d] * cr - kb[pd] * sr : kb[d] * cr + kb[pd] * sr);
+  }
   __syncthreads();
   const float scale = rsqrtf((float)HD);
-  float qr[GQA];
+  const bool has_cur = cur >= j0 && cur < j0 + cnt;
+  if (tid < HD) {
 #pragma unroll
-  for (int hh = 0; hh < GQA; ++hh) qr[hh] = d < 64 ? qs[hh][d] * cr - qs[hh][pd] * sr : qs[hh][d] * cr + qs[hh][pd] * sr;
-  const float kr = d < 64 ? kn[d] * cr - kn[pd] * sr : kn[d] * cr + kn[pd] * sr;
+    for (int hh = 0; hh < GQA; ++hh) qs[hh][d] = qr[hh] * scale;
+    if (has_cur) {  // the new key and value into the cache, as every later step reads them
+      const size_t row = tile + (size_t)(cur - j0) * HD + d;
+      const_cast<bf16*>(L.k)[row] = f2bf(kr);
+      const_cast<bf16*>(L.v)[row] = f2bf(vv);
+    }
+  }
+  // ---- the staged split; the current position's row there is stale: put the new one in
+  bool ok = mbar_wait(su32(&kv_bar), 0, A.err);
+  if (!ok) ok = mbar_wait(su32(&kv_bar), 0, A.err);  // a copy still in flight must land before exit
+  if (has_cur && tid < HD) {
+    ks[(cur - j0) * HD + d] = f2bf(kr);
+    vs[(cur - j0) * HD + d] = f2bf(vv);
+  }
   __syncthreads();
+
+  const size_t mloff = da_ml_offset(rows.n, splits);
+  const size_t hbase = ((size_t)b * HQ + kvh * GQA) * splits;  // (stream, first head of the group) x splits
+  if (ok) {
+    // ---- scores: warp w takes keys 8w .. 8w+7; lane l holds dims 4l..4l+3 of the four queries
+    {
+      float4 q4[GQA];
 #pragma unroll
-  for (int hh = 0; hh < GQA; ++hh) qs[hh][d] = round_bf(qr[hh]) * scale;
-  kn[d] = round_bf(kr);
-  const bool has_cur = cur >= j0 && cur < j1;
-  if (has_cur) {  // the new key and value into the cache (bf16, as every later step reads them)
-    bf16* kd = const_cast<bf16*>(row_ptr(L.k, cur));
-    bf16* vd = const_cast<bf16*>(row_ptr(L.v, cur));
-    kd[d] = f2bf(kn[d]);
-    vd[d] = f2bf(vn[d]);
-  }
-  __syncthreads();  // also orders the barrier's initialisation before every thread's wait
-  if (nblk && !mbar_wait(su32(&kv_bar), 0, A.err)) {
-    // a copy that never lands: report through the status word, drop this block's partial
-    asm volatile("" ::: "memory");
-  }
-  float* out = part + (((size_t)b * HQ + kvh * GQA) * splits + sp) * (HD + 2);
-  if (cnt > 0) {
-    // scores: one key per thread (span <= 128)
-    if (tid < cnt) {
-      float s[GQA] = {0.f, 0.f, 0.f, 0.f};
-      if (j0 + tid == cur) {
-        for (int c = 0; c < HD; ++c)
+      for (int hh = 0; hh < GQA; ++hh) q4[hh] = *reinterpret_cast<const float4*>(&qs[hh][4 * lane]);
+      float v[32];  // v[h * 8 + k]: this lane's partial dot of head h with key 8w + k
 #pragma unroll
-          for (int hh = 0; hh < GQA; ++hh) s[hh] += qs[hh][c] * kn[c];
-      } else {
-#pragma unroll 4
-        for (int c = 0; c < 16; ++c) {
-          // rows are 256 B apart: rotating the chunk order by the key spreads a warp's reads over all
-          // banks (and the q chunks it needs over 8 broadcast groups)
-          const int ch = (c + tid) & 15;
-          const uint4 w = *reinterpret_cast<const uint4*>(ks + tid * HD + ch * 8);
-          const float k8[8] = {bflo(w.x), bfhi(w.x), bflo(w.y), bfhi(w.y), bflo(w.z), bfhi(w.z), bflo(w.w), bfhi(w.w)};
+      for (int k = 0; k < 8; ++k) {
+        const uint2 kk = *reinterpret_cast<const uint2*>(ks + (8 * warp + k) * HD + 4 * lane);
+        const float k0 = bflo(kk.x), k1 = bfhi(kk.x), k2 = bflo(kk.y), k3 = bfhi(kk.y);
 #pragma unroll
-          for (int hh = 0; hh < GQA; ++hh)
+        for (int hh = 0; hh < GQA; ++hh) v[hh * 8 + k] = q4[hh].x * k0 + q4[hh].y * k1 + q4[hh].z * k2 + q4[hh].w * k3;
+      }
+      // butterfly: at offset o each lane keeps the half of its values selected by bit o of its
+      // lane id and adds the partner's; after five steps lane l holds the full sum of value l
 #pragma unroll
-            for (int e = 0; e < 8; ++e) s[hh] += qs[hh][ch * 8 + e] * k8[e];
+      for (int o = 16, c = 32; o >= 1; o >>= 1, c >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < c / 2; ++i) {
+          const float send = up ? v[i] : v[i + c / 2];
+          const float keep = up ? v[i + c / 2] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
         }
       }
-#pragma unroll
-      for (int hh = 0; hh < GQA; ++hh) sc[hh][tid] = s[hh];
+      const int hh = lane >> 3, j = 8 * warp + (lane & 7);
+      sc[hh][j] = j < cnt ? v[0] : -INFINITY;
     }
     __syncthreads();
-    {
-      const int hh = warp;
-      float mx = -INFINITY;
-      for (int j = lane; j < cnt; j += 32) mx = fmaxf(mx, sc[hh][j]);
-      mx = warp_max(mx);
-      float l = 0.f;
-      for (int j = lane; j < cnt; j += 32) {
-        const float p = __expf(sc[hh][j] - mx);
-        sc[hh][j] = p;
-        l += p;
+    // ---- softmax of this split: warp h < 4 takes head h
+    if (warp < GQA) {
+      const float s0 = sc[warp][lane], s1 = sc[warp][lane + 32];
+      const float m = warp_max(fmaxf(s0, s1));
+      const float p0 = __expf(s0 - m), p1 = __expf(s1 - m);
+      reinterpret_cast<float*>(&pr[lane])[warp] = p0;
+      reinterpret_cast<float*>(&pr[lane + 32])[warp] = p1;
+      const float l = warp_sum(p0 + p1);
+      if (lane == 0) {
+        part[mloff + 2 * (hbase + (size_t)warp * splits + sp)] = m;
+        part[mloff + 2 * (hbase + (size_t)warp * splits + sp) + 1] = l;
       }
-      l = warp_sum(l);
-      if (lane == 0) { ml[hh][0] = mx; ml[hh][1] = l; }
     }
     __syncthreads();
+    // ---- P V: thread = (key quarter, dimension pair); rows past the split's keys are never read
     {
-      const int par = tid >> 6, dp = (tid & 63) * 2;
+      const int qt = tid >> 6, dp = 2 * (tid & 63);
+      const int je = min(cnt, 16 * qt + 16);
       float o[GQA][2] = {};
-#pragma unroll 4
-      for (int j = par; j < cnt; j += 2) {
-        float v0, v1;
-        if (j0 + j == cur) {
-          v0 = vn[dp];
-          v1 = vn[dp + 1];
-        } else {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(vs + j * HD + dp);
-          v0 = bflo(w);
-          v1 = bfhi(w);
-        }
-#pragma unroll
-        for (int hh = 0; hh < GQA; ++hh) {
-          const float p = sc[hh][j];
-          o[hh][0] += p * v0;
-          o[hh][1] += p * v1;
-        }
+      for (int j = 16 * qt; j < je; ++j) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(vs + j * HD + dp);
+        const float v0 = bflo(w), v1 = bfhi(w);
+        const float4 p = pr[j];
+        o[0][0] += p.x * v0; o[0][1] += p.x * v1;
+        o[1][0] += p.y * v0; o[1][1] += p.y * v1;
+        o[2][0] += p.z * v0; o[2][1] += p.z * v1;
+        o[3][0] += p.w * v0; o[3][1] += p.w * v1;
       }
 #pragma unroll
-      for (int hh = 0; hh < GQA; ++hh) { ored[par][hh][dp] = o[hh][0]; ored[par][hh][dp + 1] = o[hh][1]; }
+      for (int hh = 0; hh < GQA; ++hh) *reinterpret_cast<float2*>(&obuf[qt][hh][dp]) = make_float2(o[hh][0], o[hh][1]);
     }
     __syncthreads();
-    for (int e = tid; e < GQA * HD; e += blockDim.x) {
-      const int hh = e / HD, dd = e % HD;
-      out[(size_t)hh * splits * (HD + 2) + dd] = ored[0][hh][dd] + ored[1][hh][dd];
+    if (tid < GQA * HD / 4) {
+      const int hh = tid >> 5, d4 = 4 * lane;
+      float4 s = *reinterpret_cast<const float4*>(&obuf[0][hh][d4]);
+#pragma unroll
+      for (int qt = 1; qt < 4; ++qt) {
+        const float4 t = *reinterpret_cast<const float4*>(&obuf[qt][hh][d4]);
+        s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
+      }
+      *reinterpret_cast<float4*>(part + (hbase + (size_t)hh * splits + sp) * HD + d4) = s;
     }
+  } else {  // a copy that never landed: this split contributes nothing
     if (tid < GQA) {
-      out[(size_t)tid * splits * (HD + 2) + HD] = ml[tid][0];
-      out[(size_t)tid * splits * (HD + 2) + HD + 1] = ml[tid][1];
+      part[mloff + 2 * (hbase + (size_t)tid * splits + sp)] = -INFINITY;
+      part[mloff + 2 * (hbase + (size_t)tid * splits + sp) + 1] = 0.f;
     }
-  } else {  // empty split
-    for (int e = tid; e < GQA * (HD + 2); e += blockDim.x) {
-      const int hh = e / (HD + 2), k = e % (HD + 2);
-      out[(size_t)hh * splits * (HD + 2) + k] = (k == HD) ? -INFINITY : 0.f;
-    }
+    if (tid < GQA * HD / 4)
+      *reinterpret_cast<float4*>(part + (hbase + (size_t)(tid >> 5) * splits + sp) * HD + 4 * lane) =
+          make_float4(0.f, 0.f, 0.f, 0.f);
   }
+
   // ---- the last block of (stream, kv head) merges the splits and applies the gates
+  __threadfence();
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    unsigned* ctr = A.counters + b * HKV + kvh;
-    last = atomicAdd(ctr, 1u) == (unsigned)(splits - 1);
-  }
+  if (tid == 0) last = atomicAdd(A.counters + b * HKV + kvh, 1u) == (unsigned)(nact - 1);
   __syncthreads();
   if (!last) return;
   __threadfence();
-  for (int hh = 0; hh < GQA; ++hh) {
-    const float* pp = part + ((size_t)b * HQ + kvh * GQA + hh) * splits * (HD + 2);
-    float M = -INFINITY, l = 0.f, o = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const float* q = pp + (size_t)s * (HD + 2);
-      const float ms = __ldcg(q + HD), ls = __ldcg(q + HD + 1), os = __ldcg(q + d);
-      if (ms == -INFINITY) continue;
-      const float Mn = fmaxf(M, ms);
-      const float fo = __expf(M - Mn), fs = __expf(ms - Mn);
-      l = l * fo + ls * fs;
-      o = o * fo + os * fs;
-      M = Mn;
+  // warp w: head w & 3 over the splits s = half, half + 2, ... (half = w >> 2)
+  const int hh = warp & 3, half = warp >> 2;
+  const size_t hb = hbase + (size_t)hh * splits;
+  const float2* ml = reinterpret_cast<const float2*>(part + mloff);
+  float M = -INFINITY;
+  for (int s = lane; s < nact; s += 32) M = fmaxf(M, __ldcg(&ml[hb + s].x));
+  M = warp_max(M);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.f;
+  for (int s0 = 0; s0 < nact; s0 += 32) {
+    const int s = s0 + lane;
+    float wgt = 0.f;
+    if (s < nact) {
+      const float2 m2 = __ldcg(&ml[hb + s]);
+      wgt = m2.x == -INFINITY ? 0.f : __expf(m2.x - M);
+      if ((s & 1) == half) lsum += wgt * m2.y;
     }
-    const float gt = sigmoidf_(raw[HQ * HD + 2 * HKV * HD + kvh * GQA + hh]);
-    y[(size_t)b * HQ * HD + (kvh * GQA + hh) * HD + d] = f2bf(gt * (o / l));
+    const int ns = min(32, nact - s0);
+#pragma unroll 8
+    for (int i = half; i < ns; i += 2) {
+      const float wi = __shfl_sync(0xffffffffu, wgt, i);
+      const float4 o = __ldcg(reinterpret_cast<const float4*>(part + (hb + s0 + i) * HD) + lane);
+      acc.x += wi * o.x; acc.y += wi * o.y; acc.z += wi * o.z; acc.w += wi * o.w;
+    }
+  }
+  lsum = warp_sum(lsum);
+  if (half == 1) {
+    *reinterpret_cast<float4*>(&obuf[0][hh][4 * lane]) = acc;
+    if (lane == 0) lx[hh] = lsum;
+  }
+  __syncthreads();
+  if (half == 0) {
+    const float4 t = *reinterpret_cast<const float4*>(&obuf[0][hh][4 * lane]);
+    const float l = lsum + lx[hh];
+    const float gt = sigmoidf_(raw[HQ * HD + 2 * HKV * HD + kvh * GQA + hh]) / l;
+    bf16* yo = y + (size_t)b * HQ * HD + (kvh * GQA + hh) * HD + 4 * lane;
+    uint2 w;
+    w.x = pack_bf2(gt * (acc.x + t.x), gt * (acc.y + t.y));
+    w.y = pack_bf2(gt * (acc.z + t.z), gt * (acc.w + t.w));
+    *reinterpret_cast<uint2*>(yo) = w;
   }
   if (tid == 0) A.counters[b * HKV + kvh] = 0u;
 }
 
 cudaError_t attn_decode_fused(const float* qkvg, Rows rows, AttnLayer L, const AttnDecodeArgs& A, int splits,
                               float* part, bf16* y, cudaStream_t s) {
-  return launch(k_attn_decode_fused, dim3(splits, HKV, rows.n), dim3(128), DEC_SMEM, s, qkvg, rows, L, A, splits, part,
-                y);
-}
-
-// ------------------------------------------------------------------------------------------ prefill
-constexpr int PA_ROWS = 32;        // query rows per block
-constexpr int PA_KT = 64;          // keys per tile
-constexpr int PA_THREADS = 256;    // 8 warps
-constexpr int PA_TILE_BYTES = PA_KT * HD * 2;   // 16 KB per K or V tile
-
-DEVI uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-// 16-byte chunk c (0..15) of row r in a [64][128] bf16 tile, XOR-swizzled against bank conflicts.
-DEVI uint32_t tile_off(int r, int c) { return (uint32_t)(r * 256 + ((c ^ (r & 7)) << 4)); }
-
-DEVI void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0));
-}
-DEVI void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-template <int N>
-DEVI void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
-
-DEVI void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-DEVI void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-
-struct PrefillArgs {
-  const bf16* q;     // [n][HQ][HD]
-  int n, p0, slot;
-  AttnLayer L;
-  const bf16* sk; const bf16* sv; int scratch_rows;
-  const float* gate; // [n][HQ]
-  bf16* y;           // [n][HQ*HD]
-};
-
-__global__ void __launch_bounds__(PA_THREADS) k_attn_prefill(const PrefillArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  pdl_wait();
-  pdl_launch_dependents();
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int kvh = blockIdx.y;
-  const int h = kvh * GQA + (warp & 3);
-  const int r0 = blockIdx.x * PA_ROWS + (warp >> 2) * 16;   // this warp's first row
-  const int rb0 = blockIdx.x * PA_ROWS;                    // block's first row
-  const int rb1 = min(a.n, rb0 + PA_ROWS) - 1;             // block's last row
-  const bool full = a.L.full;
-  // key index space: full -> positions; sliding -> scratch index i (position p0 - WIN + i)
-  const int koff = full ? 0 : a.p0 - WIN;
-  const int qpos_lo = a.p0 + rb0, qpos_hi = a.p0 + rb1;
-  int klo = full ? 0 : max(0, qpos_lo - (WIN - 1)) - koff;
-  const int khi = qpos_hi - koff;                          // last index needed (inclusive)
-  const int kmax_valid = a.p0 + a.n - 1 - koff;            // last written key
-  klo = (klo / PA_KT) * PA_KT;
-  const int ntiles = (khi - klo) / PA_KT + 1;
-
-  // Q fragments (16 rows x 128 dims): 8 k-steps x 4 regs
-  uint32_t qf[8][4];
-  {
-    const int ra = r0 + g, rbb = r0 + g + 8;
-    const bool va = ra < a.n, vb = rbb < a.n;
-    const bf16* qa = a.q + ((size_t)(va ? ra : 0) * HQ + h) * HD;
-    const bf16* qb = a.q + ((size_t)(vb ? rbb : 0) * HQ + h) * HD;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      qf[ks][0] = va ? *reinterpret_cast<const uint32_t*>(qa + ks * 16 + 2 * t) : 0u;
-      qf[ks][1] = vb ? *reinterpret_cast<const uint32_t*>(qb + ks * 16 + 2 * t) : 0u;
-      qf[ks][2] = va ? *reinterpret_cast<const uint32_t*>(qa + ks * 16 + 8 + 2 * t) : 0u;
-      qf[ks][3] = vb ? *reinterpret_cast<const uint32_t*>(qb + ks * 16 + 8 + 2 * t) : 0u;
-    }
-  }
-  const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;  // scale * log2(e)
-  float o[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-  const int qp0 = a.p0 + r0 + g, qp1 = qp0 + 8;  // query positions of this lane's two rows
-
-  auto issue_tile = [&](int it, int buf) {
-    const int kt0 = klo + it * PA_KT;
-    unsigned char* kb = smem + buf * 2 * PA_TILE_BYTES;
-    unsigned char* vb = kb + PA_TILE_BYTES;
-    const bf16 *ksrc, *vsrc;
-    if (full) {
-      const int page = a.L.page_table[(size_t)a.slot * a.L.max_pages + kt0 / PAGE];
-      const size_t off = ((size_t)page * HKV + kvh) * PAGE * HD;
-      ksrc = a.L.k + off;
-      vsrc = a.L.v + off;
-    } else {
-      const size_t off = ((size_t)kvh * a.scratch_rows + kt0) * HD;
-      ksrc = a.sk + off;
-      vsrc = a.sv + off;
-    }
-    // 64 rows x 16 chunks = 1024 chunks per tensor; 4 per thread each
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int idx = tid + e * PA_THREADS, r = idx >> 4, c = idx & 15;
-      const bool valid = kt0 + r <= kmax_valid;
-      const size_t so = valid ? (size_t)r * HD + c * 8 : 0;
-      cp_async16(smem_u32(kb) + tile_off(r, c), ksrc + so, valid);
-      cp_async16(smem_u32(vb) + tile_off(r, c), vsrc + so, valid);
-    }
-    cp_async_commit();
-  };
-
-  issue_tile(0, 0);
-  for (int it = 0; it < ntiles; ++it) {
-    const int buf = it & 1;
-    if (it + 1 < ntiles) {
-      issue_tile(it + 1, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint32_t kb = smem_u32(smem + buf * 2 * PA_TILE_BYTES);
-    const uint32_t vb = kb + PA_TILE_BYTES;
-    const int kt0 = klo + it * PA_KT;
-    // S = Q K^T : 16 x 64
-    float s[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ks += 2) {
-        const int m = lane >> 3;  // matrix: (ks, lo), (ks, hi), (ks+1, lo), (ks+1, hi)
-        const int r = nt * 8 + (lane & 7);
-        const int c = (ks + (m >> 1)) * 2 + (m & 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kb + tile_off(r, c), b0, b1, b2, b3);
-        mma_bf16_16816(s[nt], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b0, b1);
-        mma_bf16_16816(s[nt], qf[ks + 1][0], qf[ks + 1][1], qf[ks + 1][2], qf[ks + 1][3], b2, b3);
-      }
-    }
-    // mask + online softmax (rows g and g+8 of this warp)
-    float mnew[2] = {mrow[0], mrow[1]};
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int kp = kt0 + nt * 8 + 2 * t + (j & 1) + koff;   // key position
-        const int qp = (j < 2) ? qp0 : qp1;
-        bool ok = kp <= qp && kp >= 0;
-        if (!full) ok = ok && (qp - kp < WIN);
-        s[nt][j] = ok ? s[nt][j] * sl2 : -INFINITY;
-        mnew[j >> 1] = fmaxf(mnew[j >> 1], s[nt][j]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      mnew[i] = fmaxf(mnew[i], __shfl_xor_sync(0xffffffffu, mnew[i], 1));
-      mnew[i] = fmaxf(mnew[i], __shfl_xor_sync(0xffffffffu, mnew[i], 2));
-    }
-    float alpha[2], mu[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      mu[i] = mnew[i] == -INFINITY ? 0.f : mnew[i];
-      alpha[i] = exp2f(mrow[i] - mu[i]);
-      mrow[i] = mnew[i];
-    }
-    float lsum[2] = {0.f, 0.f};
-    uint32_t pf[4][4];  // P as A fragments: 4 k-steps of 16 keys
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const float p0 = exp2f(s[nt][0] - mu[0]), p1 = exp2f(s[nt][1] - mu[0]);
-      const float p2 = exp2f(s[nt][2] - mu[1]), p3 = exp2f(s[nt][3] - mu[1]);
-      lsum[0] += p0 + p1;
-      lsum[1] += p2 + p3;
-      const int kk = nt >> 1;
-      if ((nt & 1) == 0) {
-        pf[kk][0] = pack_bf2(p0, p1);
-        pf[kk][1] = pack_bf2(p2, p3);
-      } else {
-        pf[kk][2] = pack_bf2(p0, p1);
-        pf[kk][3] = pack_bf2(p2, p3);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      lsum[i] += __shfl_xor_sync(0xffffffffu, lsum[i], 1);
-      lsum[i] += __shfl_xor_sync(0xffffffffu, lsum[i], 2);
-      lrow[i] = lrow[i] * alpha[i] + lsum[i];
-    }
-#pragma unroll
-    for (int dt = 0; dt < 16; ++dt) {
-      o[dt][0] *= alpha[0]; o[dt][1] *= alpha[0];
-      o[dt][2] *= alpha[1]; o[dt][3] *= alpha[1];
-    }
-    // O += P V : V tile [64 keys][128 dims], B fragments via transposed ldmatrix
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-      for (int dt = 0; dt < 16; dt += 2) {
-        const int m = lane >> 3;  // (keys lo, dt), (keys hi, dt), (keys lo, dt+1), (keys hi, dt+1)
-        const int r = kk * 16 + (m & 1) * 8 + (lane & 7);
-        const int c = dt + (m >> 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vb + tile_off(r, c), b0, b1, b2, b3);
-        mma_bf16_16816(o[dt], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], b0, b1);
-        mma_bf16_16816(o[dt + 1], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], b2, b3);
-      }
-    }
-    __syncthreads();
-  }
-  // epilogue: divide, gate, store bf16
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int r = r0 + g + 8 * i;
-    if (r >= a.n) continue;
-    const float gt = sigmoidf_(a.gate[r * HQ + h]) / lrow[i];
-    bf16* dst = a.y + (size_t)r * HQ * HD + h * HD;
-#pragma unroll
-    for (int dt = 0; dt < 16; ++dt)
-      *reinterpret_cast<uint32_t*>(dst + dt * 8 + 2 * t) = pack_bf2(o[dt][2 * i] * gt, o[dt][2 * i + 1] * gt);
-  }
-}
-
-cudaError_t attn_prefill(const bf16* q, int n, int p0, int slot, AttnLayer L, const bf16* sk, const bf16* sv,
-                         int scratch_rows, const float* gate, bf16* y, cudaStream_t s) {
-  PrefillArgs a{q, n, p0, slot, L, sk, sv, scratch_rows, gate, y};
-  const size_t sm = 4 * PA_TILE_BYTES;
-  return launch(k_attn_prefill, dim3((n + PA_ROWS - 1) / PA_ROWS, HKV), dim3(PA_THREADS), sm, s, a);
+  return launch(k_attn_decode_fused, dim3(splits, HKV, rows.n), dim3(DA_THREADS), DA_SMEM, s, qkvg, rows, L, A, splits,
+                part, y);
 }
 
 cudaError_t attn_init() {
-  cudaError_t e = cudaFuncSetAttribute(k_attn_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM);
+  return cudaFuncSetAttribute(k_attn_decode_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, DA_SMEM);
+}
+
+// ------------------------------------------------------------------------------------------ fixed scratch
+// Fixed scratch for callers that cannot allocate device memory (lfm3_decode_step_noalloc): 4 MiB
+// of split partials, one copy per GPU that loads the library, kept until the process exits.
+// Host code never names the array directly: the symbol is a host-side stand-in, so its device
+// address is looked up with the device current and passed to the kernels. The address is kept
+// per CUDA context, so a context destroyed and made again (cudaDeviceReset) is looked up anew.
+constexpr size_t ATTN_STATIC_FLOATS = (size_t(4) << 20) / sizeof(float);
+static __device__ __align__(256) float g_attn_static[ATTN_STATIC_FLOATS];
+
+cudaError_t attn_static_scratch(float** ptr, size_t* nfloats) {
+  static std::mutex mu;
+  static std::vector<std::pair<unsigned long long, float*>> cache;  // (context id, address)
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!get_ctx || !get_id) {
+    cudaDriverEntryPointQueryResult q1, q2;
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+      return cudaErrorNotSupported;
+    get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f1);
+    get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f2);
+  }
+  // the current context's id (unique for the life of the process, unlike its handle)
+  auto current_id = [&](unsigned long long* id) -> bool {
+    CUcontext cx = nullptr;
+    return get_ctx(&cx) == CUDA_SUCCESS && cx && get_id(cx, id) == CUDA_SUCCESS;
+  };
+  unsigned long long id = 0;
+  if (current_id(&id))
+    for (auto& c : cache)
+      if (c.first == id) {
+        *ptr = c.second;
+        *nfloats = ATTN_STATIC_FLOATS;
+        return cudaSuccess;
+      }
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_attn_static);  // also makes the device's context current
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_attn_decode_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_attn_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, 4 * PA_TILE_BYTES);
+  if (!current_id(&id)) return cudaErrorInvalidDevice;
+  cache.emplace_back(id, static_cast<float*>(p));
+  *ptr = static_cast<float*>(p);
+  *nfloats = ATTN_STATIC_FLOATS;
+  return cudaSuccess;
 }
 
 }  // namespace lfm3

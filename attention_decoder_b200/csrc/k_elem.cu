@@ -278,9 +278,6 @@ __global__ void __launch_bounds__(256) k_qk_norm_rope_kv(const float* __restrict
     const int slot = rows.slot[r];
     const int page = kv.page_table[(size_t)slot * kv.max_pages + pos / PAGE];
     off = (((size_t)page * HKV + kvh) * PAGE + pos % PAGE) * HD;
-  } else if (kv.mode == KV_RING) {
-    const int slot = rows.slot[r];
-    off = (((size_t)slot * HKV + kvh) * WIN + pos % WIN) * HD;
   } else {
     off = ((size_t)kvh * kv.scratch_rows + WIN + r) * HD;
   }
@@ -370,6 +367,27 @@ cudaError_t finish_step(int32_t* seq_len, const int32_t* row_slot, int rows, int
                         const unsigned long long* amax, int32_t* argmax_out, cudaStream_t s) {
   return launch(k_finish, dim3(1), dim3(64), 0, s, seq_len, row_slot, rows, add_prefill, prefill_slot, amax,
                 argmax_out);
+}
+
+// ------------------------------------------------------------------------------------------
+// Self-test of the failure path: one thread waits on a fresh mbarrier that nothing will ever
+// arrive on, with the given iteration limit (the kernels' own waits use WAIT_LIMIT); when the
+// limit runs out it records the failure in the status word, as every bounded wait does, and
+// the kernel returns. Nothing is copied into the barrier's transaction, so nothing is in flight.
+__global__ void k_wait_selftest(int* err, unsigned rounds) {
+  __shared__ __align__(8) uint64_t bar;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (threadIdx.x != 0) return;
+  mbar_init(su32(&bar), 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  for (unsigned i = 0; i < rounds; ++i)
+    if (mbar_try(su32(&bar), 0)) return;
+  atomicExch(err, 2);
+}
+
+cudaError_t wait_selftest(int* err, unsigned rounds, cudaStream_t s) {
+  return launch(k_wait_selftest, dim3(1), dim3(32), 0, s, err, rounds);
 }
 
 }  // namespace lfm3

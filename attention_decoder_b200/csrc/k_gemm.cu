@@ -593,7 +593,7 @@ static int g_gemm_sms = 0;
 static int g_gemm_pairs = 0;  // clusters of two that fit on the device at once (paired kernel)
 // Paired (2-SM) tiles from this many rows on, for the FFN projections and the wide or deep ones
 // (measured on 2048-row chunks: w13 92.0 -> 91.6 us, w2 48.8 -> 46.8, in_proj 42.5 -> 40.5; the
-// 2048 x 2048 projections are 1.2 us faster on single-SM tiles); LFM3_GEMM_PAIR_MIN_M overrides.
+// 2048 x 2048 projections are 1.2 us faster on single-SM tiles).
 static int g_gemm_pair_min_m = 129;
 
 template <int BN, int EPI>
@@ -640,12 +640,10 @@ static cudaError_t launch_gemm2(const GemmPlan& p, int M, int* err, cudaStream_t
 }
 
 // Output widths from which a tile is 256 columns wide (fewer, more L2-efficient tiles) rather than
-// 128 (more tiles to spread over the SMs); LFM3_GEMM_WIDE_MIN_N overrides.
+// 128 (more tiles to spread over the SMs).
 static int g_gemm_wide_min = 2048;  // measured: 8k prefill 37.8 -> 34.6 ms against 4097
 
 cudaError_t gemm_init() {
-  if (const char* v = getenv("LFM3_GEMM_WIDE_MIN_N")) g_gemm_wide_min = atoi(v);
-  if (const char* v = getenv("LFM3_GEMM_PAIR_MIN_M")) g_gemm_pair_min_m = atoi(v);
   cudaError_t e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;

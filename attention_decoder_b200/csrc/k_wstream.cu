@@ -5,7 +5,7 @@
 // strided list of row tiles. One producer warp copies the tiles' weight rows into a padded ring of
 // shared-memory stages with 1-D bulk asynchronous copies (cp.async.bulk + mbarrier transaction
 // counts), starting before the block waits for the previous kernel - the weights do not depend on
-// it - so each launch's first stages are already in flight when its inputs become ready. Four
+// it - so each launch's first stages are already in flight when its inputs become ready. Eight
 // consumer warps read 16-byte slices of the rows and feed them to the tensor cores as the 16-row A
 // operand of m16n8k16 MMAs whose 8 columns are the streams (the activations are read with the same
 // K permutation). Per-warp partial sums are reduced in shared memory per tile, then:
@@ -53,7 +53,7 @@ struct WsGeom {
   static constexpr int REQB = 64 * BR * NKB;                  // bytes of one request: [block][row][64 B]
   static constexpr int ROWB = 64 * NKB;                       // weight bytes per row per stage
   static constexpr int SCB = FP4 ? KCH / 16 : 0;              // scale bytes per row per stage
-  static constexpr int STAGES = FP4 ? 12 : 5;  // default ring depth (runtime: a.stages); swept on B200
+  static constexpr int STAGES = FP4 ? 12 : 5;  // ring depth (passed as a.stages); swept on B200
   static constexpr int STAGE_BYTES = RPT * ROWB + RPT * SCB;
   static constexpr int TX_BYTES = STAGE_BYTES;
   static constexpr int STEPS = KCH / KB;                      // lane steps per stage
@@ -476,8 +476,7 @@ size_t ws_smem(int NT, int rows, int Kc, int stages) {
 }
 
 static int g_num_sms = 0;
-static int g_ws_bps = 2;     // blocks per SM (LFM3_WS_BLOCKS_PER_SM)
-static int g_ws_stages = 0;  // ring depth override (LFM3_WS_STAGES); 0 = the per-shape default
+constexpr int WS_BPS = 2;  // blocks per SM
 
 template <int EPI, bool FP4>
 static cudaError_t launch_ws(const WsMaps& mp, const WsArgs& a, cudaStream_t s) {
@@ -487,11 +486,11 @@ static cudaError_t launch_ws(const WsMaps& mp, const WsArgs& a, cudaStream_t s) 
   const int ntiles = (EPI == GEMV_SWIGLU) ? a.N / 8 : (EPI == GEMV_CONV ? D / 16 : a.N / 16);
   const int NT = a.rows <= 8 ? 1 : 2;
   WsArgs b = a;
-  b.stages = g_ws_stages > 0 ? g_ws_stages : G::STAGES;
+  b.stages = G::STAGES;
   const size_t smem = ws_smem<EPI, FP4>(NT, a.rows, Kc, b.stages);
   if (smem > (size_t)WS_SMEM_MAX) return cudaErrorInvalidValue;
-  // blocks per K range: g_ws_bps blocks per SM in all, spread evenly over the tiles
-  int gx = std::max(1, g_ws_bps * g_num_sms / a.splits);
+  // blocks per K range: WS_BPS blocks per SM in all, spread evenly over the tiles
+  int gx = std::max(1, WS_BPS * g_num_sms / a.splits);
   gx = std::min(gx, ntiles);
   const int per = (ntiles + gx - 1) / gx;
   gx = (ntiles + per - 1) / per;
@@ -564,8 +563,6 @@ static cudaError_t ws_attr() {
 }
 
 cudaError_t wstream_init() {
-  if (const char* v = getenv("LFM3_WS_BLOCKS_PER_SM")) g_ws_bps = std::max(1, atoi(v));
-  if (const char* v = getenv("LFM3_WS_STAGES")) g_ws_stages = std::max(2, std::min(16, atoi(v)));
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

@@ -62,10 +62,10 @@ cudaError_t conv_decode(const float* bcx, const bf16* conv_w, bf16* state_layer,
                         int rows, bf16* y, cudaStream_t s);
 cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot, int n, bf16* y, cudaStream_t s);
 
-enum KvDst { KV_PAGES = 0, KV_RING = 1, KV_SCRATCH = 2 };
+enum KvDst { KV_PAGES = 0, KV_SCRATCH = 1 };
 struct KvWrite {
   int mode;
-  bf16* k;               // pages: pool base of this layer; ring: ring base of this layer; scratch base
+  bf16* k;               // pages: pool base of this layer; scratch: sliding scratch base
   bf16* v;
   const int32_t* page_table;
   int max_pages;         // page-table width
@@ -81,6 +81,8 @@ cudaError_t scratch_to_ring(const bf16* sk, const bf16* sv, int scratch_rows, in
                             bf16* ring_v, int slot, int max_streams, cudaStream_t s);
 cudaError_t finish_step(int32_t* seq_len, const int32_t* row_slot, int rows, int add_prefill, int prefill_slot,
                         const unsigned long long* amax, int32_t* argmax_out, cudaStream_t s);
+// One bounded wait that can never complete (at most `rounds` polls), then the status word is set.
+cudaError_t wait_selftest(int* err, unsigned rounds, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode projection epilogues
 enum GemvEpi { GEMV_PARTIAL = 0, GEMV_SWIGLU = 1, GEMV_CONV = 2, GEMV_HEAD = 3 };
@@ -116,69 +118,14 @@ int ws_br(int epi);
 cudaError_t wstream(int epi, int nvfp4, const WsMaps& mp, const WsArgs& a, cudaStream_t s);
 cudaError_t wstream_init();
 
-// ---------------------------------------------------------------- persistent decode step
-constexpr int MK_MAX_NB = 4;   // streams one persistent step serves
-constexpr int MK_MAPS = 8;     // weight tensor maps per layer (the head's map follows the last layer)
-constexpr int MK_TRACE_PHASES = 256;  // phase stamps kept per block when profiling
-constexpr int MK_TRACE_BLOCKS = 160;
-constexpr int MK_TRACE_WORDS = 8;     // per phase: start, finish, data wait, last copy, prologue done, first copy
-struct MkLayer {
-  int type, kidx;                  // LFM3 layer type; index among the layers of that type
-  const bf16 *op_norm, *post_op_norm, *ffn_norm, *post_ffn_norm;
-  const bf16 *conv_w, *q_norm, *k_norm;
-  float w13_scale, w2_scale;       // NVFP4 tensor scales
-};
-// Fixed at bind: model, weight maps (device arrays) and workspace buffers.
-struct MkModel {
-  int n_layers, has_head, fp4, vocab, max_pages, max_streams, n_pages, nslot;
-  int pf;                          // stages prefetched into L2 ahead of the shared-memory loads
-  float eps;
-  const MkLayer* layers;
-  const CUtensorMap* maps;         // [n_layers * MK_MAPS + 1]
-  const bf16* embed;
-  const bf16* final_norm;
-  const float* rope_cos[2];
-  const float* rope_sin[2];
-  float *x_res, *x_res2, *part, *part2, *part3;
-  bf16 *y, *u;
-  unsigned long long* amax;
-  unsigned* sync;                  // [0] grid barrier, [1] exit count, [16..] attention merge counts
-  int* err;
-  unsigned long long* trace;       // null, or [block][MK_TRACE_PHASES][MK_TRACE_WORDS] stamps (ns)
-};
-// Per step.
-struct MkStep {
-  int nb;
-  const int32_t* slots;
-  const int32_t* tokens;
-  const bf16* embeds;
-  float* logits;
-  int32_t* argmax_out;
-  float* hidden;
-  int32_t* seq_len;
-  const int32_t* page_table;
-  bf16 *conv_state, *kv_k, *kv_v, *ring_k, *ring_v;
-  float* attn_part;
-  int attn_splits;                 // split stride of attn_part
-};
-cudaError_t mk_init();
-int mk_grid();  // blocks of one persistent launch (the SM count)
-// kv_maps: full-layer K, V pools and sliding-layer K, V rings, each viewed as [rows][128] bf16.
-cudaError_t decode_mk(const CUtensorMap* kv_maps, const MkModel& m, const MkStep& s, cudaStream_t st);
-
 // ---------------------------------------------------------------- attention
-constexpr int DEC_KEYS_FULL = 128;  // keys per decode split on full layers
-constexpr int DEC_KEYS_RING = 64;   // ring slots per decode split on sliding layers
+constexpr int DEC_KEYS = 64;  // keys per decode split: one 64-position page, or a quarter of the ring
 struct AttnLayer {
   int full;               // 1 full (pages), 0 sliding
   const bf16* k; const bf16* v;   // pages: this layer's pool; ring: this layer's ring base
   const int32_t* page_table;
   int max_pages, max_streams;
 };
-cudaError_t attn_decode(const bf16* q, Rows rows, AttnLayer L, int splits, float* part, const float* gate,
-                        bf16* y, cudaStream_t s);
-// Prefill attention for the n rows of one slot starting at position p0.
-//  full: keys through the page table; sliding: keys in scratch [HKV][scratch_rows][HD], index i <-> p0-WIN+i
 // Decode attention in one launch from the raw q|k|v|gate rows (see k_attn_decode_fused).
 struct AttnDecodeArgs {
   const bf16* q_norm;
@@ -189,13 +136,14 @@ struct AttnDecodeArgs {
   unsigned* counters;      // [streams][HKV], zero between calls
   int* err;                // status word (a bounded wait that gave up)
 };
+// Split slots a decode step reserves per (stream, head) in the partials buffer: the smallest
+// power of two >= the splits of the longest context (and >= the ring's WIN / DEC_KEYS).
+int attn_decode_splits(int max_pos);
 cudaError_t attn_decode_fused(const float* qkvg, Rows rows, AttnLayer L, const AttnDecodeArgs& A, int splits,
                               float* part, bf16* y, cudaStream_t s);
 cudaError_t attn_init();
 // Device address and size (floats) of the library's fixed attention scratch on the current device.
 cudaError_t attn_static_scratch(float** ptr, size_t* nfloats);
-cudaError_t attn_prefill(const bf16* q, int n, int p0, int slot, AttnLayer L, const bf16* sk, const bf16* sv,
-                         int scratch_rows, const float* gate, bf16* y, cudaStream_t s);
 
 // Prefill attention on tcgen05: maps over q [rows][16][128] and K/V stores viewed as [rows][128].
 struct AttnTcArgs {

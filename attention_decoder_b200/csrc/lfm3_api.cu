@@ -65,18 +65,7 @@ struct lfm3_ctx {
   GemmPlan deq_w13, deq_w2;  // NVFP4: maps over the dequantised weights (b, b3)
   CUtensorMap tm_q, tm_sk, tm_sv;  // prefill attention: q rows, sliding scratch K / V
   WsMaps ws_head;                  // decode: tied head
-  bool attn_tc = true;             // prefill attention on tcgen05 (LFM3_ATTN_MMA=1: warp MMA)
-  // persistent decode step (up to MK_MAX_NB streams; opt-in with LFM3_PERSISTENT=1)
-  MkLayer* mk_layers = nullptr;    // workspace: per-layer table
-  CUtensorMap* mk_maps = nullptr;  // workspace: weight maps
-  unsigned* mk_sync = nullptr;     // workspace: barrier and merge counters
   unsigned* attn_cnt = nullptr;    // workspace: decode attention split counts [max_batch][n_kv]
-  unsigned long long* mk_trace = nullptr;  // workspace: phase stamps while profiling
-  int mk_last_phases = 0;          // phases of the last persistent step, if it was stamped
-  int mk_last_head = 0;
-  MkModel mk{};
-  bool mk_on = false;
-  double mk_wbytes = 0;            // weight bytes one step streams
   std::string msg;
   int launches = 0;
   // decode-step CUDA graphs, keyed by batch, split count and every device pointer the step reads
@@ -138,7 +127,7 @@ size_t layout(lfm3_ctx* c, char* base) {
   // fp32 projection outputs: the conv in_proj [R][3D], qkvg [R][3088], or decode K-split partials
   c->part = reinterpret_cast<float*>(take(4 * std::max(R * 3 * D, (size_t)SPLIT_MAX * g.max_batch * NQKVG)));
   c->part2 = reinterpret_cast<float*>(take(4 * (size_t)SPLIT_MAX * g.max_batch * D));
-  c->part3 = reinterpret_cast<float*>(take(4 * (size_t)2 * g.max_batch * NQKVG));  // two K halves (persistent step)
+  c->part3 = reinterpret_cast<float*>(take(4 * (size_t)g.max_batch * NQKVG));  // decode q|k|v|gate projection
   c->q = reinterpret_cast<bf16*>(take(2 * R * HQ * HD));
   c->gate = reinterpret_cast<float*>(take(4 * R * HQ));
   c->sk = reinterpret_cast<bf16*>(take(2 * (size_t)HKV * c->scratch_rows * HD));
@@ -149,11 +138,7 @@ size_t layout(lfm3_ctx* c, char* base) {
     c->rope_sin[k] = reinterpret_cast<float*>(take(4 * (size_t)c->max_pos * (HD / 2)));
   }
   c->deq = g.ffn_format == LFM3_FFN_NVFP4 ? reinterpret_cast<bf16*>(take(2 * (size_t)2 * F * D)) : nullptr;
-  c->mk_layers = reinterpret_cast<MkLayer*>(take(sizeof(MkLayer) * (size_t)g.n_layers));
-  c->mk_maps = reinterpret_cast<CUtensorMap*>(take(sizeof(CUtensorMap) * ((size_t)g.n_layers * MK_MAPS + 1)));
-  c->mk_sync = reinterpret_cast<unsigned*>(take(256));
   c->attn_cnt = reinterpret_cast<unsigned*>(take(4 * (size_t)g.max_batch * HKV));
-  c->mk_trace = reinterpret_cast<unsigned long long*>(take(8 * (size_t)MK_TRACE_WORDS * MK_TRACE_BLOCKS * MK_TRACE_PHASES));
   return align_up(off, 256);
 }
 
@@ -370,153 +355,6 @@ lfm3_status ffn_gemm(lfm3_ctx* ctx, int l, int n, cudaStream_t s) {
   return LFM3_OK;
 }
 
-// Persistent decode step: per-layer table and weight maps in the workspace, counters zeroed.
-lfm3_status bind_persistent(lfm3_ctx* ctx) {
-  const lfm3_config& g = ctx->cfg;
-  const bool fp4 = g.ffn_format == LFM3_FFN_NVFP4;
-  std::vector<MkLayer> layers(g.n_layers);
-  std::vector<CUtensorMap> maps((size_t)g.n_layers * MK_MAPS + 1);
-  std::memset(maps.data(), 0, maps.size() * sizeof(CUtensorMap));
-  double wbytes = 0;
-  for (int l = 0; l < g.n_layers; ++l) {
-    const lfm3_layer_weights& W = ctx->L[l];
-    MkLayer& M = layers[l];
-    M = MkLayer{};
-    M.type = g.layer_type[l];
-    M.kidx = ctx->kidx[l];
-    M.op_norm = B(W.op_norm);
-    M.post_op_norm = B(W.post_op_norm);
-    M.ffn_norm = B(W.ffn_norm);
-    M.post_ffn_norm = B(W.post_ffn_norm);
-    M.conv_w = B(W.conv);
-    M.q_norm = B(W.q_norm);
-    M.k_norm = B(W.k_norm);
-    M.w13_scale = W.w13_scale;
-    M.w2_scale = W.w2_scale;
-    CUtensorMap* lm = maps.data() + (size_t)l * MK_MAPS;
-    bool ok = true;
-    if (M.type == LFM3_LAYER_CONV) {
-      ok &= make_ws_map(lm + 0, W.in_proj, 3 * D, D, 0, 16, 256);
-      ok &= make_ws_map(lm + 1, W.out_proj, D, D, 0, 16, 1024);
-      wbytes += 2.0 * 4 * D * D;
-    } else {
-      ok &= make_ws_map(lm + 0, W.qkvg, NQKVG, D, 0, 16, 1024);
-      ok &= make_ws_map(lm + 1, W.o_proj, D, HQ * HD, 0, 16, 1024);
-      wbytes += 2.0 * (NQKVG + D) * D;
-    }
-    if (fp4) {
-      ok &= make_ws_map(lm + 2, W.w1_codes, F, D, 1, 8, 2048);
-      ok &= make_ws_map(lm + 3, W.w3_codes, F, D, 1, 8, 2048);
-      ok &= make_ws_map(lm + 4, W.w2_codes, D, F, 1, 16, 2560);
-      ok &= make_ws_scale_map(lm + 5, W.w1_scales, F, D, 8, 2048);
-      ok &= make_ws_scale_map(lm + 6, W.w3_scales, F, D, 8, 2048);
-      ok &= make_ws_scale_map(lm + 7, W.w2_scales, D, F, 16, 2560);
-      wbytes += 3.0 * ((double)F * D / 2 + (double)F * D / 16);
-    } else {
-      ok &= make_ws_map(lm + 2, W.w1, F, D, 0, 8, 1024);
-      ok &= make_ws_map(lm + 3, W.w3, F, D, 0, 8, 1024);
-      ok &= make_ws_map(lm + 4, W.w2, D, F, 0, 16, 960);
-      wbytes += 2.0 * 3 * F * D;
-    }
-    if (!ok) return fail(ctx, LFM3_E_CUDA, "layer %d: persistent-step tensor map encoding failed", l);
-  }
-  if (g.has_head) {
-    if (!make_ws_map(maps.data() + (size_t)g.n_layers * MK_MAPS, ctx->embed, g.vocab, D, 0, 16, 1024))
-      return fail(ctx, LFM3_E_CUDA, "persistent-step head tensor map encoding failed");
-  }
-  CK(cudaMemcpy(ctx->mk_layers, layers.data(), layers.size() * sizeof(MkLayer), cudaMemcpyHostToDevice));
-  CK(cudaMemcpy(ctx->mk_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
-  CK(cudaMemset(ctx->mk_sync, 0, 256));
-  CK(cudaMemset(ctx->attn_cnt, 0, 4 * (size_t)g.max_batch * HKV));
-  MkModel& m = ctx->mk;
-  m = MkModel{};
-  m.n_layers = g.n_layers;
-  m.has_head = g.has_head;
-  m.fp4 = fp4;
-  m.vocab = g.vocab;
-  m.max_pages = g.max_pages_per_stream;
-  m.max_streams = g.max_streams;
-  m.n_pages = g.n_pages;
-  m.eps = g.eps;
-  m.pf = 12;
-  if (const char* v = getenv("LFM3_MK_PREFETCH")) m.pf = std::max(0, std::min(64, atoi(v)));
-  m.layers = ctx->mk_layers;
-  m.maps = ctx->mk_maps;
-  m.embed = ctx->embed;
-  m.final_norm = ctx->final_norm;
-  for (int k = 0; k < 2; ++k) {
-    m.rope_cos[k] = ctx->rope_cos[k];
-    m.rope_sin[k] = ctx->rope_sin[k];
-  }
-  m.x_res = ctx->x_res;
-  m.x_res2 = ctx->x_res2;
-  m.part = ctx->part;
-  m.part2 = ctx->part2;
-  m.part3 = ctx->part3;
-  m.y = ctx->y;
-  m.u = ctx->big;
-  m.amax = ctx->amax;
-  m.sync = ctx->mk_sync;
-  m.err = ctx->err;
-  ctx->mk_wbytes = wbytes;
-  return LFM3_OK;
-}
-
-bool use_persistent(const lfm3_ctx* ctx, int nb) { return ctx->mk_on && nb <= MK_MAX_NB; }
-
-// One decode step as a single persistent launch (see k_decode_mk.cu).
-lfm3_status enqueue_decode_mk(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* h_slots,
-                              const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds, float* d_logits,
-                              int32_t* d_argmax, float* d_hidden, int splits_full, float* attn_part, cudaStream_t s) {
-  const lfm3_config& g = ctx->cfg;
-  CUtensorMap kv[4];
-  const void* dummy = ctx->rope_cos[0];  // any mapped buffer of >= 64 rows of 256 bytes; never read
-  const uint64_t full_rows = (uint64_t)ctx->n_full * g.n_pages * HKV * PAGE;
-  const uint64_t ring_rows = (uint64_t)ctx->n_sliding * g.max_streams * HKV * WIN;
-  bool ok = true;
-  ok &= make_tmap_kv(&kv[0], ctx->n_full ? st->kv_k : dummy, ctx->n_full ? full_rows : 64);
-  ok &= make_tmap_kv(&kv[1], ctx->n_full ? st->kv_v : dummy, ctx->n_full ? full_rows : 64);
-  ok &= make_tmap_kv(&kv[2], ctx->n_sliding ? st->ring_k : dummy, ctx->n_sliding ? ring_rows : 64);
-  ok &= make_tmap_kv(&kv[3], ctx->n_sliding ? st->ring_v : dummy, ctx->n_sliding ? ring_rows : 64);
-  if (!ok) return fail(ctx, LFM3_E_CUDA, "key/value tensor map encoding failed");
-  MkStep S{};
-  S.nb = nb;
-  S.slots = d_slots;
-  S.tokens = g.has_head ? d_tokens : nullptr;
-  S.embeds = B(d_embeds);
-  S.logits = d_logits;
-  S.argmax_out = d_argmax;
-  S.hidden = d_hidden;
-  S.seq_len = st->seq_len;
-  S.page_table = st->page_table;
-  S.conv_state = reinterpret_cast<bf16*>(st->conv_state);
-  S.kv_k = reinterpret_cast<bf16*>(st->kv_k);
-  S.kv_v = reinterpret_cast<bf16*>(st->kv_v);
-  S.ring_k = reinterpret_cast<bf16*>(st->ring_k);
-  S.ring_v = reinterpret_cast<bf16*>(st->ring_v);
-  S.attn_part = attn_part;
-  S.attn_splits = std::max(splits_full, WIN / DEC_KEYS_RING);
-  // algorithmic bytes of the step: every weight once, plus the cached keys and values read
-  double kvb = 0;
-  for (int b = 0; b < nb; ++b) {
-    const double pos = (double)st->h_seq_len[h_slots[b]];
-    kvb += 2.0 * 2 * HKV * HD * (ctx->n_full * (pos + 1) + ctx->n_sliding * std::min(pos + 1, (double)WIN));
-  }
-  const double head = (g.has_head && (d_logits || d_argmax)) ? 2.0 * g.vocab * D : 0.0;
-  MkModel mm = ctx->mk;
-  mm.trace = ctx->prof ? ctx->mk_trace : nullptr;
-  ctx->mk_last_phases = 0;
-  if (ctx->prof) {
-    for (int l = 0; l < g.n_layers; ++l) ctx->mk_last_phases += g.layer_type[l] == LFM3_LAYER_CONV ? 4 : 5;
-    ctx->mk_last_head = head > 0;
-    ctx->mk_last_phases += ctx->mk_last_head;
-  }
-  if (mm.trace) CK(cudaMemsetAsync(ctx->mk_trace, 0, 8 * (size_t)MK_TRACE_WORDS * MK_TRACE_BLOCKS * MK_TRACE_PHASES, s));
-  Bracket br(ctx, s, ctx->mk_wbytes + head + kvb, 0.0);
-  CK(decode_mk(kv, mm, S, s));
-  return LFM3_OK;
-}
-
 }  // namespace
 
 // ======================================================================================== ABI
@@ -544,7 +382,7 @@ extern "C" lfm3_status lfm3_create(const lfm3_config* cfg, const lfm3_weights* w
   }
   c->max_pos = cfg->max_pages_per_stream * PAGE;
   c->R = std::max(cfg->max_chunk, cfg->max_batch);
-  c->max_splits = std::max((c->max_pos + DEC_KEYS_FULL - 1) / DEC_KEYS_FULL, WIN / DEC_KEYS_RING);
+  c->max_splits = attn_decode_splits(c->max_pos);
   c->scratch_rows = WIN + cfg->max_chunk;
   c->ws_bytes = layout(c, nullptr);
   *workspace_bytes = c->ws_bytes;
@@ -563,7 +401,6 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
   CK(gemm_init());
   CK(attn_init());
   CK(attn_tc_init());
-  CK(mk_init());
   layout(ctx, reinterpret_cast<char*>(d_ws));
   const lfm3_config& g = ctx->cfg;
   const int R = ctx->R;
@@ -585,6 +422,7 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
     }
   }
   CK(cudaMemset(ctx->err, 0, 256));
+  CK(cudaMemset(ctx->attn_cnt, 0, 4 * (size_t)g.max_batch * HKV));
   // GEMM plans (tensor maps over the weights and the workspace activations)
   ctx->plans.assign(g.n_layers, LayerPlan{});
   for (int l = 0; l < g.n_layers; ++l) {
@@ -652,14 +490,8 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
     ok &= plan_gemm(&ctx->deq_w2, GEMM_F32, ctx->big, R, ctx->deq, nullptr, D, F, ctx->part, D, 1.f);
     if (!ok) return fail(ctx, LFM3_E_CUDA, "NVFP4 tensor map encoding failed");
   }
-  {
-    lfm3_status ms = bind_persistent(ctx);
-    if (ms != LFM3_OK) return ms;
-  }
   CK(cudaDeviceSynchronize());
   ctx->graphs_on = getenv("LFM3_NO_GRAPH") == nullptr;
-  ctx->mk_on = getenv("LFM3_PERSISTENT") != nullptr;
-  ctx->attn_tc = getenv("LFM3_ATTN_MMA") == nullptr;
   if (!make_tmap_q(&ctx->tm_q, ctx->q, (uint64_t)R) ||
       !make_tmap_kv(&ctx->tm_sk, ctx->sk, (uint64_t)HKV * ctx->scratch_rows) ||
       !make_tmap_kv(&ctx->tm_sv, ctx->sv, (uint64_t)HKV * ctx->scratch_rows))
@@ -724,30 +556,25 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
         const int k = full ? 0 : 1;
         CK(qk_norm_rope_kv(ctx->part, 1, 0, B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], rows, eps,
                            ctx->q, ctx->gate, kw, s));
-        if (ctx->attn_tc) {
-          CUtensorMap tk, tv;
-          if (full) {
-            const uint64_t rows = (uint64_t)g.n_pages * HKV * PAGE;
-            if (!make_tmap_kv(&tk, v.kv_k, rows) || !make_tmap_kv(&tv, v.kv_v, rows))
-              return fail(ctx, LFM3_E_CUDA, "layer %d: K/V pool tensor map encoding failed", l);
-          }
-          AttnTcArgs ta{};
-          ta.n = nc;
-          ta.p0 = p0;
-          ta.slot = slot;
-          ta.full = full;
-          ta.row0 = 0;
-          ta.page_table = st->page_table;
-          ta.max_pages = g.max_pages_per_stream;
-          ta.scratch_rows = ctx->scratch_rows;
-          ta.gate = ctx->gate;
-          ta.y = ctx->y;
-          ta.err = ctx->err;
-          CK(attn_prefill_tc(ctx->tm_q, full ? tk : ctx->tm_sk, full ? tv : ctx->tm_sv, ta, s));
-        } else {
-          CK(attn_prefill(ctx->q, nc, p0, slot, attn_layer(ctx, st, l, v), ctx->sk, ctx->sv, ctx->scratch_rows,
-                          ctx->gate, ctx->y, s));
+        CUtensorMap tk, tv;
+        if (full) {
+          const uint64_t rows = (uint64_t)g.n_pages * HKV * PAGE;
+          if (!make_tmap_kv(&tk, v.kv_k, rows) || !make_tmap_kv(&tv, v.kv_v, rows))
+            return fail(ctx, LFM3_E_CUDA, "layer %d: K/V pool tensor map encoding failed", l);
         }
+        AttnTcArgs ta{};
+        ta.n = nc;
+        ta.p0 = p0;
+        ta.slot = slot;
+        ta.full = full;
+        ta.row0 = 0;
+        ta.page_table = st->page_table;
+        ta.max_pages = g.max_pages_per_stream;
+        ta.scratch_rows = ctx->scratch_rows;
+        ta.gate = ctx->gate;
+        ta.y = ctx->y;
+        ta.err = ctx->err;
+        CK(attn_prefill_tc(ctx->tm_q, full ? tk : ctx->tm_sk, full ? tv : ctx->tm_sv, ta, s));
         if (!full)
           CK(scratch_to_ring(ctx->sk, ctx->sv, ctx->scratch_rows, nc, p0, v.ring_k, v.ring_v, slot, g.max_streams, s));
         CK(run_gemm(ctx, P.o_proj, nc, s));
@@ -798,46 +625,24 @@ lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, co
     const lfm3_layer_weights& W = ctx->L[l];
     const LayerPlan& P = ctx->plans[l];
     const Views v = views(ctx, st, l);
-    int np = 1;
-    long pstride = 0;
     if (g.layer_type[l] == LFM3_LAYER_CONV) {
-      {
-        CK(run_gemm(ctx, P.in_proj, nb, s));
-        CK(conv_decode(ctx->part, B(W.conv), v.conv_layer, ctx->row_slot, nb, ctx->y, s));
-        CK(run_gemm(ctx, P.out_proj, nb, s));
-      }
+      CK(run_gemm(ctx, P.in_proj, nb, s));
+      CK(conv_decode(ctx->part, B(W.conv), v.conv_layer, ctx->row_slot, nb, ctx->y, s));
+      CK(run_gemm(ctx, P.out_proj, nb, s));
     } else {
       const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
-      int nq = 1;
-      long qstride = 0;
-      {
-        CK(run_gemm(ctx, P.qkvg, nb, s));
-      }
-      KvWrite kw{};
-      kw.mode = full ? KV_PAGES : KV_RING;
-      kw.k = full ? v.kv_k : v.ring_k;
-      kw.v = full ? v.kv_v : v.ring_v;
-      kw.page_table = st->page_table;
-      kw.max_pages = g.max_pages_per_stream;
-      kw.max_streams = g.max_streams;
+      CK(run_gemm(ctx, P.qkvg, nb, s));
       const int k = full ? 0 : 1;
-      CK(qk_norm_rope_kv(ctx->part, nq, qstride, B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], rows,
-                         eps, ctx->q, ctx->gate, kw, s));
-      CK(attn_decode(ctx->q, rows, attn_layer(ctx, st, l, v), full ? splits_full : WIN / DEC_KEYS_RING, attn_part, ctx->gate,
-                     ctx->y, s));
-      {
-        CK(run_gemm(ctx, P.o_proj, nb, s));
-      }
+      AttnDecodeArgs A{B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], eps, ctx->attn_cnt, ctx->err};
+      CK(attn_decode_fused(ctx->part, rows, attn_layer(ctx, st, l, v), A, full ? splits_full : WIN / DEC_KEYS,
+                           attn_part, ctx->y, s));
+      CK(run_gemm(ctx, P.o_proj, nb, s));
     }
-    CK(resid_norm(ctx->x_res, ctx->part, np, pstride, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nb, eps, nullptr, s));
-    np = 1;
-    pstride = 0;
-    {
-      lfm3_status fs = ffn_gemm(ctx, l, nb, s);
-      if (fs != LFM3_OK) return fs;
-    }
+    CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nb, eps, nullptr, s));
+    lfm3_status fs = ffn_gemm(ctx, l, nb, s);
+    if (fs != LFM3_OK) return fs;
     const bf16* gnext = l + 1 < g.n_layers ? B(ctx->L[l + 1].op_norm) : (g.has_head ? ctx->final_norm : nullptr);
-    CK(resid_norm(ctx->x_res, ctx->part, np, pstride, B(W.post_ffn_norm), gnext, ctx->xn, nb, eps,
+    CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_ffn_norm), gnext, ctx->xn, nb, eps,
                   d_hidden ? d_hidden + (size_t)(l + 1) * nb * D : nullptr, s));
   }
   const bool head = g.has_head && (d_logits || d_argmax);
@@ -931,7 +736,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       advance();
       const int k = full ? 0 : 1;
       AttnDecodeArgs A{B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], eps, ctx->attn_cnt, ctx->err};
-      CK(attn_decode_fused(ctx->part3, rows, attn_layer(ctx, st, l, v), A, full ? splits_full : WIN / DEC_KEYS_RING,
+      CK(attn_decode_fused(ctx->part3, rows, attn_layer(ctx, st, l, v), A, full ? splits_full : WIN / DEC_KEYS,
                            attn_part, ctx->y, s));
       WsArgs o{};
       base(o, HQ * HD, D, SPLIT_DD);
@@ -1028,9 +833,7 @@ lfm3_status validate_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const i
     if (vs != LFM3_OK) return vs;
     maxpos = std::max(maxpos, (int)st->h_seq_len[s]);
   }
-  int splits_full = 1;
-  while (splits_full < maxpos / DEC_KEYS_FULL + 1) splits_full *= 2;
-  *splits_out = std::min(splits_full, ctx->max_splits);
+  *splits_out = std::min(attn_decode_splits(maxpos + 1), ctx->max_splits);
   return LFM3_OK;
 }
 
@@ -1046,12 +849,7 @@ extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int
   if (vs != LFM3_OK) return vs;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   g_launches = 0;
-  if (use_persistent(ctx, nb)) {
-    lfm3_status es = enqueue_decode_mk(ctx, st, nb, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax,
-                                       d_hidden, splits_full, ctx->attn_part, s);
-    if (es != LFM3_OK) return es;
-    ctx->launches = g_launches;
-  } else if (!ctx->graphs_on || ctx->prof) {
+  if (!ctx->graphs_on || ctx->prof) {
     lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
                                     splits_full, ctx->attn_part, s);
     if (es != LFM3_OK) return es;
@@ -1109,7 +907,7 @@ extern "C" lfm3_status lfm3_decode_step_noalloc(lfm3_ctx* ctx, const lfm3_state*
   float* scratch = nullptr;
   size_t cap = 0;
   CK(attn_static_scratch(&scratch, &cap));
-  const size_t need = (size_t)nb * HQ * std::max(splits_full, WIN / DEC_KEYS_RING) * (HD + 2);
+  const size_t need = (size_t)nb * HQ * splits_full * (HD + 2);
   if (need > cap)
     return fail(ctx, LFM3_E_CAPACITY,
                 "lfm3_decode_step_noalloc: %d streams x %d key splits need %zu bytes of attention scratch, more "
@@ -1117,12 +915,8 @@ extern "C" lfm3_status lfm3_decode_step_noalloc(lfm3_ctx* ctx, const lfm3_state*
                 nb, splits_full, need * sizeof(float), cap * sizeof(float));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   g_launches = 0;
-  lfm3_status es =
-      use_persistent(ctx, nb)
-          ? enqueue_decode_mk(ctx, st, nb, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
-                              splits_full, scratch, s)
-          : enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden, splits_full,
-                           scratch, s);
+  lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                                  splits_full, scratch, s);
   if (es != LFM3_OK) return es;
   ctx->launches = g_launches;
   for (int b = 0; b < nb; ++b) st->h_seq_len[h_slots[b]] += 1;
@@ -1137,9 +931,18 @@ extern "C" lfm3_status lfm3_check_device_errors(lfm3_ctx* ctx, void* stream) {
   CK(cudaMemcpy(&e, ctx->err, sizeof e, cudaMemcpyDeviceToHost));
   if (e) {
     CK(cudaMemset(ctx->err, 0, sizeof e));
-    CK(cudaMemset(ctx->mk_sync, 0, 256));  // a persistent step that gave up left its counters mid-way
+    // a step that gave up can leave the attention's split counts mid-way
+    CK(cudaMemset(ctx->attn_cnt, 0, 4 * (size_t)ctx->cfg.max_batch * HKV));
     return fail(ctx, LFM3_E_TIMEOUT, "a device-side bounded wait gave up (status %d)", e);
   }
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_selftest_wait(lfm3_ctx* ctx, unsigned rounds, void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
+  if (rounds < 1 || rounds > (1u << 16)) return fail(ctx, LFM3_E_ARG, "rounds %u outside 1..65536", rounds);
+  CK(wait_selftest(ctx->err, rounds, reinterpret_cast<cudaStream_t>(stream)));
   return LFM3_OK;
 }
 
@@ -1176,77 +979,6 @@ extern "C" lfm3_status lfm3_profile_read(lfm3_ctx* ctx, int* launches, double* m
   const int over = ctx->ev_overflow;
   ctx->ev_used = ctx->ev_overflow = 0;
   if (over) return fail(ctx, LFM3_E_CAPACITY, "%d launches ran unbracketed (capacity exceeded)", over);
-  return LFM3_OK;
-}
-
-extern "C" lfm3_status lfm3_profile_phases(lfm3_ctx* ctx, void* stream, int cap, int* n_phases, int* kind,
-                                           double* span_us, double* work_us, double* work_max_us, double* wait_us,
-                                           double* lead_us, double* prologue_us, double* ahead_us) {
-  if (!ctx || !n_phases) return LFM3_E_ARG;
-  *n_phases = 0;
-  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
-  if (!ctx->prof || ctx->mk_last_phases == 0)
-    return fail(ctx, LFM3_E_STATE, "no stamped persistent decode step (profiling off, or another path ran)");
-  const int G = mk_grid();
-  if (G > MK_TRACE_BLOCKS) return fail(ctx, LFM3_E_UNSUPPORTED, "%d blocks exceed the stamp table", G);
-  CK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
-  std::vector<unsigned long long> t((size_t)G * MK_TRACE_PHASES * MK_TRACE_WORDS);
-  CK(cudaMemcpy(t.data(), ctx->mk_trace, t.size() * 8, cudaMemcpyDeviceToHost));
-  const lfm3_config& g = ctx->cfg;
-  std::vector<int> kinds;
-  for (int l = 0; l < g.n_layers; ++l) {
-    if (g.layer_type[l] == LFM3_LAYER_CONV) kinds.insert(kinds.end(), {0, 3, 4, 5});
-    else kinds.insert(kinds.end(), {1, 2, 3, 4, 5});
-  }
-  if (ctx->mk_last_head) kinds.push_back(6);
-  const int n = std::min({(int)kinds.size(), cap, MK_TRACE_PHASES});
-  for (int p = 0; p < n; ++p) {
-    unsigned long long lo = ~0ull, hi = 0;
-    double sum = 0, mx = 0, wsum = 0, lsum = 0, psum = 0, asum = 0;
-    int ln = 0, an = 0;
-    for (int b = 0; b < G; ++b) {
-      const unsigned long long* r = t.data() + ((size_t)b * MK_TRACE_PHASES + p) * MK_TRACE_WORDS;
-      const unsigned long long a = r[0], e = r[1];
-      lo = std::min(lo, a);
-      hi = std::max(hi, e);
-      const double w = e > a ? (e - a) * 1e-3 : 0.0;
-      sum += w;
-      mx = std::max(mx, w);
-      wsum += r[2] * 1e-3;
-      if (r[3] && e > r[3]) {
-        lsum += (e - r[3]) * 1e-3;
-        ++ln;
-      }
-      if (r[4] > a) psum += (r[4] - a) * 1e-3;
-      if (r[5]) {
-        asum += ((double)a - (double)r[5]) * 1e-3;
-        ++an;
-      }
-    }
-    if (prologue_us) prologue_us[p] = psum / G;
-    if (ahead_us) ahead_us[p] = an ? asum / an : 0.0;
-    if (wait_us) wait_us[p] = wsum / G;
-    if (lead_us) lead_us[p] = ln ? lsum / ln : 0.0;
-    if (kind) kind[p] = kinds[p];
-    if (span_us) span_us[p] = hi > lo ? (hi - lo) * 1e-3 : 0.0;
-    if (work_us) work_us[p] = sum / G;
-    if (work_max_us) work_max_us[p] = mx;
-  }
-  *n_phases = n;
-  return LFM3_OK;
-}
-
-extern "C" lfm3_status lfm3_profile_stamps(lfm3_ctx* ctx, void* stream, uint64_t* out, size_t cap, int* n_blocks) {
-  if (!ctx || !out || !n_blocks) return LFM3_E_ARG;
-  *n_blocks = 0;
-  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
-  if (!ctx->prof || ctx->mk_last_phases == 0)
-    return fail(ctx, LFM3_E_STATE, "no stamped persistent decode step (profiling off, or another path ran)");
-  const int G = std::min(mk_grid(), MK_TRACE_BLOCKS);
-  CK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
-  const size_t n = std::min(cap, (size_t)G * MK_TRACE_PHASES * MK_TRACE_WORDS);
-  CK(cudaMemcpy(out, ctx->mk_trace, n * 8, cudaMemcpyDeviceToHost));
-  *n_blocks = G;
   return LFM3_OK;
 }
 

@@ -121,35 +121,14 @@ class Lfm3Model:
         check(L.lfm3_profile_read(self.ctx, C.byref(n), C.byref(ms), C.byref(b), C.byref(f)), self.ctx)
         return {"launches": n.value, "ms": ms.value, "bytes": b.value, "flops": f.value}
 
-    PHASE_KINDS = ("conv", "qkvg", "attn", "out", "w13", "w2", "head")
-
-    def profile_phases(self, stream=None) -> list:
-        """Per-phase timing of the last persistent decode step (profiling on): one dict per phase
-        with its kind, span (first start to last finish over blocks) and mean / max block work, us."""
-        cap = 256
-        n = C.c_int()
-        kind = (C.c_int * cap)()
-        span, work, wmax, wait, lead, pro, ahead = ((C.c_double * cap)() for _ in range(7))
-        check(L.lfm3_profile_phases(self.ctx, _stream(stream), cap, C.byref(n), kind, span, work, wmax, wait, lead,
-                                    pro, ahead), self.ctx)
-        return [{"kind": self.PHASE_KINDS[kind[i]], "span_us": span[i], "work_us": work[i], "work_max_us": wmax[i],
-                 "wait_us": wait[i], "lead_us": lead[i], "prologue_us": pro[i], "ahead_us": ahead[i]}
-                for i in range(n.value)]
-
-    def profile_stamps(self, stream=None) -> np.ndarray:
-        """Raw phase stamps of the last persistent decode step: uint64 [blocks][256][8] (ns)."""
-        cap = 160 * 256 * 8
-        buf = np.zeros(cap, dtype=np.uint64)
-        nb = C.c_int()
-        check(L.lfm3_profile_stamps(self.ctx, _stream(stream), buf.ctypes.data_as(C.POINTER(C.c_uint64)), cap,
-                                    C.byref(nb)), self.ctx)
-        return buf[: nb.value * 256 * 8].reshape(nb.value, 256, 8)
-
     def last_launch_count(self) -> int:
         return L.lfm3_last_launch_count(self.ctx)
 
     def check_device_errors(self, stream=None):
         check(L.lfm3_check_device_errors(self.ctx, _stream(stream)), self.ctx)
+
+    def selftest_wait(self, rounds=4096, stream=None):
+        check(L.lfm3_selftest_wait(self.ctx, rounds, _stream(stream)), self.ctx)
 
     # ------------------------------------------------------------------ calls
     def prefill(self, st, slot, tokens=None, embeds=None, logits=True, argmax=True, hidden=False, stream=None,

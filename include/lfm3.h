@@ -14,14 +14,20 @@
  *
  * Conventions for every entry point
  *   - Ownership: the CALLER owns all device memory (weights, state, workspace, outputs) and
- *     every host array passed in. The library owns only its host-side context.
+ *     every host array passed in. The library owns only its host-side context. The per-slot
+ *     state the pages' engine keeps for itself (TensorFold PR #1508, "What": a 6-row conv state
+ *     per slot, a per-slot ring for the sliding layers, pages of a pool for the full layers;
+ *     pool-leasing commit: the tables and conv states of the slots) is here a caller-allocated
+ *     lfm3_state whose layout this header fixes and which only this library writes.
  *   - All pointers named d_* or documented "device" are device pointers; h_* are host.
  *   - bf16 tensors are IEEE bfloat16 bit patterns, row-major, densely packed.
  *   - Calls enqueue work on the given CUDA stream (a cudaStream_t passed as void*; NULL =
  *     legacy default stream) and return without synchronising.
  *   - Errors: arguments, configuration and capacity are checked on the host BEFORE anything
  *     is enqueued; on any error nothing is launched and no state is modified. CUDA launch
- *     errors map to LFM3_E_CUDA. lfm3_last_error() gives a message naming the refusal.
+ *     errors map to LFM3_E_CUDA. lfm3_last_error() gives a message naming the refusal
+ *     (TensorFold PR #1508, NVFP4 admission commit: an unsupported layout is refused by name,
+ *     e.g. "Lfm3UnsupportedGeometry: d_model = 4096").
  *   - The library never allocates device memory and never reads /writes device memory from
  *     the host, except lfm3_bind_workspace (which uploads constant tables into the workspace)
  *     and lfm3_check_device_errors (which reads one status word).
@@ -137,28 +143,50 @@ typedef struct {
 
 /* Validates cfg and w (no device access, no launches) and returns the number of workspace
  * bytes the context needs. On success *out owns a context (free with lfm3_free); on failure
- * *out is NULL and lfm3_last_error(NULL) names the refusal. */
+ * *out is NULL and lfm3_last_error(NULL) names the refusal: LFM3_E_UNSUPPORTED for a geometry or
+ * FFN format the kernels do not implement, named in the message as the pages' admission does
+ * (TensorFold PR #1508, NVFP4 admission commit: "refuse the other by name"), LFM3_E_CONFIG for an
+ * inconsistent configuration, LFM3_E_ARG for a NULL or misaligned weight pointer. The geometry is
+ * the pages' LFM3-1.7B one (coreai-model-zoo note "lfm3-1.7b-port", LFM2.5 -> LFM3 diff table and
+ * "Unchanged" paragraph). */
 lfm3_status lfm3_create(const lfm3_config* cfg, const lfm3_weights* w, size_t* workspace_bytes,
                         lfm3_ctx** out);
 
 /* Binds caller-owned device workspace (>= the size lfm3_create reported, 256-byte aligned) and
- * uploads the rotary tables into it (synchronous). Must precede prefill/decode. */
+ * uploads the rotary tables into it (synchronous). Must precede prefill/decode. The tables hold
+ * cos/sin of p * theta^(-2i/128) per position p and pair i, built in double precision and stored
+ * fp32 (coreai-model-zoo note "lfm3-1.7b-port", partial-rotary paragraph: theta 1e6 on pairs
+ * i < 32 of full layers, theta 1e4 on all 64 pairs of sliding layers). Errors: LFM3_E_ARG for a
+ * NULL, misaligned or short workspace; LFM3_E_CUDA if a copy or a tensor-map encoding fails. */
 lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_workspace, size_t bytes);
 
 /* Prompt pass for one slot: consumes n rows at positions h_seq_len[slot] .. +n-1, in chunks
  * of at most max_chunk rows, updating conv state, ring, pages and seq_len in place.
+ * Positions come from the state alone and there is no mask input: a key is visible to a query
+ * iff its position is not later and, on sliding layers, fewer than 256 positions earlier
+ * (coreai-model-zoo note "lfm3-1.7b-port", "window_size, with no mask input"). The conv state
+ * after a chunk of n rows is columns [n, n + 6) of [state | Bx] (same note, chunked-prefill
+ * paragraph).
  *   d_tokens    device int32 [n] (has_head == 1) or NULL
  *   d_embeds    device bf16 [n][d_model] input vectors (has_head == 0) or NULL
  *   d_logits    device fp32 [vocab]: logits of the LAST row (has_head == 1), or NULL
  *   d_argmax    device int32 [1]: greedy id of the last row, or NULL
  *   d_hidden    device fp32 [n_layers+1][n][d_model]: the residual stream entering layer 0 and
  *               leaving every layer (the per-layer parity tap), or NULL
- * Refuses with LFM3_E_CAPACITY if the slot's pages cannot hold seq_len + n positions. */
+ * Refuses with LFM3_E_CAPACITY, before anything is enqueued, if the slot's pages cannot hold
+ * seq_len + n positions or a page-table entry it would write is outside the pool (TensorFold
+ * PR #1508, pool-leasing commit: "forward refuses rows past a slot's pages"); LFM3_E_ARG for a bad
+ * slot, an empty call, or inputs that do not match has_head; LFM3_E_STATE before
+ * lfm3_bind_workspace. */
 lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slot, const int32_t* d_tokens,
                          const void* d_embeds, int n, float* d_logits, int32_t* d_argmax,
                          float* d_hidden, void* stream);
 
-/* One decode step for n_streams distinct slots (one row each, at position seq_len[slot]).
+/* One decode step for n_streams distinct slots (one row each, at position seq_len[slot]; as for
+ * lfm3_prefill the position comes from the state and there is no mask input - coreai-model-zoo
+ * note "lfm3-1.7b-port", "window_size, with no mask input"). Streams share no state; the pages'
+ * engine checks that concurrent == solo (TensorFold PR #1508, "Verification"), which holds here
+ * bit for bit at up to 16 streams.
  *   h_slots     HOST int32 [n_streams] slot ids (checked; must equal d_slots)
  *   d_slots     device int32 [n_streams]
  *   d_tokens    device int32 [n_streams] (has_head == 1) or NULL; may alias d_argmax of the
@@ -166,7 +194,11 @@ lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slot, const in
  *   d_embeds    device bf16 [n_streams][d_model] (has_head == 0) or NULL
  *   d_logits    device fp32 [n_streams][vocab] or NULL
  *   d_argmax    device int32 [n_streams] greedy ids, or NULL
- *   d_hidden    device fp32 [n_layers+1][n_streams][d_model] or NULL                        */
+ *   d_hidden    device fp32 [n_layers+1][n_streams][d_model] or NULL
+ * Errors (nothing enqueued, no state touched): LFM3_E_CAPACITY if a slot's pages cannot hold one
+ * more position (TensorFold PR #1508, pool-leasing commit: "forward refuses rows past a slot's
+ * pages"); LFM3_E_ARG for a slot out of range or listed twice, n_streams outside 1..max_batch,
+ * or inputs that do not match has_head; LFM3_E_STATE before lfm3_bind_workspace. */
 lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int n_streams, const int32_t* h_slots,
                              const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
                              float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream);
@@ -179,27 +211,40 @@ lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int n_streams,
  *   a bound workspace is still required). The difference: the attention's per-split partial
  *   results go to a fixed 4 MiB array inside the library's own device image instead of the
  *   workspace, and the step is launched kernel by kernel (no captured graph).
- *   Limit: n_streams x 16 heads x splits x 130 floats must fit in the 4 MiB, where splits is
- *   max(4, the smallest power of two >= (longest context / 128) + 1); larger calls are refused
- *   with LFM3_E_CAPACITY and a message giving both sizes. One stream fits any context below
- *   32768 positions; 64 streams fit contexts below 384.
+ *   Limit: n_streams x 16 heads x splits x 130 floats must fit in the 4 MiB, where splits is the
+ *   smallest power of two >= 4 with 64 x splits >= (longest context + 1); larger calls are
+ *   refused with LFM3_E_CAPACITY and a message giving both sizes. One stream fits any context
+ *   below 16384 positions; 64 streams fit contexts below 256.
  *   Nothing in the array has to start at zero: every call writes all the partials it reads.
  *   The array is one per GPU for the whole process and every call shares it, so calls that can
  *   overlap on the GPU (different streams, different contexts) race on it; serialise them.
- *   The first call on each device looks the array's address up (cudaGetSymbolAddress) with that
- *   device current; make that first call before any stream capture. No device memory is
- *   allocated or freed by this call. */
+ *   The first call in each CUDA context looks the array's address up (cudaGetSymbolAddress) with
+ *   that context current; make that first call before any stream capture. A context destroyed
+ *   and created again (cudaDeviceReset) is a new context: its first call looks the address up
+ *   again. No device memory is allocated or freed by this call. */
 lfm3_status lfm3_decode_step_noalloc(lfm3_ctx* ctx, const lfm3_state* st, int n_streams, const int32_t* h_slots,
                                      const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
                                      float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream);
 
 /* Synchronises the stream and reads the device status word that bounded device-side waits set
- * when they give up. Returns LFM3_OK or LFM3_E_TIMEOUT (and clears the word). */
+ * when they give up (every wait on a copy or a peer block in the kernels has an iteration limit
+ * and then records the failure and returns instead of spinning). Returns LFM3_OK or
+ * LFM3_E_TIMEOUT; on LFM3_E_TIMEOUT it clears the word and the attention's split counters, so
+ * the context stays usable, but the results of the calls since the last check are invalid. The
+ * pages have no counterpart: a service of this library. */
 lfm3_status lfm3_check_device_errors(lfm3_ctx* ctx, void* stream);
 
-/* Kernel timing for measurement. While enabled, every projection kernel that prefill/decode
- * enqueue (the weight-streaming GEMVs of decode and the tensor-core GEMMs of prefill) is
- * bracketed by two CUDA events recorded on the call's stream. Event handles are host objects
+/* Self-test of the failure path (no counterpart on the pages): enqueues one kernel whose single
+ * bounded wait can never complete - a fresh barrier that nothing arrives on - so that after at
+ * most `rounds` polls (1..65536) it gives up and sets the status word exactly as the kernels' own
+ * waits do. A following lfm3_check_device_errors returns LFM3_E_TIMEOUT and clears the word; the
+ * state and the context are untouched and stay usable. Nothing faults, traps or hangs. */
+lfm3_status lfm3_selftest_wait(lfm3_ctx* ctx, unsigned rounds, void* stream);
+
+/* Kernel timing for measurement (no counterpart on the pages). While enabled, every projection
+ * kernel that prefill/decode enqueue (the weight-streaming GEMVs of decode and the tensor-core
+ * GEMMs of prefill) is bracketed by two CUDA events recorded on the call's stream; decode steps
+ * then run launch by launch rather than from their captured graph. Event handles are host objects
  * created here (up to `capacity` brackets between reads); no device memory is allocated. */
 lfm3_status lfm3_profile_enable(lfm3_ctx* ctx, int on, int capacity);
 
@@ -209,29 +254,6 @@ lfm3_status lfm3_profile_enable(lfm3_ctx* ctx, int on, int capacity);
  * record. Returns LFM3_E_CAPACITY if more brackets were requested than `capacity` (the
  * excess launches ran unbracketed). */
 lfm3_status lfm3_profile_read(lfm3_ctx* ctx, int* launches, double* ms, double* bytes, double* flops);
-
-/* Phase timing of the persistent decode step (the one-launch step lfm3_decode_step uses for up
- * to 4 streams). While profiling is enabled each block of that launch stamps the device clock
- * (ns) when it starts a phase and when it has finished its share of it, into the workspace.
- * After a decode step, this synchronises the stream and, for each phase p < *n_phases (at most
- * `cap`), writes: kind[p] (0 conv in_proj+conv, 1 q|k|v|gate, 2 attention, 3 out/o_proj,
- * 4 w1|w3, 5 w2, 6 head), span_us[p] (first start to last finish over the blocks), work_us[p]
- * (mean over blocks of finish - start), work_max_us[p], wait_us[p] (mean over blocks of the
- * time the first consumer warp waited for streamed data) and lead_us[p] (mean over blocks of
- * the time from the block's last copy issue in the phase to its finish), prologue_us[p] (mean
- * time spent on the phase's input step before its units) and ahead_us[p] (mean over blocks of
- * how long before the phase started the block's first copy for it was issued). Any output array
- * may be NULL. Returns LFM3_E_STATE if profiling is off or the last decode step did not run as
- * one persistent launch. */
-lfm3_status lfm3_profile_phases(lfm3_ctx* ctx, void* stream, int cap, int* n_phases, int* kind, double* span_us,
-                                double* work_us, double* work_max_us, double* wait_us, double* lead_us,
-                                double* prologue_us, double* ahead_us);
-
-/* The raw stamps behind lfm3_profile_phases: synchronises the stream and copies up to `cap`
- * uint64 words laid out [block][256 phases][8] (device clock, ns; 0 = not stamped): phase
- * start, finish, first warp's data wait, last copy issued, input step done, first copy issued,
- * sandwich loads in, sandwich done. *n_blocks receives the number of blocks. */
-lfm3_status lfm3_profile_stamps(lfm3_ctx* ctx, void* stream, uint64_t* out, size_t cap, int* n_blocks);
 
 /* Number of kernels the last prefill/decode call enqueued. */
 int lfm3_last_launch_count(const lfm3_ctx* ctx);

@@ -223,13 +223,15 @@ def test_nvfp4_model_prefill_and_batched_decode(lib):
 # ------------------------------------------------------------------------------ 64 streams, drawn state
 
 def test_nvfp4_64_streams_on_drawn_state_sampled(lib):
-    """64 streams with shuffled pages and drawn K/V, conv and ring state; two streams checked."""
+    """64 NVFP4 streams with contexts uniform in [256, 8192] (the batched-decode workload), shuffled
+    pages and drawn K/V, conv and ring state; eight streams checked, the shortest and the longest
+    among them."""
     g = lfm3_1p7b()
     W = make_weights(g, 0, ffn="nvfp4")
     B = 64
-    ctx = context_lengths(1, "ctx64", B, 256, 1024)
+    ctx = context_lengths(1, "ctx64", B, 256, 8192)
     syn = synthetic_state(g, 1, ctx)
-    mpp = 17
+    mpp = 8192 // 64 + 1
     m = lib(W, max_streams=B, max_pages_per_stream=mpp, max_batch=B)
     pt = page_permutation(1, "pages64", B * mpp).reshape(B, mpp)
     st = m.new_state(page_table=pt)
@@ -238,10 +240,12 @@ def test_nvfp4_64_streams_on_drawn_state_sampled(lib):
     out = m.decode(st, list(range(B)), tokens=torch.from_numpy(tok).cuda())
     torch.cuda.synchronize()
     o = Lfm3Oracle(W, bf16=True)
-    for s in (0, 37):
+    order = np.argsort(ctx, kind="stable")
+    picks = sorted({int(order[0]), int(order[-1]), 0, 13, 29, 37, 50, 63})
+    for s in picks:
         ost = o.state_from_synthetic(syn, s, int(ctx[s]))
         r = o.forward_chunk(ost, tokens=tok[s:s + 1])
-        assert_logits(out["logits"][s], r["logits"], out["argmax"][s:s + 1], what=f"B=64 stream {s}")
+        assert_logits(out["logits"][s], r["logits"], out["argmax"][s:s + 1], what=f"B=64 stream {s} ctx {ctx[s]}")
     assert st.h_seq_len.tolist() == [int(c) + 1 for c in ctx]
 
 
