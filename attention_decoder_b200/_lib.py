@@ -16,10 +16,10 @@ STATUS = {0: "LFM3_OK", -1: "LFM3_E_ARG", -2: "LFM3_E_CONFIG", -3: "LFM3_E_CAPAC
           -5: "LFM3_E_UNSUPPORTED", -6: "LFM3_E_TIMEOUT", -7: "LFM3_E_STATE"}
 
 # exported entry points (every one declared in include/lfm3.h)
-SYMBOLS = ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_decode_step", "lfm3_decode_step_noalloc",
-           "lfm3_check_device_errors", "lfm3_selftest_wait",
-           "lfm3_profile_enable", "lfm3_profile_read",
-           "lfm3_last_launch_count", "lfm3_last_error", "lfm3_free")
+SYMBOLS = ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_prefill_padded", "lfm3_decode_step",
+           "lfm3_decode_step_noalloc", "lfm3_state_bytes", "lfm3_keep", "lfm3_restore", "lfm3_check_device_errors",
+           "lfm3_selftest_wait", "lfm3_profile_enable", "lfm3_profile_read", "lfm3_last_launch_count",
+           "lfm3_last_error", "lfm3_free")
 
 
 class lfm3_config(C.Structure):
@@ -64,10 +64,15 @@ def lib():
     L.lfm3_create.argtypes = [C.POINTER(lfm3_config), C.POINTER(lfm3_weights), C.POINTER(C.c_size_t), C.POINTER(vp)]
     L.lfm3_bind_workspace.argtypes = [vp, vp, C.c_size_t]
     L.lfm3_prefill.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, vp, vp, C.c_int, vp, vp, vp, vp]
+    L.lfm3_prefill_padded.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, vp, vp, C.c_int, C.c_int, vp, vp, vp, vp]
     L.lfm3_decode_step.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, i32p, vp, vp, vp, vp, vp, vp, vp]
     L.lfm3_decode_step_noalloc.argtypes = L.lfm3_decode_step.argtypes
     L.lfm3_check_device_errors.argtypes = [vp, vp]
     L.lfm3_selftest_wait.argtypes = [vp, C.c_uint, vp]
+    L.lfm3_state_bytes.argtypes = [vp, C.c_int]
+    L.lfm3_state_bytes.restype = C.c_size_t
+    L.lfm3_keep.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, vp, C.c_size_t, C.POINTER(C.c_int), vp]
+    L.lfm3_restore.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, vp, C.c_size_t, C.c_int, vp]
     L.lfm3_profile_enable.argtypes = [vp, C.c_int, C.c_int]
     dp = C.POINTER(C.c_double)
     L.lfm3_profile_read.argtypes = [vp, C.POINTER(C.c_int), dp, dp, dp]
@@ -76,9 +81,9 @@ def lib():
     L.lfm3_last_error.restype = C.c_char_p
     L.lfm3_free.argtypes = [vp]
     L.lfm3_free.restype = None
-    for name in ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_decode_step", "lfm3_decode_step_noalloc",
-                 "lfm3_check_device_errors", "lfm3_selftest_wait", "lfm3_profile_enable", "lfm3_profile_read",
-                 "lfm3_last_launch_count"):
+    for name in ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_prefill_padded", "lfm3_decode_step",
+                 "lfm3_decode_step_noalloc", "lfm3_keep", "lfm3_restore", "lfm3_check_device_errors",
+                 "lfm3_selftest_wait", "lfm3_profile_enable", "lfm3_profile_read", "lfm3_last_launch_count"):
         getattr(L, name).restype = C.c_int
     _lib = L
     return L
@@ -110,6 +115,11 @@ def lfm3_prefill(ctx, st, slot, d_tokens, d_embeds, n, d_logits, d_argmax, d_hid
     return lib().lfm3_prefill(ctx, st, slot, d_tokens, d_embeds, n, d_logits, d_argmax, d_hidden, stream)
 
 
+def lfm3_prefill_padded(ctx, st, slot, d_tokens, d_embeds, n_rows, n_real, d_logits, d_argmax, d_hidden, stream):
+    return lib().lfm3_prefill_padded(ctx, st, slot, d_tokens, d_embeds, n_rows, n_real, d_logits, d_argmax, d_hidden,
+                                     stream)
+
+
 def lfm3_decode_step(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden, stream):
     return lib().lfm3_decode_step(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax,
                                   d_hidden, stream)
@@ -119,6 +129,18 @@ def lfm3_decode_step_noalloc(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_e
                              stream):
     return lib().lfm3_decode_step_noalloc(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits,
                                           d_argmax, d_hidden, stream)
+
+
+def lfm3_state_bytes(ctx, at):
+    return lib().lfm3_state_bytes(ctx, at)
+
+
+def lfm3_keep(ctx, st, slot, d_snap, nbytes, at_out, stream):
+    return lib().lfm3_keep(ctx, st, slot, d_snap, nbytes, at_out, stream)
+
+
+def lfm3_restore(ctx, st, slot, d_snap, nbytes, at, stream):
+    return lib().lfm3_restore(ctx, st, slot, d_snap, nbytes, at, stream)
 
 
 def lfm3_check_device_errors(ctx, stream):

@@ -165,10 +165,14 @@ cudaError_t conv_decode(const float* bcx, const bf16* conv_w, bf16* state_layer,
 
 // Prefill: n consecutive rows of one slot. Block (channel group, row group of 32). Only the
 // first row group reads the carried state (rows < 6), and it also writes the new state, so
-// the read precedes the write within one thread.
+// the read precedes the write within one thread. The new state is columns [n_state, n_state + 6)
+// of [state | bx]: n_state = n, or the real rows of a chunk padded at its end (coreai-model-zoo
+// note "lfm3-1.7b-port", pad-tail paragraph: "columns [n, n + 6) of [state | Bx], n = the
+// number of query position ids >= 0").
 constexpr int CONV_RG = 32;
 __global__ void __launch_bounds__(128) k_conv_prefill(const float* __restrict__ bcx, const bf16* __restrict__ conv_w,
-                                                      bf16* __restrict__ state, int n, bf16* __restrict__ y) {
+                                                      bf16* __restrict__ state, int n, int n_state,
+                                                      bf16* __restrict__ y) {
   pdl_wait();
   pdl_launch_dependents();
   const int c = blockIdx.x * 128 + threadIdx.x;
@@ -199,15 +203,16 @@ __global__ void __launch_bounds__(128) k_conv_prefill(const float* __restrict__ 
   if (blockIdx.y == 0) {
     float ns[CST];
 #pragma unroll
-    for (int j = 0; j < CST; ++j) ns[j] = win_at(n + j);
+    for (int j = 0; j < CST; ++j) ns[j] = win_at(n_state + j);
 #pragma unroll
     for (int j = 0; j < CST; ++j) state[(size_t)j * D + c] = f2bf(ns[j]);
   }
 }
 
-cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot, int n, bf16* y, cudaStream_t s) {
+cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot, int n, int n_state, bf16* y,
+                         cudaStream_t s) {
   return launch(k_conv_prefill, dim3(D / 128, (n + CONV_RG - 1) / CONV_RG), dim3(128), 0, s, bcx, conv_w,
-                state_slot, n, y);
+                state_slot, n, n_state, y);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -388,6 +393,73 @@ __global__ void k_wait_selftest(int* err, unsigned rounds) {
 
 cudaError_t wait_selftest(int* err, unsigned rounds, cudaStream_t s) {
   return launch(k_wait_selftest, dim3(1), dim3(32), 0, s, err, rounds);
+}
+
+// ------------------------------------------------------------------------------------------
+// Kept state of one slot at a mark (TensorFold PR #1508, prompt-cache paragraph: the slot's
+// conv states and its keys and values at positions [0, at); on LFM3 also the sliding rings).
+// The snapshot is [conv: n_conv][6][D] | [ring: n_sliding][K, V][HKV][WIN][HD] |
+// [pages: n_full][K, V][ceil(at / 64)][HKV][PAGE][HD], bf16. One block per 8 KB unit of it;
+// pages are found through the slot's page table. keep: state -> snapshot; restore: snapshot ->
+// state, and seq_len[slot] = at.
+constexpr int SNAP_UNIT = 8192;
+constexpr int SNAP_CONV_UNITS = CST * D * 2 / SNAP_UNIT;              // 3
+constexpr int SNAP_RING_UNITS = HKV * WIN * HD * 2 / SNAP_UNIT;       // 32 per K or V
+constexpr int SNAP_PAGE_UNITS = HKV * PAGE * HD * 2 / SNAP_UNIT;      // 8 per K or V
+static_assert(CST * D * 2 % SNAP_UNIT == 0, "conv columns in whole units");
+
+__global__ void __launch_bounds__(256) k_state_copy(SnapArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
+  int u = blockIdx.x;
+  const char* src;
+  char* dst;
+  char* snap = reinterpret_cast<char*>(a.snap);
+  size_t soff;
+  char* st;
+  if (u < a.n_conv * SNAP_CONV_UNITS) {
+    const int j = u / SNAP_CONV_UNITS, part = u % SNAP_CONV_UNITS;
+    soff = (size_t)j * CST * D * 2 + (size_t)part * SNAP_UNIT;
+    st = reinterpret_cast<char*>(a.conv) + ((size_t)j * a.max_streams + a.slot) * CST * D * 2 + (size_t)part * SNAP_UNIT;
+  } else if ((u -= a.n_conv * SNAP_CONV_UNITS) < a.n_sliding * 2 * SNAP_RING_UNITS) {
+    const int j = u / (2 * SNAP_RING_UNITS), kv = (u / SNAP_RING_UNITS) & 1, part = u % SNAP_RING_UNITS;
+    soff = (size_t)a.n_conv * CST * D * 2 + (((size_t)j * 2 + kv) * SNAP_RING_UNITS + part) * SNAP_UNIT;
+    st = reinterpret_cast<char*>(kv ? a.ring_v : a.ring_k) + ((size_t)j * a.max_streams + a.slot) * HKV * WIN * HD * 2 +
+         (size_t)part * SNAP_UNIT;
+  } else {
+    u -= a.n_sliding * 2 * SNAP_RING_UNITS;
+    const int per = 2 * a.npg * SNAP_PAGE_UNITS;
+    const int j = u / per, kv = (u / (a.npg * SNAP_PAGE_UNITS)) & 1, pg = (u / SNAP_PAGE_UNITS) % a.npg,
+              part = u % SNAP_PAGE_UNITS;
+    soff = (size_t)a.n_conv * CST * D * 2 + (size_t)a.n_sliding * 2 * SNAP_RING_UNITS * SNAP_UNIT +
+           ((((size_t)j * 2 + kv) * a.npg + pg) * SNAP_PAGE_UNITS + part) * SNAP_UNIT;
+    const int page = a.page_table[(size_t)a.slot * a.max_pages + pg];
+    st = reinterpret_cast<char*>(kv ? a.kv_v : a.kv_k) + (((size_t)j * a.n_pages + page) * HKV * PAGE * HD) * 2 +
+         (size_t)part * SNAP_UNIT;
+  }
+  if (a.restore) {
+    src = snap + soff;
+    dst = st;
+  } else {
+    src = st;
+    dst = snap + soff;
+  }
+  for (int i = threadIdx.x; i < SNAP_UNIT / 16; i += blockDim.x)
+    stg16(dst + 16 * i, ldg16(src + 16 * i));
+  if (a.restore && blockIdx.x == 0 && threadIdx.x == 0) a.seq_len[a.slot] = a.at;
+}
+
+size_t snapshot_bytes(int n_conv, int n_sliding, int n_full, int at) {
+  const size_t npg = ((size_t)at + PAGE - 1) / PAGE;
+  return (size_t)n_conv * CST * D * 2 + (size_t)n_sliding * 2 * HKV * WIN * HD * 2 +
+         (size_t)n_full * 2 * npg * HKV * PAGE * HD * 2;
+}
+
+cudaError_t state_copy(const SnapArgs& a, cudaStream_t s) {
+  const int units = a.n_conv * SNAP_CONV_UNITS + a.n_sliding * 2 * SNAP_RING_UNITS +
+                    a.n_full * 2 * a.npg * SNAP_PAGE_UNITS;
+  if (units == 0) return cudaSuccess;
+  return launch(k_state_copy, dim3(units), dim3(256), 0, s, a);
 }
 
 }  // namespace lfm3

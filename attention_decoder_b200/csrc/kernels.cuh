@@ -60,7 +60,9 @@ cudaError_t resid_norm(float* x_res, const float* part, int n_part, long part_st
                        const bf16* g_next, bf16* xn, int rows, float eps, float* dump, cudaStream_t s);
 cudaError_t conv_decode(const float* bcx, const bf16* conv_w, bf16* state_layer, const int32_t* row_slot,
                         int rows, bf16* y, cudaStream_t s);
-cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot, int n, bf16* y, cudaStream_t s);
+// n rows; the new state is columns [n_state, n_state + 6) of [state | bx] (n_state <= n)
+cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot, int n, int n_state, bf16* y,
+                         cudaStream_t s);
 
 enum KvDst { KV_PAGES = 0, KV_SCRATCH = 1 };
 struct KvWrite {
@@ -83,6 +85,18 @@ cudaError_t finish_step(int32_t* seq_len, const int32_t* row_slot, int rows, int
                         const unsigned long long* amax, int32_t* argmax_out, cudaStream_t s);
 // One bounded wait that can never complete (at most `rounds` polls), then the status word is set.
 cudaError_t wait_selftest(int* err, unsigned rounds, cudaStream_t s);
+
+// Kept state of one slot at mark `at` (see k_state_copy): state -> snapshot (keep) or back.
+struct SnapArgs {
+  int restore, slot, at, npg;          // npg = ceil(at / PAGE) pages per full layer
+  int n_conv, n_sliding, n_full, max_streams, n_pages, max_pages;
+  void* snap;
+  bf16* conv; bf16* ring_k; bf16* ring_v; bf16* kv_k; bf16* kv_v;
+  const int32_t* page_table;
+  int32_t* seq_len;
+};
+size_t snapshot_bytes(int n_conv, int n_sliding, int n_full, int at);
+cudaError_t state_copy(const SnapArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- decode projection epilogues
 enum GemvEpi { GEMV_PARTIAL = 0, GEMV_SWIGLU = 1, GEMV_CONV = 2, GEMV_HEAD = 3 };

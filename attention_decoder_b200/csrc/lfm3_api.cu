@@ -501,10 +501,14 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
   return LFM3_OK;
 }
 
-extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slot, const int32_t* d_tokens,
-                                    const void* d_embeds, int n, float* d_logits, int32_t* d_argmax, float* d_hidden,
-                                    void* stream) {
-  if (!ctx) return LFM3_E_ARG;
+namespace {
+
+// The prompt pass of lfm3_prefill; the last n_pad rows (of the last chunk) are padding: they go
+// through the row-independent steps but not into attention, the caches, the conv state, the head
+// or seq_len.
+lfm3_status prefill_rows(lfm3_ctx* ctx, const lfm3_state* st, int slot, const int32_t* d_tokens,
+                         const void* d_embeds, int n, int n_pad, float* d_logits, int32_t* d_argmax, float* d_hidden,
+                         void* stream) {
   if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
   const lfm3_config& g = ctx->cfg;
   lfm3_status vs = check_state(ctx, st);
@@ -516,7 +520,8 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
   if (!g.has_head && (d_logits || d_argmax)) return fail(ctx, LFM3_E_ARG, "a model without head has no logits");
   const long p_start = st->h_seq_len[slot];
   if (p_start < 0) return fail(ctx, LFM3_E_ARG, "h_seq_len[%d] = %ld", slot, p_start);
-  vs = check_pages(ctx, st, slot, p_start + n);
+  const int n_real = n - n_pad;
+  vs = check_pages(ctx, st, slot, p_start + n_real);
   if (vs != LFM3_OK) return vs;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -526,8 +531,9 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
     const int nc = std::min(g.max_chunk, n - c0);
     const int p0 = (int)p_start + c0;
     const bool last = c0 + nc == n;
+    const int nr = last ? nc - n_pad : nc;  // real rows of this chunk
     CK(setup_rows(1, slot, nullptr, st->seq_len, nc, ctx->row_slot, ctx->row_pos, ctx->amax, s));
-    const Rows rows{ctx->row_slot, ctx->row_pos, nc};
+    const Rows rows{ctx->row_slot, ctx->row_pos, nr};
     CK(embed_rows(d_tokens ? d_tokens + c0 : nullptr, ctx->embed,
                   d_embeds ? B(d_embeds) + (size_t)c0 * D : nullptr, nc, ctx->x_res,
                   d_hidden ? d_hidden + (size_t)c0 * D : nullptr, s));
@@ -538,7 +544,7 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
       const Views v = views(ctx, st, l);
       if (g.layer_type[l] == LFM3_LAYER_CONV) {
         CK(run_gemm(ctx, P.in_proj, nc, s));
-        CK(conv_prefill(ctx->part, B(W.conv), v.conv_layer + (size_t)slot * CST * D, nc, ctx->y, s));
+        CK(conv_prefill(ctx->part, B(W.conv), v.conv_layer + (size_t)slot * CST * D, nc, nr, ctx->y, s));
         CK(run_gemm(ctx, P.out_proj, nc, s));
       } else {
         const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
@@ -563,7 +569,7 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
             return fail(ctx, LFM3_E_CUDA, "layer %d: K/V pool tensor map encoding failed", l);
         }
         AttnTcArgs ta{};
-        ta.n = nc;
+        ta.n = nr;
         ta.p0 = p0;
         ta.slot = slot;
         ta.full = full;
@@ -576,7 +582,7 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
         ta.err = ctx->err;
         CK(attn_prefill_tc(ctx->tm_q, full ? tk : ctx->tm_sk, full ? tv : ctx->tm_sv, ta, s));
         if (!full)
-          CK(scratch_to_ring(ctx->sk, ctx->sv, ctx->scratch_rows, nc, p0, v.ring_k, v.ring_v, slot, g.max_streams, s));
+          CK(scratch_to_ring(ctx->sk, ctx->sv, ctx->scratch_rows, nr, p0, v.ring_k, v.ring_v, slot, g.max_streams, s));
         CK(run_gemm(ctx, P.o_proj, nc, s));
       }
       CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nc, eps, nullptr, s));
@@ -591,7 +597,7 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
       WsArgs a{};
       a.w = ctx->embed;
       a.pro = WS_PRO_LOAD;
-      a.x = ctx->xn + (size_t)(nc - 1) * D;
+      a.x = ctx->xn + (size_t)(nr - 1) * D;
       a.K = D;
       a.N = g.vocab;
       a.rows = 1;
@@ -601,11 +607,31 @@ extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slo
       a.err = ctx->err;
       CK(run_ws(ctx, GEMV_HEAD, 0, ctx->ws_head, a, s));
     }
-    CK(finish_step(st->seq_len, ctx->row_slot, nc, nc, slot, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
+    CK(finish_step(st->seq_len, ctx->row_slot, nc, nr, slot, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
   }
-  st->h_seq_len[slot] += n;
+  st->h_seq_len[slot] += n_real;
   ctx->launches = g_launches;
   return LFM3_OK;
+}
+
+}  // namespace
+
+extern "C" lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slot, const int32_t* d_tokens,
+                                    const void* d_embeds, int n, float* d_logits, int32_t* d_argmax, float* d_hidden,
+                                    void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  return prefill_rows(ctx, st, slot, d_tokens, d_embeds, n, 0, d_logits, d_argmax, d_hidden, stream);
+}
+
+extern "C" lfm3_status lfm3_prefill_padded(lfm3_ctx* ctx, const lfm3_state* st, int slot, const int32_t* d_tokens,
+                                           const void* d_embeds, int n_rows, int n_real, float* d_logits,
+                                           int32_t* d_argmax, float* d_hidden, void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  if (n_rows < 1 || n_rows > ctx->cfg.max_chunk)
+    return fail(ctx, LFM3_E_ARG, "a padded chunk has 1..%d rows, not %d", ctx->cfg.max_chunk, n_rows);
+  if (n_real < 1 || n_real > n_rows) return fail(ctx, LFM3_E_ARG, "n_real %d outside 1..%d", n_real, n_rows);
+  return prefill_rows(ctx, st, slot, d_tokens, d_embeds, n_rows, n_rows - n_real, d_logits, d_argmax, d_hidden,
+                      stream);
 }
 
 namespace {
@@ -935,6 +961,84 @@ extern "C" lfm3_status lfm3_check_device_errors(lfm3_ctx* ctx, void* stream) {
     CK(cudaMemset(ctx->attn_cnt, 0, 4 * (size_t)ctx->cfg.max_batch * HKV));
     return fail(ctx, LFM3_E_TIMEOUT, "a device-side bounded wait gave up (status %d)", e);
   }
+  return LFM3_OK;
+}
+
+// ---------------------------------------------------------------- kept states (prompt cache)
+namespace {
+
+lfm3_status snap_args(lfm3_ctx* ctx, const lfm3_state* st, int slot, const void* d_snap, size_t bytes, int at,
+                      SnapArgs* a) {
+  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
+  lfm3_status vs = check_state(ctx, st);
+  if (vs != LFM3_OK) return vs;
+  const lfm3_config& g = ctx->cfg;
+  if (slot < 0 || slot >= g.max_streams) return fail(ctx, LFM3_E_ARG, "slot %d outside 0..%d", slot, g.max_streams - 1);
+  if (!d_snap || (reinterpret_cast<uintptr_t>(d_snap) & 15))
+    return fail(ctx, LFM3_E_ARG, "the kept-state buffer must be non-NULL and 16-byte aligned");
+  if (at < 0) return fail(ctx, LFM3_E_ARG, "mark %d < 0", at);
+  const size_t need = snapshot_bytes(ctx->n_conv, ctx->n_sliding, ctx->n_full, at);
+  if (bytes < need)
+    return fail(ctx, LFM3_E_CAPACITY, "a state at %d needs %zu bytes, the buffer has %zu", at, need, bytes);
+  vs = check_pages(ctx, st, slot, at);
+  if (vs != LFM3_OK) return vs;
+  *a = SnapArgs{};
+  a->slot = slot;
+  a->at = at;
+  a->npg = (at + PAGE - 1) / PAGE;
+  a->n_conv = ctx->n_conv;
+  a->n_sliding = ctx->n_sliding;
+  a->n_full = ctx->n_full;
+  a->max_streams = g.max_streams;
+  a->n_pages = g.n_pages;
+  a->max_pages = g.max_pages_per_stream;
+  a->snap = const_cast<void*>(d_snap);
+  a->conv = reinterpret_cast<bf16*>(st->conv_state);
+  a->ring_k = reinterpret_cast<bf16*>(st->ring_k);
+  a->ring_v = reinterpret_cast<bf16*>(st->ring_v);
+  a->kv_k = reinterpret_cast<bf16*>(st->kv_k);
+  a->kv_v = reinterpret_cast<bf16*>(st->kv_v);
+  a->page_table = st->page_table;
+  a->seq_len = st->seq_len;
+  return LFM3_OK;
+}
+
+}  // namespace
+
+extern "C" size_t lfm3_state_bytes(const lfm3_ctx* ctx, int at) {
+  if (!ctx || at < 0) return 0;
+  return snapshot_bytes(ctx->n_conv, ctx->n_sliding, ctx->n_full, at);
+}
+
+extern "C" lfm3_status lfm3_keep(lfm3_ctx* ctx, const lfm3_state* st, int slot, void* d_snap, size_t bytes,
+                                 int* at_out, void* stream) {
+  if (!ctx || !at_out) return LFM3_E_ARG;
+  if (!st || !st->h_seq_len) return fail(ctx, LFM3_E_ARG, "state / h_seq_len is NULL");
+  if (slot < 0 || slot >= ctx->cfg.max_streams) return fail(ctx, LFM3_E_ARG, "slot %d outside 0..%d", slot,
+                                                            ctx->cfg.max_streams - 1);
+  SnapArgs a;
+  const int at = st->h_seq_len[slot];
+  lfm3_status vs = snap_args(ctx, st, slot, d_snap, bytes, at, &a);
+  if (vs != LFM3_OK) return vs;
+  g_launches = 0;
+  a.restore = 0;
+  CK(state_copy(a, reinterpret_cast<cudaStream_t>(stream)));
+  ctx->launches = g_launches;
+  *at_out = at;
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_restore(lfm3_ctx* ctx, const lfm3_state* st, int slot, const void* d_snap, size_t bytes,
+                                    int at, void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  SnapArgs a;
+  lfm3_status vs = snap_args(ctx, st, slot, d_snap, bytes, at, &a);
+  if (vs != LFM3_OK) return vs;
+  g_launches = 0;
+  a.restore = 1;
+  CK(state_copy(a, reinterpret_cast<cudaStream_t>(stream)));
+  ctx->launches = g_launches;
+  st->h_seq_len[slot] = at;
   return LFM3_OK;
 }
 

@@ -127,6 +127,23 @@ class Lfm3Model:
     def check_device_errors(self, stream=None):
         check(L.lfm3_check_device_errors(self.ctx, _stream(stream)), self.ctx)
 
+    def state_bytes(self, at: int) -> int:
+        return int(L.lfm3_state_bytes(self.ctx, at))
+
+    def keep(self, st, slot, buf=None, stream=None):
+        """Keeps slot's state at its current position; returns (mark, device buffer)."""
+        at = int(st.h_seq_len[slot])
+        n = self.state_bytes(at)
+        if buf is None:
+            buf = torch.empty(n, dtype=torch.uint8, device=self.device)
+        out = C.c_int()
+        check(L.lfm3_keep(self.ctx, C.byref(st.struct), slot, _ptr(buf), buf.numel(), C.byref(out), _stream(stream)),
+              self.ctx)
+        return out.value, buf
+
+    def restore(self, st, slot, at, buf, stream=None):
+        check(L.lfm3_restore(self.ctx, C.byref(st.struct), slot, _ptr(buf), buf.numel(), at, _stream(stream)), self.ctx)
+
     def selftest_wait(self, rounds=4096, stream=None):
         check(L.lfm3_selftest_wait(self.ctx, rounds, _stream(stream)), self.ctx)
 
@@ -146,6 +163,23 @@ class Lfm3Model:
             out["hidden"] = torch.empty(g.n_layers + 1, n, g.d_model, dtype=torch.float32, device=self.device)
         check(L.lfm3_prefill(self.ctx, C.byref(st.struct), slot, _ptr(tokens), _ptr(embeds), n, _ptr(out.get("logits")),
                              _ptr(out.get("argmax")), _ptr(out.get("hidden")), _stream(stream)), self.ctx)
+        return out
+
+    def prefill_padded(self, st, slot, n_real, tokens=None, embeds=None, logits=True, argmax=True, hidden=False,
+                       stream=None):
+        """One chunk whose rows past n_real are padding (see lfm3_prefill_padded)."""
+        g = self.geom
+        n = int(tokens.shape[0] if tokens is not None else embeds.shape[0])
+        out = {}
+        if g.has_head and logits:
+            out["logits"] = torch.empty(g.vocab, dtype=torch.float32, device=self.device)
+        if g.has_head and argmax:
+            out["argmax"] = torch.empty(1, dtype=torch.int32, device=self.device)
+        if hidden:
+            out["hidden"] = torch.empty(g.n_layers + 1, n, g.d_model, dtype=torch.float32, device=self.device)
+        check(L.lfm3_prefill_padded(self.ctx, C.byref(st.struct), slot, _ptr(tokens), _ptr(embeds), n, n_real,
+                                    _ptr(out.get("logits")), _ptr(out.get("argmax")), _ptr(out.get("hidden")),
+                                    _stream(stream)), self.ctx)
         return out
 
     def decode(self, st, slots, tokens=None, embeds=None, logits=True, argmax=True, hidden=False, stream=None,

@@ -182,6 +182,20 @@ lfm3_status lfm3_prefill(lfm3_ctx* ctx, const lfm3_state* st, int slot, const in
                          const void* d_embeds, int n, float* d_logits, int32_t* d_argmax,
                          float* d_hidden, void* stream);
 
+/* A prompt chunk padded at its end (coreai-model-zoo note "lfm3-1.7b-port", pad-tail paragraph):
+ * n_rows rows (1..max_chunk) of which the first n_real (>= 1) are the prompt and the rest are
+ * padding (the pages' engine writes token 0 there). Every row goes through the row-wise steps (the
+ * projections, norms and FFN), so a caller can keep one fixed chunk shape; but no real row sees a
+ * pad, the pads' keys and values are not stored, the conv state is columns [n_real, n_real + 6)
+ * of [state | Bx] ("n = the number of query position ids >= 0") rather than the last 6, d_logits
+ * and d_argmax belong to row n_real - 1, and seq_len advances by n_real. The real rows' results
+ * and the state equal those of lfm3_prefill on the n_real rows alone. d_hidden, if given, holds
+ * n_rows rows; the pad rows' values there are unspecified. Capacity is checked for the real rows
+ * only. Errors: as lfm3_prefill, and LFM3_E_ARG for n_rows or n_real out of range. */
+lfm3_status lfm3_prefill_padded(lfm3_ctx* ctx, const lfm3_state* st, int slot, const int32_t* d_tokens,
+                                const void* d_embeds, int n_rows, int n_real, float* d_logits, int32_t* d_argmax,
+                                float* d_hidden, void* stream);
+
 /* One decode step for n_streams distinct slots (one row each, at position seq_len[slot]; as for
  * lfm3_prefill the position comes from the state and there is no mask input - coreai-model-zoo
  * note "lfm3-1.7b-port", "window_size, with no mask input"). Streams share no state; the pages'
@@ -225,6 +239,36 @@ lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int n_streams,
 lfm3_status lfm3_decode_step_noalloc(lfm3_ctx* ctx, const lfm3_state* st, int n_streams, const int32_t* h_slots,
                                      const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
                                      float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream);
+
+/* Kept states (the prompt cache; TensorFold PR #1508, prompt-cache paragraph): "a state at `at` is
+ * the slot's conv states and its keys and values at positions [0, at)"; on LFM3 it also holds
+ * every sliding layer's ring, the model's other fixed region (same PR, "One backend" paragraph).
+ * A state is kept behind a prompt chunk that ends at the mark and restored into another slot (its
+ * own pages) before that slot's next chunk, so the later pass starts at its history; resumed ==
+ * fresh, bit for bit. The buffer is caller-owned device memory, 16-byte aligned, laid out as
+ *   [n_conv][conv_taps-1][d_model] | [n_sliding][K, V][n_kv][window][head_dim] |
+ *   [n_full][K, V][ceil(at / page_size)][n_kv][page_size][head_dim]            (bf16)
+ * Both calls enqueue one copy kernel on `stream` and allocate nothing. A mark inside a chunk
+ * (the pages' "taps") is not offered: on LFM3 it needs the rings as they stood at the mark. */
+
+/* Bytes of a state kept at mark `at` (0 for a NULL context or a negative mark). */
+size_t lfm3_state_bytes(const lfm3_ctx* ctx, int at);
+
+/* Keeps the state of `slot` at its current position: *at_out = h_seq_len[slot], and d_snap
+ * (>= lfm3_state_bytes(at) bytes) receives its conv columns, rings and pages [0, at).
+ * Errors: LFM3_E_CAPACITY if the buffer is too small; LFM3_E_ARG for a bad slot or buffer;
+ * LFM3_E_STATE before lfm3_bind_workspace. Nothing is enqueued on error. */
+lfm3_status lfm3_keep(lfm3_ctx* ctx, const lfm3_state* st, int slot, void* d_snap, size_t bytes, int* at_out,
+                      void* stream);
+
+/* Restores a state kept at mark `at` into `slot`: conv columns and rings are overwritten, the
+ * kept pages are written into the slot's own pages (through its page table), and seq_len[slot]
+ * and h_seq_len[slot] become `at`. The slot's previous contents are discarded. Errors:
+ * LFM3_E_CAPACITY if the slot's pages cannot hold [0, at) or the buffer is too small (TensorFold
+ * PR #1508, pool-leasing commit: "forward refuses rows past a slot's pages"); LFM3_E_ARG for a
+ * bad slot, buffer or mark. Nothing is enqueued and no state is touched on error. */
+lfm3_status lfm3_restore(lfm3_ctx* ctx, const lfm3_state* st, int slot, const void* d_snap, size_t bytes, int at,
+                         void* stream);
 
 /* Synchronises the stream and reads the device status word that bounded device-side waits set
  * when they give up (every wait on a copy or a peer block in the kernels has an iteration limit

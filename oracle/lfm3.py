@@ -395,6 +395,17 @@ class Lfm3Oracle:
             out["logits"] = self.logits(x)
         return out
 
+    def keep(self, st: OracleState) -> OracleState:
+        """The state at the mark at = st.seq_len, as an independent copy: the conv columns, the
+        sliding rings and the keys / values of positions [0, at) of the full layers (TensorFold
+        PR #1508, prompt-cache paragraph: "a state at `at` is the slot's conv states and its keys
+        and values at positions [0, at)"). Restoring is continuing from the copy."""
+        return OracleState(conv=[a.copy() for a in st.conv],
+                           full_k=[a[:st.seq_len].copy() for a in st.full_k],
+                           full_v=[a[:st.seq_len].copy() for a in st.full_v],
+                           ring_k=[a.copy() for a in st.ring_k], ring_v=[a.copy() for a in st.ring_v],
+                           ring_pos=[a.copy() for a in st.ring_pos], seq_len=st.seq_len)
+
     def greedy(self, st: OracleState, first_token: int, steps: int):
         """Greedy decode: feed ``first_token``, then each argmax (ties -> lowest id).
         Returns (tokens fed [steps], logits [steps, V])."""

@@ -121,3 +121,27 @@ def test_three_block_slice_modes_agree():
     for li in range(1, g.n_layers + 1):
         dlt = ref["hidden"][li] - ref["hidden"][li - 1]
         assert 0.3 < np.sqrt(np.mean(dlt * dlt)) < 5.0
+
+
+@pytest.mark.parametrize("at", [5, 8, 13])
+def test_kept_state_resumes_like_the_fresh_pass(tiny, at):
+    """Keep at a mark (a chunk that ends at position `at`), then continue both the original and
+    the kept copy with the rest of the prompt: both equal the full-sequence pass, and continuing
+    one does not disturb the other (TensorFold PR #1508: "resumed against fresh")."""
+    g, W, tok, o, ref = tiny
+    st = o.new_state()
+    o.forward_chunk(st, tokens=tok[:at], logits="all")
+    kept = o.keep(st)
+    a = o.forward_chunk(st, tokens=tok[at:], logits="all")
+    b = o.forward_chunk(kept, tokens=tok[at:], logits="all")
+    assert np.array_equal(a["logits"], b["logits"])
+    assert _close(b["logits"], ref["logits"][at:])
+    for li in range(g.n_layers + 1):
+        assert _close(b["hidden"][li], ref["hidden"][li][at:]), li
+    # a second resume from a fresh keep of the same mark gives the same rows again
+    st2 = o.new_state()
+    o.forward_chunk(st2, tokens=tok[:at], logits="all")
+    k2 = o.keep(st2)
+    o.forward_chunk(st2, tokens=tok[at:at + 3], logits="all")   # the source moves on
+    c = o.forward_chunk(k2, tokens=tok[at:], logits="all")
+    assert np.array_equal(c["logits"], b["logits"])

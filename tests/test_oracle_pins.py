@@ -445,3 +445,23 @@ def test_bf16_boundary_mode_keeps_the_invariants_and_stores_bf16_state():
     exact = Lfm3Oracle(W).forward_full(tokens=tok, logits="all")
     d = np.abs(full["hidden"][-1] - exact["hidden"][-1]).max() / np.abs(exact["hidden"][-1]).max()
     assert 1e-5 < d < 5e-2
+
+
+@pytest.mark.parametrize("n_real,n_pad", [(1, 63), (5, 59), (6, 58), (37, 27), (64, 0)])
+def test_pad_tail_state_is_columns_n_to_n_plus_6_of_the_padded_window(n_real, n_pad):
+    """coreai-model-zoo note "lfm3-1.7b-port", pad-tail paragraph: a chunk padded at its end reads
+    its new conv state from columns [n, n + 6) of [state | Bx], n = the real rows. The oracle's
+    chunked conv, run on the real rows alone, commits exactly those columns of the padded window
+    whatever the pads hold, and the real rows' conv outputs do not see the pads."""
+    r = np.random.default_rng(14)
+    C = 24
+    w = r.standard_normal((C, 7))
+    state = r.standard_normal((6, C))
+    bx = r.standard_normal((n_real, C))
+    pads = np.full((n_pad, C), np.nan)
+    win = np.concatenate([state, bx, pads], axis=0)
+    z, st_new = causal_conv_chunk(state, bx, w)
+    assert np.array_equal(win[n_real:n_real + 6], st_new)
+    pads = r.standard_normal((n_pad, C)) * 1e3
+    z_pad, _ = causal_conv_chunk(state, np.concatenate([bx, pads], axis=0), w)
+    assert np.array_equal(z_pad[:n_real], z)
