@@ -17,7 +17,7 @@ STATUS = {0: "LFM3_OK", -1: "LFM3_E_ARG", -2: "LFM3_E_CONFIG", -3: "LFM3_E_CAPAC
 
 # exported entry points (every one declared in include/lfm3.h)
 SYMBOLS = ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_prefill_padded", "lfm3_decode_step",
-           "lfm3_decode_step_noalloc", "lfm3_state_bytes", "lfm3_keep", "lfm3_restore", "lfm3_check_device_errors",
+           "lfm3_verify", "lfm3_commit", "lfm3_decode_step_noalloc", "lfm3_state_bytes", "lfm3_keep", "lfm3_restore", "lfm3_check_device_errors",
            "lfm3_selftest_wait", "lfm3_profile_enable", "lfm3_profile_read", "lfm3_last_launch_count",
            "lfm3_last_error", "lfm3_free")
 
@@ -67,6 +67,8 @@ def lib():
     L.lfm3_prefill_padded.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, vp, vp, C.c_int, C.c_int, vp, vp, vp, vp]
     L.lfm3_decode_step.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, i32p, vp, vp, vp, vp, vp, vp, vp]
     L.lfm3_decode_step_noalloc.argtypes = L.lfm3_decode_step.argtypes
+    L.lfm3_verify.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, i32p, vp, C.c_int, vp, vp, vp, vp, vp, vp]
+    L.lfm3_commit.argtypes = [vp, C.POINTER(lfm3_state), C.c_int, i32p, i32p, vp]
     L.lfm3_check_device_errors.argtypes = [vp, vp]
     L.lfm3_selftest_wait.argtypes = [vp, C.c_uint, vp]
     L.lfm3_state_bytes.argtypes = [vp, C.c_int]
@@ -82,7 +84,7 @@ def lib():
     L.lfm3_free.argtypes = [vp]
     L.lfm3_free.restype = None
     for name in ("lfm3_create", "lfm3_bind_workspace", "lfm3_prefill", "lfm3_prefill_padded", "lfm3_decode_step",
-                 "lfm3_decode_step_noalloc", "lfm3_keep", "lfm3_restore", "lfm3_check_device_errors",
+                 "lfm3_verify", "lfm3_commit", "lfm3_decode_step_noalloc", "lfm3_keep", "lfm3_restore", "lfm3_check_device_errors",
                  "lfm3_selftest_wait", "lfm3_profile_enable", "lfm3_profile_read", "lfm3_last_launch_count"):
         getattr(L, name).restype = C.c_int
     _lib = L
@@ -123,6 +125,15 @@ def lfm3_prefill_padded(ctx, st, slot, d_tokens, d_embeds, n_rows, n_real, d_log
 def lfm3_decode_step(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden, stream):
     return lib().lfm3_decode_step(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax,
                                   d_hidden, stream)
+
+
+def lfm3_verify(ctx, st, n_streams, h_slots, d_slots, W, d_tokens, d_embeds, d_logits, d_argmax, d_hidden, stream):
+    return lib().lfm3_verify(ctx, st, n_streams, h_slots, d_slots, W, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                             stream)
+
+
+def lfm3_commit(ctx, st, n_streams, h_slots, h_accept, stream):
+    return lib().lfm3_commit(ctx, st, n_streams, h_slots, h_accept, stream)
 
 
 def lfm3_decode_step_noalloc(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,

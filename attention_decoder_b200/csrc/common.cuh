@@ -110,3 +110,27 @@ DEVI void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) 
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
 }
+
+// ---------------------------------------------------------------- optional launch timeline
+// Built only with -DLFM3_TRACE (a diagnostic build): blocks stamp the global timer (ns) into a
+// caller-provided buffer [launch][block][8]; the product build has none of this.
+#ifdef LFM3_TRACE
+constexpr int TRACE_BLOCKS = 512;
+DEVI void trace_at(unsigned long long* buf, int id, int slot) {
+  if (!buf || id < 0 || id >= 256) return;
+  const unsigned blk = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  if (blk >= TRACE_BLOCKS) return;
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  if (slot == 7) {
+    unsigned sm;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+    t = sm;
+  }
+  buf[((size_t)id * TRACE_BLOCKS + blk) * 8 + slot] = t;
+}
+#define TRACE(buf, id, slot) trace_at(buf, id, slot)
+#else
+#define TRACE(buf, id, slot) ((void)0)
+#endif
+

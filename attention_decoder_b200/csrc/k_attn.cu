@@ -59,11 +59,19 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
   __shared__ __align__(16) float obuf[4][GQA][HD];       // PV of the four key quarters
   __shared__ float red[GQA + 1][4];
   __shared__ float lx[GQA];
+  __shared__ __align__(16) bf16 wk[MAX_WIN][HD], wv[MAX_WIN][HD];  // earlier rows of a verify window
+  __shared__ float kw[HD];
   __shared__ __align__(8) uint64_t kv_bar;
   __shared__ int last;
 
   const int sp = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#ifdef LFM3_TRACE
+  if (tid == 0) {
+    TRACE(A.trace, A.trace_id, 0);
+    TRACE(A.trace, A.trace_id, 7);
+  }
+#endif
   // rows were set by the first kernel of the step, which has completed (reads go to L2)
   const int slot = __ldcg(rows.slot + b), pos = __ldcg(rows.pos + b);
   const int nkeys = L.full ? pos + 1 : min(pos + 1, WIN);
@@ -90,6 +98,9 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
   const float cr = A.rope_cos[(size_t)pos * (HD / 2) + ir], sr = A.rope_sin[(size_t)pos * (HD / 2) + ir];
   pdl_wait();
   pdl_launch_dependents();
+#ifdef LFM3_TRACE
+  if (tid == 0) TRACE(A.trace, A.trace_id, 2);
+#endif
 
   // ---- queries and the new key / value (threads 0..127: thread = dimension d of each head)
   const float* raw = qkvg + (size_t)b * NQKVG;
@@ -129,21 +140,62 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
   __syncthreads();
   const float scale = rsqrtf((float)HD);
   const bool has_cur = cur >= j0 && cur < j0 + cnt;
+  const int wi = b % A.win;  // this row's index in its stream's verify window (0 when decoding)
   if (tid < HD) {
 #pragma unroll
     for (int hh = 0; hh < GQA; ++hh) qs[hh][d] = qr[hh] * scale;
     if (has_cur) {  // the new key and value into the cache, as every later step reads them
-      const size_t row = tile + (size_t)(cur - j0) * HD + d;
-      const_cast<bf16*>(L.k)[row] = f2bf(kr);
-      const_cast<bf16*>(L.v)[row] = f2bf(vv);
+      if (L.full || A.win == 1) {
+        const size_t row = tile + (size_t)(cur - j0) * HD + d;
+        const_cast<bf16*>(L.k)[row] = f2bf(kr);
+        const_cast<bf16*>(L.v)[row] = f2bf(vv);
+      } else {  // a verify window's sliding rows wait for the commit in the side buffer
+        A.side_k[((size_t)b * HKV + kvh) * HD + d] = f2bf(kr);
+        A.side_v[((size_t)b * HKV + kvh) * HD + d] = f2bf(vv);
+      }
     }
   }
-  // ---- the staged split; the current position's row there is stale: put the new one in
+  // the window's earlier rows (positions pos - wi .. pos - 1) are not in the cache yet: compute
+  // their keys and values here (norm, rotary at their own positions, bf16) for this split
+  for (int ip = 0; ip < wi; ++ip) {
+    const int pp = pos - wi + ip;
+    const int kidx = L.full ? pp : pp % WIN;
+    if (kidx < j0 || kidx >= j0 + cnt) continue;  // uniform over the block
+    const float* rw = qkvg + (size_t)(b - wi + ip) * NQKVG;
+    float k1 = 0.f, v1 = 0.f;
+    if (tid < HD) {
+      k1 = rw[HQ * HD + kvh * HD + d];
+      v1 = rw[HQ * HD + HKV * HD + kvh * HD + d];
+      const float s2 = warp_sum(k1 * k1);
+      if (lane == 0) red[0][warp] = s2;
+    }
+    __syncthreads();
+    if (tid < HD) kw[d] = gk * (k1 * rsqrtf((red[0][0] + red[0][1] + red[0][2] + red[0][3]) * (1.0f / HD) + A.eps));
+    __syncthreads();
+    if (tid < HD) {
+      const float c1 = A.rope_cos[(size_t)pp * (HD / 2) + ir], s1 = A.rope_sin[(size_t)pp * (HD / 2) + ir];
+      wk[ip][d] = f2bf(d < 64 ? kw[d] * c1 - kw[pd] * s1 : kw[d] * c1 + kw[pd] * s1);
+      wv[ip][d] = f2bf(v1);
+    }
+    __syncthreads();
+  }
+  // ---- the staged split; the rows of the current position (and of the window's earlier ones)
+  // there are stale: put the new ones in
   bool ok = mbar_wait(su32(&kv_bar), 0, A.err);
   if (!ok) ok = mbar_wait(su32(&kv_bar), 0, A.err);  // a copy still in flight must land before exit
-  if (has_cur && tid < HD) {
-    ks[(cur - j0) * HD + d] = f2bf(kr);
-    vs[(cur - j0) * HD + d] = f2bf(vv);
+  if (tid < HD) {
+    if (has_cur) {
+      ks[(cur - j0) * HD + d] = f2bf(kr);
+      vs[(cur - j0) * HD + d] = f2bf(vv);
+    }
+    for (int ip = 0; ip < wi; ++ip) {
+      const int pp = pos - wi + ip;
+      const int kidx = L.full ? pp : pp % WIN;
+      if (kidx >= j0 && kidx < j0 + cnt) {
+        ks[(kidx - j0) * HD + d] = wk[ip][d];
+        vs[(kidx - j0) * HD + d] = wv[ip][d];
+      }
+    }
   }
   __syncthreads();
 
@@ -234,6 +286,9 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
   // ---- the last block of (stream, kv head) merges the splits and applies the gates
   __threadfence();
   __syncthreads();
+#ifdef LFM3_TRACE
+  if (tid == 0) TRACE(A.trace, A.trace_id, 3);
+#endif
   if (tid == 0) last = atomicAdd(A.counters + b * HKV + kvh, 1u) == (unsigned)(nact - 1);
   __syncthreads();
   if (!last) return;
@@ -280,12 +335,23 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
     *reinterpret_cast<uint2*>(yo) = w;
   }
   if (tid == 0) A.counters[b * HKV + kvh] = 0u;
+#ifdef LFM3_TRACE
+  if (tid == 0) TRACE(A.trace, A.trace_id, 5);
+#endif
 }
 
 cudaError_t attn_decode_fused(const float* qkvg, Rows rows, AttnLayer L, const AttnDecodeArgs& A, int splits,
                               float* part, bf16* y, cudaStream_t s) {
+#ifdef LFM3_TRACE
+  AttnDecodeArgs At = A;
+  At.trace = g_trace;
+  At.trace_id = g_launches;
+  return launch(k_attn_decode_fused, dim3(splits, HKV, rows.n), dim3(DA_THREADS), DA_SMEM, s, qkvg, rows, L, At,
+                splits, part, y);
+#else
   return launch(k_attn_decode_fused, dim3(splits, HKV, rows.n), dim3(DA_THREADS), DA_SMEM, s, qkvg, rows, L, A, splits,
                 part, y);
+#endif
 }
 
 cudaError_t attn_init() {

@@ -6,13 +6,16 @@
 namespace lfm3 {
 
 thread_local int g_launches = 0;
+#ifdef LFM3_TRACE
+unsigned long long* g_trace = nullptr;
+#endif
 
 // ------------------------------------------------------------------------------------------
 // Row bookkeeping: prefill rows are consecutive positions of one slot; decode rows are one
 // position of each listed slot. Also clears the per-row greedy cells.
 __global__ void k_setup_rows(int prefill, int slot, const int32_t* __restrict__ d_slots,
-                             const int32_t* __restrict__ seq_len, int rows, int32_t* row_slot, int32_t* row_pos,
-                             unsigned long long* amax) {
+                             const int32_t* __restrict__ seq_len, int rows, int win, int32_t* row_slot,
+                             int32_t* row_pos, unsigned long long* amax) {
   pdl_wait();
   pdl_launch_dependents();
   int r = blockIdx.x * blockDim.x + threadIdx.x;
@@ -21,17 +24,17 @@ __global__ void k_setup_rows(int prefill, int slot, const int32_t* __restrict__ 
     row_slot[r] = slot;
     row_pos[r] = seq_len[slot] + r;
   } else {
-    int s = d_slots[r];
+    int s = d_slots[r / win];
     row_slot[r] = s;
-    row_pos[r] = seq_len[s];
+    row_pos[r] = seq_len[s] + r % win;
   }
   if (amax) amax[r] = 0ull;
 }
 
-cudaError_t setup_rows(int prefill, int slot, const int32_t* d_slots, const int32_t* seq_len, int rows,
+cudaError_t setup_rows(int prefill, int slot, const int32_t* d_slots, const int32_t* seq_len, int rows, int win,
                        int32_t* row_slot, int32_t* row_pos, unsigned long long* amax, cudaStream_t s) {
   return launch(k_setup_rows, dim3((rows + 127) / 128), dim3(128), 0, s, prefill, slot, d_slots, seq_len, rows,
-                row_slot, row_pos, amax);
+                win < 1 ? 1 : win, row_slot, row_pos, amax);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -135,32 +138,50 @@ cudaError_t resid_norm(float* x_res, const float* part, int n_part, long part_st
 // Decode: one row per stream, state [slot][6][D] shifts by one column.
 __global__ void __launch_bounds__(256) k_conv_decode(const float* __restrict__ bcx, const bf16* __restrict__ conv_w,
                                                      bf16* __restrict__ state, const int32_t* __restrict__ row_slot,
-                                                     bf16* __restrict__ y) {
+                                                     int win, bf16* __restrict__ snap, bf16* __restrict__ y) {
   pdl_wait();
   pdl_launch_dependents();
   const int b = blockIdx.y;
   const int c = blockIdx.x * 256 + threadIdx.x;
   const float* row = bcx + (size_t)b * 3 * D;
-  const float Bv = row[c], Cv = row[D + c], Xv = row[2 * D + c];
-  const float bx = round_bf(Bv * Xv);
+  const float Cv = row[D + c];
   bf16* st = state + (size_t)row_slot[b] * CST * D + c;
-  float win[CST];
-#pragma unroll
-  for (int j = 0; j < CST; ++j) win[j] = bf2f(st[(size_t)j * D]);
   const bf16* w = conv_w + (size_t)c * TAPS;
+  if (win <= 1) {
+    const float bx = round_bf(row[c] * row[2 * D + c]);
+    float win6[CST];
+#pragma unroll
+    for (int j = 0; j < CST; ++j) win6[j] = bf2f(st[(size_t)j * D]);
+    float z = 0.f;
+#pragma unroll
+    for (int k = 0; k < CST; ++k) z += bf2f(w[k]) * win6[k];
+    z += bf2f(w[CST]) * bx;
+    y[(size_t)b * D + c] = f2bf(Cv * z);
+#pragma unroll
+    for (int j = 0; j < CST - 1; ++j) st[(size_t)j * D] = f2bf(win6[j + 1]);
+    st[(size_t)(CST - 1) * D] = f2bf(bx);
+    return;
+  }
+  // verify window: row wi of its stream sees [state | bx of the window's rows 0..wi]
+  const int wi = b % win, b0 = b - wi;
+  float wnd[CST + MAX_WIN];
+#pragma unroll
+  for (int j = 0; j < CST; ++j) wnd[j] = bf2f(st[(size_t)j * D]);
+  for (int i = 0; i <= wi; ++i) {
+    const float* ri = bcx + (size_t)(b0 + i) * 3 * D;
+    wnd[CST + i] = round_bf(ri[c] * ri[2 * D + c]);
+  }
   float z = 0.f;
 #pragma unroll
-  for (int k = 0; k < CST; ++k) z += bf2f(w[k]) * win[k];
-  z += bf2f(w[CST]) * bx;
+  for (int k = 0; k < TAPS; ++k) z += bf2f(w[k]) * wnd[wi + k];
   y[(size_t)b * D + c] = f2bf(Cv * z);
 #pragma unroll
-  for (int j = 0; j < CST - 1; ++j) st[(size_t)j * D] = f2bf(win[j + 1]);
-  st[(size_t)(CST - 1) * D] = f2bf(bx);
+  for (int j = 0; j < CST; ++j) snap[((size_t)b * CST + j) * D + c] = f2bf(wnd[wi + 1 + j]);
 }
 
 cudaError_t conv_decode(const float* bcx, const bf16* conv_w, bf16* state_layer, const int32_t* row_slot, int rows,
-                        bf16* y, cudaStream_t s) {
-  return launch(k_conv_decode, dim3(D / 256, rows), dim3(256), 0, s, bcx, conv_w, state_layer, row_slot, y);
+                        int win, bf16* snap, bf16* y, cudaStream_t s) {
+  return launch(k_conv_decode, dim3(D / 256, rows), dim3(256), 0, s, bcx, conv_w, state_layer, row_slot, win, snap, y);
 }
 
 // Prefill: n consecutive rows of one slot. Block (channel group, row group of 32). Only the
@@ -351,7 +372,8 @@ cudaError_t scratch_to_ring(const bf16* sk, const bf16* sv, int scratch_rows, in
 // End of a call: advance seq_len and publish greedy ids (the cells hold (ordered value << 32) |
 // (0xffffffff - id), so the max is the largest logit with the lowest id among ties).
 __global__ void k_finish(int32_t* seq_len, const int32_t* __restrict__ row_slot, int rows, int add_prefill,
-                         int prefill_slot, const unsigned long long* __restrict__ amax, int32_t* argmax_out) {
+                         int prefill_slot, const unsigned long long* __restrict__ amax, int32_t* argmax_out,
+                         int advance) {
   pdl_wait();
   pdl_launch_dependents();
   const int r = threadIdx.x;
@@ -363,15 +385,50 @@ __global__ void k_finish(int32_t* seq_len, const int32_t* __restrict__ row_slot,
     return;
   }
   if (r < rows) {
-    seq_len[row_slot[r]] += 1;
+    if (advance) seq_len[row_slot[r]] += 1;
     if (argmax_out && amax) argmax_out[r] = (int32_t)(0xffffffffu - (uint32_t)(amax[r] & 0xffffffffull));
   }
 }
 
 cudaError_t finish_step(int32_t* seq_len, const int32_t* row_slot, int rows, int add_prefill, int prefill_slot,
-                        const unsigned long long* amax, int32_t* argmax_out, cudaStream_t s) {
+                        const unsigned long long* amax, int32_t* argmax_out, int advance, cudaStream_t s) {
   return launch(k_finish, dim3(1), dim3(64), 0, s, seq_len, row_slot, rows, add_prefill, prefill_slot, amax,
-                argmax_out);
+                argmax_out, advance);
+}
+
+// ------------------------------------------------------------------------------------------
+// Commit of verify windows (TensorFold PR #1508, lfm2_moe.cu paragraph: "the commit of an
+// accepted row's conv state"): for stream i, with k = a.k[i] accepted rows of its window,
+// the conv state becomes the snapshot after row k - 1, the sliding rings take the window's first
+// k rows at their slots, and seq_len advances by k. Block (stream, unit): units 0 .. n_conv - 1
+// copy one layer's conv columns, the rest one (sliding layer, accepted row).
+__global__ void __launch_bounds__(256) k_commit(CommitArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int i = blockIdx.x, u = blockIdx.y;
+  const int slot = a.slot[i], k = a.k[i];
+  if (u < a.n_conv) {
+    const uint4* src = reinterpret_cast<const uint4*>(
+        a.snap + (((size_t)u * a.max_batch + (size_t)i * a.W + k - 1) * CST) * D);
+    uint4* dst = reinterpret_cast<uint4*>(a.conv + (((size_t)u * a.max_streams + slot) * CST) * D);
+    for (int e = threadIdx.x; e < CST * D / 8; e += blockDim.x) dst[e] = src[e];
+  } else {
+    const int j = (u - a.n_conv) / MAX_WIN, r = (u - a.n_conv) % MAX_WIN;
+    if (r < k) {
+      const int ringpos = (a.pos[i] + r) % WIN;
+      for (int e = threadIdx.x; e < 2 * HKV * HD / 8; e += blockDim.x) {
+        const int kv = e / (HKV * HD / 8), hc = e % (HKV * HD / 8), h = hc / (HD / 8), c8 = hc % (HD / 8);
+        const bf16* sb = (kv ? a.side_v : a.side_k) + (((size_t)j * a.max_batch + (size_t)i * a.W + r) * HKV + h) * HD;
+        bf16* rb = (kv ? a.ring_v : a.ring_k) + ((((size_t)j * a.max_streams + slot) * HKV + h) * WIN + ringpos) * HD;
+        reinterpret_cast<uint4*>(rb)[c8] = reinterpret_cast<const uint4*>(sb)[c8];
+      }
+    }
+  }
+  if (u == 0 && threadIdx.x == 0) a.seq_len[slot] = a.pos[i] + k;
+}
+
+cudaError_t commit_windows(const CommitArgs& a, cudaStream_t s) {
+  return launch(k_commit, dim3(a.n, a.n_conv + a.n_sliding * MAX_WIN), dim3(256), 0, s, a);
 }
 
 // ------------------------------------------------------------------------------------------

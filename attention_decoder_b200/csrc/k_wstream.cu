@@ -27,8 +27,23 @@
 
 #include <algorithm>
 #include <cstdlib>
+#include <mutex>
 
 #include "kernels.cuh"
+
+// Ring depths (stages) and blocks per SM; compile-time, measured on B200.
+#ifndef LFM3_WS_STAGES_BF16
+#define LFM3_WS_STAGES_BF16 5
+#endif
+#ifndef LFM3_WS_STAGES_CONV
+#define LFM3_WS_STAGES_CONV 5
+#endif
+#ifndef LFM3_WS_STAGES_FP4
+#define LFM3_WS_STAGES_FP4 12
+#endif
+#ifndef LFM3_WS_BPS
+#define LFM3_WS_BPS 2
+#endif
 
 namespace lfm3 {
 
@@ -47,22 +62,29 @@ struct WsGeom {
   static constexpr int RPT = 16 * NRT;                        // weight rows per tile
   static constexpr int BR = EPI == GEMV_SWIGLU ? 8 : 16;      // rows per copy request (w1 | w3 halves)
   static constexpr int NREQ = RPT / BR;                       // copy requests per stage
-  static constexpr int KB = FP4 ? 128 : 32;                   // K per lane step (64 bytes of a row)
+  static constexpr int KBLK = FP4 ? 128 : 32;                 // K per 64-byte block of a row
+  // K per lane step: a bf16 step reads 16 B of a row per lane; an NVFP4 step reads 8 B (16 codes,
+  // one E4M3 block), so that a stage has 8 steps and every consumer warp has one
+  static constexpr int KSTEP = FP4 ? 64 : 32;
   static constexpr int KCH = FP4 ? 512 : (NRT == 3 ? 256 : 512);  // K per stage
-  static constexpr int NKB = KCH / KB;                        // 64-byte blocks per row per stage
+  static constexpr int NKB = KCH / KBLK;                      // 64-byte blocks per row per stage
   static constexpr int REQB = 64 * BR * NKB;                  // bytes of one request: [block][row][64 B]
   static constexpr int ROWB = 64 * NKB;                       // weight bytes per row per stage
   static constexpr int SCB = FP4 ? KCH / 16 : 0;              // scale bytes per row per stage
-  static constexpr int STAGES = FP4 ? 12 : 5;  // ring depth (passed as a.stages); swept on B200
+  static constexpr int STAGES = FP4 ? LFM3_WS_STAGES_FP4 : (NRT == 3 ? LFM3_WS_STAGES_CONV : LFM3_WS_STAGES_BF16);
   static constexpr int STAGE_BYTES = RPT * ROWB + RPT * SCB;
   static constexpr int TX_BYTES = STAGE_BYTES;
-  static constexpr int STEPS = KCH / KB;                      // lane steps per stage
+  static constexpr int STEPS = KCH / KSTEP;                   // lane steps per stage
 };
 
-// Byte offset, inside a stage, of the 16 bytes lane chunk t reads from row r at step j.
-template <class G>
+// Byte offset, inside a stage, of what lane chunk t reads from row r at step j: 16 bytes of the
+// j-th 64-byte block (bf16), or 8 bytes of the (j / 2)-th block's half j % 2 (NVFP4).
+template <class G, bool FP4>
 DEVI int ws_woff(int r, int j, int t) {
-  return (r / G::BR) * G::REQB + j * (G::BR * 64) + (r % G::BR) * 64 + t * 16;
+  if constexpr (FP4)
+    return (r / G::BR) * G::REQB + (j >> 1) * (G::BR * 64) + (r % G::BR) * 64 + (j & 1) * 32 + t * 8;
+  else
+    return (r / G::BR) * G::REQB + j * (G::BR * 64) + (r % G::BR) * 64 + t * 16;
 }
 
 // Row of tile `tile`, sub-tile rt, fragment row g (0..15); `which` selects w3 for SwiGLU.
@@ -78,8 +100,6 @@ DEVI int ws_row(int tile, int rt, int g, int& which) {
     return tile * 16 + g;
   }
 }
-
-constexpr int WS_LUT_BYTES = 256 * 32 * 4;
 
 // E2M1 code (bit 3 sign, bits 2..1 exponent with bias 1, bit 0 mantissa) -> bf16 bits, exact:
 // 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives.
@@ -129,7 +149,7 @@ __host__ __device__ inline size_t ws_stage_base(int rows, int Kc, bool fp4) {
 }
 
 template <int EPI, int NT, bool FP4>
-__global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ CUtensorMap tw,
+__global__ void __launch_bounds__(WS_THREADS, 2) k_wstream(const __grid_constant__ CUtensorMap tw,
                                                         const __grid_constant__ CUtensorMap tw3,
                                                         const __grid_constant__ CUtensorMap tsc,
                                                         const __grid_constant__ CUtensorMap tsc3, const WsArgs a) {
@@ -157,6 +177,14 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
   const int ntiles = (EPI == GEMV_SWIGLU) ? a.N / 8 : (EPI == GEMV_CONV ? D / 16 : a.N / 16);
   const uint32_t full0 = su32(bars), empty0 = su32(bars + NS);
 
+#ifdef LFM3_TRACE
+  unsigned long long* const trb = a.trace;
+  const int trid = a.trace_id;
+  if (tid == 0) {
+    TRACE(trb, trid, 0);
+    TRACE(trb, trid, 7);
+  }
+#endif
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full0 + 8 * s, 1);
@@ -182,12 +210,15 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
           mbar_expect_tx(full0 + 8 * s, G::TX_BYTES);
           unsigned char* st = stages + (size_t)s * G::STAGE_BYTES;
           const int k0 = kcta + ch * G::KCH;
+#ifdef LFM3_TRACE
+          if (it == 0) TRACE(trb, trid, 1);
+#endif
 #pragma unroll
           for (int q = 0; q < G::NREQ; ++q) {
             int which;
             const int row = ws_row<EPI>(tile, (q * G::BR) / 16, (q * G::BR) % 16, which);
             const CUtensorMap* m = which ? &tw3 : &tw;
-            ws_tma3(su32(st + q * G::REQB), m, 0, row, k0 / G::KB, full0 + 8 * s);
+            ws_tma3(su32(st + q * G::REQB), m, 0, row, k0 / G::KBLK, full0 + 8 * s);
             if constexpr (FP4)
               ws_tma2(su32(st + G::RPT * G::ROWB + q * G::BR * G::SCB), which ? &tsc3 : &tsc, k0 / 16, row,
                       full0 + 8 * s);
@@ -195,6 +226,9 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
         }
       }
     }
+#ifdef LFM3_TRACE
+    if (lane == 0) TRACE(trb, trid, 6);
+#endif
     pdl_wait();
     pdl_launch_dependents();
     if (!ok) {
@@ -227,6 +261,9 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
   }
   pdl_wait();
   pdl_launch_dependents();
+#ifdef LFM3_TRACE
+  if (ct == 0) TRACE(trb, trid, 2);
+#endif
   if (ct < 8) reinterpret_cast<uint4*>(smem)[ct] = make_uint4(0, 0, 0, 0);
   if constexpr (FP4) {
     for (int i = ct; i < 256 * 32; i += WS_CW * 32) {
@@ -317,6 +354,9 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
   consumers_sync();
 
   // -------------------------------------------------------------- consumers: main loop
+#ifdef LFM3_TRACE
+  if (ct == 0) TRACE(trb, trid, 3);
+#endif
   const int g = lane >> 2, t = lane & 3;
   constexpr int LDR = NT * 8;
   int it = 0;
@@ -338,6 +378,9 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
       if (ok) {
         bool got = true;
         if (lane == 0) got = mbar_wait(full0 + 8 * s, ph, a.err);
+#ifdef LFM3_TRACE
+        if (it == 0 && ct == 0) TRACE(trb, trid, 4);
+#endif
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) {
           ok = false;
@@ -348,12 +391,12 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
         const unsigned char* st = stages + (size_t)s * G::STAGE_BYTES;
 #pragma unroll
         for (int j = warp; j < G::STEPS; j += WS_CW) {
-          const int kx = ch * G::KCH + j * G::KB;  // K offset of this step in the block's range
+          const int kx = ch * G::KCH + j * G::KSTEP;  // K offset of this step in the block's range
 #pragma unroll
           for (int rt = 0; rt < NRT; ++rt) {
-            const uint4 wa = *reinterpret_cast<const uint4*>(st + ws_woff<G>(rt * 16 + g, j, t));
-            const uint4 wb = *reinterpret_cast<const uint4*>(st + ws_woff<G>(rt * 16 + g + 8, j, t));
             if constexpr (!FP4) {
+              const uint4 wa = *reinterpret_cast<const uint4*>(st + ws_woff<G, FP4>(rt * 16 + g, j, t));
+              const uint4 wb = *reinterpret_cast<const uint4*>(st + ws_woff<G, FP4>(rt * 16 + g + 8, j, t));
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
                 const int sr = nt * 8 + g;
@@ -362,27 +405,27 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
                 mma_bf16_16816(acc[rt][nt], wa.z, wb.z, wa.w, wb.w, xv.z, xv.w);
               }
             } else {
-              const unsigned char* sc = st + G::RPT * G::ROWB;  // scales: [request][row][SCB]
-              const uint32_t sa = *reinterpret_cast<const uint16_t*>(sc + (rt * 16 + g) * G::SCB + j * 8 + 2 * t);
-              const uint32_t sb = *reinterpret_cast<const uint16_t*>(sc + (rt * 16 + g + 8) * G::SCB + j * 8 + 2 * t);
-              const uint32_t s0a = ws_e4m3x2(sa & 0xFF), s1a = ws_e4m3x2(sa >> 8);
-              const uint32_t s0b = ws_e4m3x2(sb & 0xFF), s1b = ws_e4m3x2(sb >> 8);
-              const uint32_t wA[4] = {wa.x, wa.y, wa.z, wa.w};
-              const uint32_t wB[4] = {wb.x, wb.y, wb.z, wb.w};
+              // 16 codes of rows g and g + 8: one E4M3 block scale each
+              const uint2 wa = *reinterpret_cast<const uint2*>(st + ws_woff<G, FP4>(rt * 16 + g, j, t));
+              const uint2 wb = *reinterpret_cast<const uint2*>(st + ws_woff<G, FP4>(rt * 16 + g + 8, j, t));
+              const unsigned char* sc = st + G::RPT * G::ROWB;  // scales: [row][SCB]
+              const uint32_t sA = ws_e4m3x2(sc[(rt * 16 + g) * G::SCB + j * 4 + t]);
+              const uint32_t sB = ws_e4m3x2(sc[(rt * 16 + g + 8) * G::SCB + j * 4 + t]);
+              const uint32_t wA[2] = {wa.x, wa.y};
+              const uint32_t wB[2] = {wb.x, wb.y};
               const uint32_t* tab = lut + lane;  // this lane's copy of the table
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
+              for (int q = 0; q < 2; ++q) {
                 uint32_t a01 = tab[(wA[q] & 0xFFu) << 5], a23 = tab[((wA[q] >> 8) & 0xFFu) << 5];
                 uint32_t a45 = tab[((wA[q] >> 16) & 0xFFu) << 5], a67 = tab[(wA[q] >> 24) << 5];
                 uint32_t b01 = tab[(wB[q] & 0xFFu) << 5], b23 = tab[((wB[q] >> 8) & 0xFFu) << 5];
                 uint32_t b45 = tab[((wB[q] >> 16) & 0xFFu) << 5], b67 = tab[(wB[q] >> 24) << 5];
-                const uint32_t sA = q < 2 ? s0a : s1a, sB = q < 2 ? s0b : s1b;
                 a01 = ws_hmul2(a01, sA); a23 = ws_hmul2(a23, sA); a45 = ws_hmul2(a45, sA); a67 = ws_hmul2(a67, sA);
                 b01 = ws_hmul2(b01, sB); b23 = ws_hmul2(b23, sB); b45 = ws_hmul2(b45, sB); b67 = ws_hmul2(b67, sB);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                   const int sr = nt * 8 + g;
-                  const uint4 xv = *reinterpret_cast<const uint4*>(sr < a.rows ? xs + (size_t)sr * XS + kx + 32 * t + 8 * q
+                  const uint4 xv = *reinterpret_cast<const uint4*>(sr < a.rows ? xs + (size_t)sr * XS + kx + 16 * t + 8 * q
                                                                                : xzero);
                   mma_bf16_16816(acc[rt][nt], a01, b01, a23, b23, xv.x, xv.y);
                   mma_bf16_16816(acc[rt][nt], a45, b45, a67, b67, xv.z, xv.w);
@@ -432,21 +475,37 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
     } else if constexpr (EPI == GEMV_CONV) {
       for (int e = ct; e < 16 * a.rows; e += WS_CW * 32) {
         const int cl = e & 15, b = e >> 4, c = tile * 16 + cl;
-        const float Bv = res[cl * LDR + b], Cv = res[(16 + cl) * LDR + b], Xv = res[(32 + cl) * LDR + b];
-        const float bx = round_bf(Bv * Xv);
+        const float Cv = res[(16 + cl) * LDR + b];
         bf16* stt = a.conv_state + (size_t)a.row_slot[b] * CST * D + c;
-        float win[CST];
-#pragma unroll
-        for (int j = 0; j < CST; ++j) win[j] = bf2f(stt[(size_t)j * D]);
         const bf16* w = a.conv_w + (size_t)c * TAPS;
-        float z = 0.f;
+        if (a.win <= 1) {
+          const float bx = round_bf(res[cl * LDR + b] * res[(32 + cl) * LDR + b]);
+          float win[CST];
 #pragma unroll
-        for (int k = 0; k < CST; ++k) z += bf2f(w[k]) * win[k];
-        z += bf2f(w[CST]) * bx;
-        a.y[(size_t)b * D + c] = f2bf(Cv * z);
+          for (int j = 0; j < CST; ++j) win[j] = bf2f(stt[(size_t)j * D]);
+          float z = 0.f;
 #pragma unroll
-        for (int j = 0; j < CST - 1; ++j) stt[(size_t)j * D] = f2bf(win[j + 1]);
-        stt[(size_t)(CST - 1) * D] = f2bf(bx);
+          for (int k = 0; k < CST; ++k) z += bf2f(w[k]) * win[k];
+          z += bf2f(w[CST]) * bx;
+          a.y[(size_t)b * D + c] = f2bf(Cv * z);
+#pragma unroll
+          for (int j = 0; j < CST - 1; ++j) stt[(size_t)j * D] = f2bf(win[j + 1]);
+          stt[(size_t)(CST - 1) * D] = f2bf(bx);
+        } else {
+          // verify window: row wi of its stream sees [state | bx of the window's rows 0..wi]; the
+          // state stays as it is and the state after this row goes to the snapshot
+          const int wi = b % a.win, b0 = b - wi;
+          float wnd[CST + MAX_WIN];
+#pragma unroll
+          for (int j = 0; j < CST; ++j) wnd[j] = bf2f(stt[(size_t)j * D]);
+          for (int i = 0; i <= wi; ++i) wnd[CST + i] = round_bf(res[cl * LDR + b0 + i] * res[(32 + cl) * LDR + b0 + i]);
+          float z = 0.f;
+#pragma unroll
+          for (int k = 0; k < TAPS; ++k) z += bf2f(w[k]) * wnd[wi + k];
+          a.y[(size_t)b * D + c] = f2bf(Cv * z);
+#pragma unroll
+          for (int j = 0; j < CST; ++j) a.conv_snap[((size_t)b * CST + j) * D + c] = f2bf(wnd[wi + 1 + j]);
+        }
       }
     } else if constexpr (EPI == GEMV_HEAD) {
       for (int b = warp; b < a.rows; b += WS_CW) {
@@ -465,6 +524,9 @@ __global__ void __launch_bounds__(WS_THREADS) k_wstream(const __grid_constant__ 
     }
     consumers_sync();
   }
+#ifdef LFM3_TRACE
+  if (ct == 0) TRACE(trb, trid, 5);
+#endif
 }
 
 template <int EPI, bool FP4>
@@ -476,7 +538,28 @@ size_t ws_smem(int NT, int rows, int Kc, int stages) {
 }
 
 static int g_num_sms = 0;
-constexpr int WS_BPS = 2;  // blocks per SM
+constexpr int WS_BPS = LFM3_WS_BPS;  // blocks per SM, at most
+
+// Blocks of `kern` that fit on one SM with `smem` bytes of dynamic shared memory (at most WS_BPS):
+// the grid is one wave of them, so no block waits for a second wave.
+template <typename K>
+static int ws_fit(K kern, size_t smem) {
+  struct Entry { const void* k; size_t smem; int n; };
+  static Entry cache[64];
+  static int used = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].k == reinterpret_cast<const void*>(kern) && cache[i].smem == smem) return cache[i].n;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, WS_THREADS, smem) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    n = 1;
+  }
+  n = std::min(n, WS_BPS);
+  if (used < 64) cache[used++] = Entry{reinterpret_cast<const void*>(kern), smem, n};
+  return n;
+}
 
 template <int EPI, bool FP4>
 static cudaError_t launch_ws(const WsMaps& mp, const WsArgs& a, cudaStream_t s) {
@@ -487,16 +570,21 @@ static cudaError_t launch_ws(const WsMaps& mp, const WsArgs& a, cudaStream_t s) 
   const int NT = a.rows <= 8 ? 1 : 2;
   WsArgs b = a;
   b.stages = G::STAGES;
+#ifdef LFM3_TRACE
+  b.trace = g_trace;
+  b.trace_id = g_launches;
+#endif
   const size_t smem = ws_smem<EPI, FP4>(NT, a.rows, Kc, b.stages);
   if (smem > (size_t)WS_SMEM_MAX) return cudaErrorInvalidValue;
-  // blocks per K range: WS_BPS blocks per SM in all, spread evenly over the tiles
-  int gx = std::max(1, WS_BPS * g_num_sms / a.splits);
+  // blocks per K range: as many blocks as fit on the SMs at once (one wave), spread evenly
+  // over the tiles
+  auto kern = NT == 1 ? k_wstream<EPI, 1, FP4> : k_wstream<EPI, 2, FP4>;
+  int gx = std::max(1, ws_fit(kern, smem) * g_num_sms / a.splits);
   gx = std::min(gx, ntiles);
   const int per = (ntiles + gx - 1) / gx;
   gx = (ntiles + per - 1) / per;
   dim3 grid(gx, a.splits);
-  if (NT == 1) return launch(k_wstream<EPI, 1, FP4>, grid, dim3(WS_THREADS), smem, s, mp.w, mp.w3, mp.s, mp.s3, b);
-  return launch(k_wstream<EPI, 2, FP4>, grid, dim3(WS_THREADS), smem, s, mp.w, mp.w3, mp.s, mp.s3, b);
+  return launch(kern, grid, dim3(WS_THREADS), smem, s, mp.w, mp.w3, mp.s, mp.s3, b);
 }
 
 cudaError_t wstream(int epi, int nvfp4, const WsMaps& mp, const WsArgs& a, cudaStream_t s) {

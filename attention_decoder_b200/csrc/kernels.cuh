@@ -24,6 +24,9 @@ constexpr int GQA = HQ / HKV;
 
 // Launch counter of the calling thread (reset by the API at each call).
 extern thread_local int g_launches;
+#ifdef LFM3_TRACE
+extern unsigned long long* g_trace;  // timeline buffer of the diagnostic build (lfm3_trace_set)
+#endif
 
 // Every kernel is launched with programmatic stream serialisation (see pdl_wait()).
 template <typename... KArgs, typename... Args>
@@ -51,15 +54,18 @@ struct Rows {
 };
 
 // ---------------------------------------------------------------- elementwise / small kernels
-cudaError_t setup_rows(int prefill, int slot, const int32_t* d_slots, const int32_t* seq_len, int rows,
+// decode: `win` consecutive rows per listed slot (1, or a verify window) at seq_len[slot] + r % win
+cudaError_t setup_rows(int prefill, int slot, const int32_t* d_slots, const int32_t* seq_len, int rows, int win,
                        int32_t* row_slot, int32_t* row_pos, unsigned long long* amax, cudaStream_t s);
 cudaError_t embed_rows(const int32_t* tokens, const bf16* table, const bf16* vecs, int rows, float* x_res,
                        float* dump, cudaStream_t s);
 // x_res[r] += g_post * RMS(sum_s part[s][r]) (if n_part > 0); dump x_res; xn = g_next * RMS(x_res)
 cudaError_t resid_norm(float* x_res, const float* part, int n_part, long part_stride, const bf16* g_post,
                        const bf16* g_next, bf16* xn, int rows, float eps, float* dump, cudaStream_t s);
+// one row per stream (win 1: the state shifts), or verify windows of `win` rows per stream (the
+// state is left alone; the state after each row goes to snap [rows][CST][D])
 cudaError_t conv_decode(const float* bcx, const bf16* conv_w, bf16* state_layer, const int32_t* row_slot,
-                        int rows, bf16* y, cudaStream_t s);
+                        int rows, int win, bf16* snap, bf16* y, cudaStream_t s);
 // n rows; the new state is columns [n_state, n_state + 6) of [state | bx] (n_state <= n)
 cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot, int n, int n_state, bf16* y,
                          cudaStream_t s);
@@ -81,8 +87,20 @@ cudaError_t ring_to_scratch(const bf16* ring_k, const bf16* ring_v, int slot, in
                             bf16* sk, bf16* sv, int scratch_rows, cudaStream_t s);
 cudaError_t scratch_to_ring(const bf16* sk, const bf16* sv, int scratch_rows, int n, int p0, bf16* ring_k,
                             bf16* ring_v, int slot, int max_streams, cudaStream_t s);
+// advance = 0 leaves seq_len alone (a verify window)
 cudaError_t finish_step(int32_t* seq_len, const int32_t* row_slot, int rows, int add_prefill, int prefill_slot,
-                        const unsigned long long* amax, int32_t* argmax_out, cudaStream_t s);
+                        const unsigned long long* amax, int32_t* argmax_out, int advance, cudaStream_t s);
+
+// Commit of verify windows: per stream, the first k of its W rows become state.
+struct CommitArgs {
+  int n, W, n_conv, n_sliding, max_streams, max_batch;
+  int slot[64], pos[64], k[64];      // slot, position of the window's first row, rows accepted
+  const bf16* snap;                  // [n_conv][max_batch][CST][D]
+  const bf16* side_k; const bf16* side_v;  // [n_sliding][max_batch][HKV][HD]
+  bf16* conv; bf16* ring_k; bf16* ring_v;
+  int32_t* seq_len;
+};
+cudaError_t commit_windows(const CommitArgs& a, cudaStream_t s);
 // One bounded wait that can never complete (at most `rounds` polls), then the status word is set.
 cudaError_t wait_selftest(int* err, unsigned rounds, cudaStream_t s);
 
@@ -118,9 +136,14 @@ struct WsArgs {
   float* part_out;                                 // PARTIAL: [splits][rows][N]
   bf16* out;                                       // SWIGLU: [rows][N]
   const bf16* conv_w; bf16* conv_state; const int32_t* row_slot; bf16* y;  // CONV
+  int win; bf16* conv_snap;                        // CONV in a verify window (win > 1), see conv_decode
   unsigned long long* amax; float* logits;         // HEAD (logits may be null)
   int* err;
   int stages;                                      // set by the launcher
+#ifdef LFM3_TRACE
+  unsigned long long* trace;
+  int trace_id;
+#endif
 };
 struct WsMaps {
   CUtensorMap w, w3, s, s3;  // weights (SwiGLU: w1, w3) or NVFP4 codes; NVFP4 scales
@@ -134,6 +157,7 @@ cudaError_t wstream_init();
 
 // ---------------------------------------------------------------- attention
 constexpr int DEC_KEYS = 64;  // keys per decode split: one 64-position page, or a quarter of the ring
+constexpr int MAX_WIN = 8;    // rows per stream in one verify window
 struct AttnLayer {
   int full;               // 1 full (pages), 0 sliding
   const bf16* k; const bf16* v;   // pages: this layer's pool; ring: this layer's ring base
@@ -149,6 +173,15 @@ struct AttnDecodeArgs {
   float eps;
   unsigned* counters;      // [streams][HKV], zero between calls
   int* err;                // status word (a bounded wait that gave up)
+  // verify windows: rows come in groups of `win` consecutive positions of one stream (1 when
+  // decoding); a sliding layer's window rows go to side_k / side_v [rows][HKV][HD], not the ring
+  int win;
+  bf16* side_k;
+  bf16* side_v;
+#ifdef LFM3_TRACE
+  unsigned long long* trace;
+  int trace_id;
+#endif
 };
 // Split slots a decode step reserves per (stream, head) in the partials buffer: the smallest
 // power of two >= the splits of the longest context (and >= the ring's WIN / DEC_KEYS).

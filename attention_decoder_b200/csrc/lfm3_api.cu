@@ -66,6 +66,12 @@ struct lfm3_ctx {
   CUtensorMap tm_q, tm_sk, tm_sv;  // prefill attention: q rows, sliding scratch K / V
   WsMaps ws_head;                  // decode: tied head
   unsigned* attn_cnt = nullptr;    // workspace: decode attention split counts [max_batch][n_kv]
+  bf16* conv_snap = nullptr;       // workspace: verify windows' conv states [n_conv][max_batch][6][D]
+  bf16* side_k = nullptr;          // workspace: verify windows' sliding keys [n_sliding][max_batch][n_kv][hd]
+  bf16* side_v = nullptr;
+  // the last verify window, which lfm3_commit applies
+  int vw_n = 0, vw_W = 0;
+  std::vector<int> vw_slots, vw_pos;
   std::string msg;
   int launches = 0;
   // decode-step CUDA graphs, keyed by batch, split count and every device pointer the step reads
@@ -139,6 +145,9 @@ size_t layout(lfm3_ctx* c, char* base) {
   }
   c->deq = g.ffn_format == LFM3_FFN_NVFP4 ? reinterpret_cast<bf16*>(take(2 * (size_t)2 * F * D)) : nullptr;
   c->attn_cnt = reinterpret_cast<unsigned*>(take(4 * (size_t)g.max_batch * HKV));
+  c->conv_snap = reinterpret_cast<bf16*>(take(2 * (size_t)c->n_conv * g.max_batch * CST * D));
+  c->side_k = reinterpret_cast<bf16*>(take(2 * (size_t)c->n_sliding * g.max_batch * HKV * HD));
+  c->side_v = reinterpret_cast<bf16*>(take(2 * (size_t)c->n_sliding * g.max_batch * HKV * HD));
   return align_up(off, 256);
 }
 
@@ -532,7 +541,7 @@ lfm3_status prefill_rows(lfm3_ctx* ctx, const lfm3_state* st, int slot, const in
     const int p0 = (int)p_start + c0;
     const bool last = c0 + nc == n;
     const int nr = last ? nc - n_pad : nc;  // real rows of this chunk
-    CK(setup_rows(1, slot, nullptr, st->seq_len, nc, ctx->row_slot, ctx->row_pos, ctx->amax, s));
+    CK(setup_rows(1, slot, nullptr, st->seq_len, nc, 1, ctx->row_slot, ctx->row_pos, ctx->amax, s));
     const Rows rows{ctx->row_slot, ctx->row_pos, nr};
     CK(embed_rows(d_tokens ? d_tokens + c0 : nullptr, ctx->embed,
                   d_embeds ? B(d_embeds) + (size_t)c0 * D : nullptr, nc, ctx->x_res,
@@ -607,7 +616,8 @@ lfm3_status prefill_rows(lfm3_ctx* ctx, const lfm3_state* st, int slot, const in
       a.err = ctx->err;
       CK(run_ws(ctx, GEMV_HEAD, 0, ctx->ws_head, a, s));
     }
-    CK(finish_step(st->seq_len, ctx->row_slot, nc, nr, slot, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
+    CK(finish_step(st->seq_len, ctx->row_slot, nc, nr, slot, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, 1,
+                   s));
   }
   st->h_seq_len[slot] += n_real;
   ctx->launches = g_launches;
@@ -637,13 +647,33 @@ extern "C" lfm3_status lfm3_prefill_padded(lfm3_ctx* ctx, const lfm3_state* st, 
 namespace {
 
 // Every launch of one decode step, in order, on stream s.
-lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* d_slots,
+AttnDecodeArgs attn_args(lfm3_ctx* ctx, int l, int win) {
+  const lfm3_layer_weights& W = ctx->L[l];
+  const int k = ctx->cfg.layer_type[l] == LFM3_LAYER_FULL ? 0 : 1;
+  AttnDecodeArgs A{};
+  A.q_norm = B(W.q_norm);
+  A.k_norm = B(W.k_norm);
+  A.rope_cos = ctx->rope_cos[k];
+  A.rope_sin = ctx->rope_sin[k];
+  A.eps = ctx->cfg.eps;
+  A.counters = ctx->attn_cnt;
+  A.err = ctx->err;
+  A.win = win;
+  if (k == 1) {
+    const size_t per = (size_t)ctx->cfg.max_batch * HKV * HD;
+    A.side_k = ctx->side_k + (size_t)ctx->kidx[l] * per;
+    A.side_v = ctx->side_v + (size_t)ctx->kidx[l] * per;
+  }
+  return A;
+}
+
+// win > 1: nb rows are verify windows of win rows per stream (nothing committed, see lfm3_verify).
+lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, int win, const int32_t* d_slots,
                            const int32_t* d_tokens, const void* d_embeds, float* d_logits, int32_t* d_argmax,
                            float* d_hidden, int splits_full, float* attn_part, cudaStream_t s) {
   const lfm3_config& g = ctx->cfg;
   const float eps = g.eps;
-  const bool fp4 = g.ffn_format == LFM3_FFN_NVFP4;
-  CK(setup_rows(0, 0, d_slots, st->seq_len, nb, ctx->row_slot, ctx->row_pos, ctx->amax, s));
+  CK(setup_rows(0, 0, d_slots, st->seq_len, nb, win, ctx->row_slot, ctx->row_pos, ctx->amax, s));
   const Rows rows{ctx->row_slot, ctx->row_pos, nb};
   CK(embed_rows(d_tokens, ctx->embed, B(d_embeds), nb, ctx->x_res, d_hidden, s));
   CK(resid_norm(ctx->x_res, nullptr, 0, 0, nullptr, B(ctx->L[0].op_norm), ctx->xn, nb, eps, nullptr, s));
@@ -653,13 +683,13 @@ lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, co
     const Views v = views(ctx, st, l);
     if (g.layer_type[l] == LFM3_LAYER_CONV) {
       CK(run_gemm(ctx, P.in_proj, nb, s));
-      CK(conv_decode(ctx->part, B(W.conv), v.conv_layer, ctx->row_slot, nb, ctx->y, s));
+      CK(conv_decode(ctx->part, B(W.conv), v.conv_layer, ctx->row_slot, nb, win,
+                     ctx->conv_snap + (size_t)ctx->kidx[l] * g.max_batch * CST * D, ctx->y, s));
       CK(run_gemm(ctx, P.out_proj, nb, s));
     } else {
       const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
       CK(run_gemm(ctx, P.qkvg, nb, s));
-      const int k = full ? 0 : 1;
-      AttnDecodeArgs A{B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], eps, ctx->attn_cnt, ctx->err};
+      AttnDecodeArgs A = attn_args(ctx, l, win);
       CK(attn_decode_fused(ctx->part, rows, attn_layer(ctx, st, l, v), A, full ? splits_full : WIN / DEC_KEYS,
                            attn_part, ctx->y, s));
       CK(run_gemm(ctx, P.o_proj, nb, s));
@@ -688,19 +718,20 @@ lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, co
       CK(run_ws(ctx, GEMV_HEAD, 0, ctx->ws_head, a, s));
     }
   }
-  CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
+  CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr,
+                 win == 1, s));
   return LFM3_OK;
 }
 
 // Decode for up to 16 streams: the weight-streaming kernel, whose prologue also applies the
 // previous projection's residual add + post-norm and this projection's input norm.
-lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* d_slots,
+lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, int win, const int32_t* d_slots,
                                   const int32_t* d_tokens, const void* d_embeds, float* d_logits, int32_t* d_argmax,
                                   float* d_hidden, int splits_full, float* attn_part, cudaStream_t s) {
   const lfm3_config& g = ctx->cfg;
   const float eps = g.eps;
   const bool fp4 = g.ffn_format == LFM3_FFN_NVFP4;
-  CK(setup_rows(0, 0, d_slots, st->seq_len, nb, ctx->row_slot, ctx->row_pos, ctx->amax, s));
+  CK(setup_rows(0, 0, d_slots, st->seq_len, nb, win, ctx->row_slot, ctx->row_pos, ctx->amax, s));
   const Rows rows{ctx->row_slot, ctx->row_pos, nb};
   CK(embed_rows(d_tokens, ctx->embed, B(d_embeds), nb, ctx->x_res, d_hidden, s));
   float* cur = ctx->x_res;
@@ -741,6 +772,8 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       c.conv_state = v.conv_layer;
       c.row_slot = ctx->row_slot;
       c.y = ctx->y;
+      c.win = win;
+      c.conv_snap = ctx->conv_snap + (size_t)ctx->kidx[l] * g.max_batch * CST * D;
       norm_in(c, B(W.op_norm), dump_l);
       CK(run_ws(ctx, GEMV_CONV, 0, ctx->plans[l].ws_in, c, s));
       advance();
@@ -760,8 +793,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
       norm_in(q, B(W.op_norm), dump_l);
       CK(run_ws(ctx, GEMV_PARTIAL, 0, ctx->plans[l].ws_qkvg, q, s));
       advance();
-      const int k = full ? 0 : 1;
-      AttnDecodeArgs A{B(W.q_norm), B(W.k_norm), ctx->rope_cos[k], ctx->rope_sin[k], eps, ctx->attn_cnt, ctx->err};
+      AttnDecodeArgs A = attn_args(ctx, l, win);
       CK(attn_decode_fused(ctx->part3, rows, attn_layer(ctx, st, l, v), A, full ? splits_full : WIN / DEC_KEYS,
                            attn_part, ctx->y, s));
       WsArgs o{};
@@ -817,17 +849,18 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, c
   } else if (dump_last) {
     CK(resid_norm(cur, pend, pend_n, (long)nb * D, pend_g, nullptr, nullptr, nb, eps, dump_last, s));
   }
-  CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, s));
+  CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr,
+                 win == 1, s));
   return LFM3_OK;
 }
 
-lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* d_slots,
+lfm3_status enqueue_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, int win, const int32_t* d_slots,
                            const int32_t* d_tokens, const void* d_embeds, float* d_logits, int32_t* d_argmax,
                            float* d_hidden, int splits_full, float* attn_part, cudaStream_t s) {
   if (nb <= GEMV_MAX_ROWS)
-    return enqueue_decode_stream(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+    return enqueue_decode_stream(ctx, st, nb, win, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
                                  splits_full, attn_part, s);
-  return enqueue_decode_large(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden, splits_full,
+  return enqueue_decode_large(ctx, st, nb, win, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden, splits_full,
                               attn_part, s);
 }
 
@@ -865,6 +898,57 @@ lfm3_status validate_decode(lfm3_ctx* ctx, const lfm3_state* st, int nb, const i
 
 }  // namespace
 
+namespace {
+
+// Enqueues nr rows (win per stream) on stream s, from the step's captured graph when graphs are on.
+lfm3_status run_decode(lfm3_ctx* ctx, const lfm3_state* st, int nr, int win, int splits_full, const int32_t* d_slots,
+                       const int32_t* d_tokens, const void* d_embeds, float* d_logits, int32_t* d_argmax,
+                       float* d_hidden, cudaStream_t s) {
+  g_launches = 0;
+  if (!ctx->graphs_on || ctx->prof) {
+    lfm3_status es = enqueue_decode(ctx, st, nr, win, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                                    splits_full, ctx->attn_part, s);
+    if (es != LFM3_OK) return es;
+    ctx->launches = g_launches;
+    return LFM3_OK;
+  }
+  std::vector<const void*> key = {reinterpret_cast<const void*>((intptr_t)nr), reinterpret_cast<const void*>((intptr_t)win),
+                                  reinterpret_cast<const void*>((intptr_t)splits_full), d_slots, d_tokens, d_embeds,
+                                  d_logits, d_argmax, d_hidden, st->conv_state, st->ring_k, st->ring_v, st->kv_k,
+                                  st->kv_v, st->page_table, st->seq_len};
+  lfm3_ctx::GraphEntry* hit = nullptr;
+  for (auto& e : ctx->graphs)
+    if (e.key == key) hit = &e;
+  if (!hit) {
+    if (!ctx->cap_stream) CK(cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking));
+    if (ctx->graphs.size() >= 32) {
+      for (auto& e : ctx->graphs) cudaGraphExecDestroy(e.exec);
+      ctx->graphs.clear();
+    }
+    cudaGraph_t graph = nullptr;
+    CK(cudaStreamBeginCapture(ctx->cap_stream, cudaStreamCaptureModeThreadLocal));
+    lfm3_status es = enqueue_decode(ctx, st, nr, win, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                                    splits_full, ctx->attn_part, ctx->cap_stream);
+    cudaError_t ce = cudaStreamEndCapture(ctx->cap_stream, &graph);
+    if (es != LFM3_OK) {
+      if (graph) cudaGraphDestroy(graph);
+      return es;
+    }
+    CK(ce);
+    cudaGraphExec_t exec = nullptr;
+    ce = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    CK(ce);
+    ctx->graphs.push_back({key, exec, g_launches});
+    hit = &ctx->graphs.back();
+  }
+  CK(cudaGraphLaunch(hit->exec, s));
+  ctx->launches = hit->launches;
+  return LFM3_OK;
+}
+
+}  // namespace
+
 extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int nb, const int32_t* h_slots,
                                         const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
                                         float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream) {
@@ -873,48 +957,84 @@ extern "C" lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int
   lfm3_status vs = validate_decode(ctx, st, nb, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax,
                                    &splits_full);
   if (vs != LFM3_OK) return vs;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  g_launches = 0;
-  if (!ctx->graphs_on || ctx->prof) {
-    lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
-                                    splits_full, ctx->attn_part, s);
-    if (es != LFM3_OK) return es;
-    ctx->launches = g_launches;
-  } else {
-    std::vector<const void*> key = {reinterpret_cast<const void*>((intptr_t)nb),
-                                    reinterpret_cast<const void*>((intptr_t)splits_full), d_slots, d_tokens, d_embeds,
-                                    d_logits, d_argmax, d_hidden, st->conv_state, st->ring_k, st->ring_v, st->kv_k,
-                                    st->kv_v, st->page_table, st->seq_len};
-    lfm3_ctx::GraphEntry* hit = nullptr;
-    for (auto& e : ctx->graphs)
-      if (e.key == key) hit = &e;
-    if (!hit) {
-      if (!ctx->cap_stream) CK(cudaStreamCreateWithFlags(&ctx->cap_stream, cudaStreamNonBlocking));
-      if (ctx->graphs.size() >= 32) {
-        for (auto& e : ctx->graphs) cudaGraphExecDestroy(e.exec);
-        ctx->graphs.clear();
-      }
-      cudaGraph_t graph = nullptr;
-      CK(cudaStreamBeginCapture(ctx->cap_stream, cudaStreamCaptureModeThreadLocal));
-      lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
-                                      splits_full, ctx->attn_part, ctx->cap_stream);
-      cudaError_t ce = cudaStreamEndCapture(ctx->cap_stream, &graph);
-      if (es != LFM3_OK) {
-        if (graph) cudaGraphDestroy(graph);
-        return es;
-      }
-      CK(ce);
-      cudaGraphExec_t exec = nullptr;
-      ce = cudaGraphInstantiate(&exec, graph, 0);
-      cudaGraphDestroy(graph);
-      CK(ce);
-      ctx->graphs.push_back({key, exec, g_launches});
-      hit = &ctx->graphs.back();
-    }
-    CK(cudaGraphLaunch(hit->exec, s));
-    ctx->launches = hit->launches;
-  }
+  vs = run_decode(ctx, st, nb, 1, splits_full, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                  reinterpret_cast<cudaStream_t>(stream));
+  if (vs != LFM3_OK) return vs;
+  ctx->vw_n = 0;  // a decode step ends any verify window
   for (int b = 0; b < nb; ++b) st->h_seq_len[h_slots[b]] += 1;
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_verify(lfm3_ctx* ctx, const lfm3_state* st, int n_streams, const int32_t* h_slots,
+                                   const int32_t* d_slots, int W, const int32_t* d_tokens, const void* d_embeds,
+                                   float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  if (W < 1 || W > MAX_WIN) return fail(ctx, LFM3_E_ARG, "window of %d rows outside 1..%d", W, MAX_WIN);
+  if (n_streams < 1 || (long)n_streams * W > ctx->cfg.max_batch)
+    return fail(ctx, LFM3_E_ARG, "%d streams x %d rows outside 1..max_batch (%d)", n_streams, W, ctx->cfg.max_batch);
+  int splits_full = 1;
+  // the row checks of a decode step, per stream; then room for the window's last row
+  lfm3_status vs = validate_decode(ctx, st, n_streams, h_slots, d_slots, d_tokens, d_embeds, d_logits, d_argmax,
+                                   &splits_full);
+  if (vs != LFM3_OK) return vs;
+  int maxpos = 0;
+  for (int i = 0; i < n_streams; ++i) {
+    vs = check_pages(ctx, st, h_slots[i], (long)st->h_seq_len[h_slots[i]] + W);
+    if (vs != LFM3_OK) return vs;
+    maxpos = std::max(maxpos, (int)st->h_seq_len[h_slots[i]] + W - 1);
+  }
+  splits_full = std::min(attn_decode_splits(maxpos + 1), ctx->max_splits);
+  vs = run_decode(ctx, st, n_streams * W, W, splits_full, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+                  reinterpret_cast<cudaStream_t>(stream));
+  if (vs != LFM3_OK) return vs;
+  ctx->vw_n = n_streams;
+  ctx->vw_W = W;
+  ctx->vw_slots.assign(h_slots, h_slots + n_streams);
+  ctx->vw_pos.resize(n_streams);
+  for (int i = 0; i < n_streams; ++i) ctx->vw_pos[i] = st->h_seq_len[h_slots[i]];
+  return LFM3_OK;
+}
+
+extern "C" lfm3_status lfm3_commit(lfm3_ctx* ctx, const lfm3_state* st, int n_streams, const int32_t* h_slots,
+                                   const int32_t* h_accept, void* stream) {
+  if (!ctx) return LFM3_E_ARG;
+  if (!ctx->bound) return fail(ctx, LFM3_E_STATE, "workspace not bound");
+  lfm3_status vs = check_state(ctx, st);
+  if (vs != LFM3_OK) return vs;
+  if (!h_slots || !h_accept) return fail(ctx, LFM3_E_ARG, "h_slots / h_accept is NULL");
+  if (ctx->vw_n == 0) return fail(ctx, LFM3_E_STATE, "no verify window to commit");
+  if (n_streams != ctx->vw_n) return fail(ctx, LFM3_E_ARG, "%d streams, the window had %d", n_streams, ctx->vw_n);
+  CommitArgs a{};
+  a.n = n_streams;
+  a.W = ctx->vw_W;
+  for (int i = 0; i < n_streams; ++i) {
+    if (h_slots[i] != ctx->vw_slots[i])
+      return fail(ctx, LFM3_E_ARG, "stream %d is slot %d, the window's was slot %d", i, h_slots[i], ctx->vw_slots[i]);
+    if (st->h_seq_len[h_slots[i]] != ctx->vw_pos[i])
+      return fail(ctx, LFM3_E_STATE, "slot %d moved since its verify window", h_slots[i]);
+    if (h_accept[i] < 1 || h_accept[i] > a.W)
+      return fail(ctx, LFM3_E_ARG, "slot %d: %d rows accepted, outside 1..%d", h_slots[i], h_accept[i], a.W);
+    a.slot[i] = h_slots[i];
+    a.pos[i] = ctx->vw_pos[i];
+    a.k[i] = h_accept[i];
+  }
+  const lfm3_config& g = ctx->cfg;
+  a.n_conv = ctx->n_conv;
+  a.n_sliding = ctx->n_sliding;
+  a.max_streams = g.max_streams;
+  a.max_batch = g.max_batch;
+  a.snap = ctx->conv_snap;
+  a.side_k = ctx->side_k;
+  a.side_v = ctx->side_v;
+  a.conv = reinterpret_cast<bf16*>(st->conv_state);
+  a.ring_k = reinterpret_cast<bf16*>(st->ring_k);
+  a.ring_v = reinterpret_cast<bf16*>(st->ring_v);
+  a.seq_len = st->seq_len;
+  g_launches = 0;
+  CK(commit_windows(a, reinterpret_cast<cudaStream_t>(stream)));
+  ctx->launches = g_launches;
+  for (int i = 0; i < n_streams; ++i) st->h_seq_len[h_slots[i]] += h_accept[i];
+  ctx->vw_n = 0;
   return LFM3_OK;
 }
 
@@ -941,10 +1061,11 @@ extern "C" lfm3_status lfm3_decode_step_noalloc(lfm3_ctx* ctx, const lfm3_state*
                 nb, splits_full, need * sizeof(float), cap * sizeof(float));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   g_launches = 0;
-  lfm3_status es = enqueue_decode(ctx, st, nb, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
+  lfm3_status es = enqueue_decode(ctx, st, nb, 1, d_slots, d_tokens, d_embeds, d_logits, d_argmax, d_hidden,
                                   splits_full, scratch, s);
   if (es != LFM3_OK) return es;
   ctx->launches = g_launches;
+  ctx->vw_n = 0;
   for (int b = 0; b < nb; ++b) st->h_seq_len[h_slots[b]] += 1;
   return LFM3_OK;
 }
@@ -1085,6 +1206,11 @@ extern "C" lfm3_status lfm3_profile_read(lfm3_ctx* ctx, int* launches, double* m
   if (over) return fail(ctx, LFM3_E_CAPACITY, "%d launches ran unbracketed (capacity exceeded)", over);
   return LFM3_OK;
 }
+
+#ifdef LFM3_TRACE
+// Diagnostic builds only: the device buffer [256 launches][512 blocks][8] uint64 the kernels stamp.
+extern "C" void lfm3_trace_set(void* d_buf) { g_trace = static_cast<unsigned long long*>(d_buf); }
+#endif
 
 extern "C" int lfm3_last_launch_count(const lfm3_ctx* ctx) { return ctx ? ctx->launches : 0; }
 

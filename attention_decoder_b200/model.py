@@ -202,6 +202,31 @@ class Lfm3Model:
                                  _ptr(out.get("argmax")), _ptr(out.get("hidden")), _stream(stream)), self.ctx)
         return out
 
+    def verify(self, st, slots, W, tokens=None, embeds=None, hidden=False, stream=None):
+        """One verify window of W rows per listed slot (see lfm3_verify); nothing is committed.
+        tokens: device int32 [len(slots) * W], stream-major. Returns logits [n*W, V], argmax [n*W]."""
+        g = self.geom
+        h_slots = np.ascontiguousarray(slots, dtype=np.int32)
+        rows = len(h_slots) * W
+        d_slots = torch.from_numpy(h_slots).to(self.device)
+        out = {}
+        if g.has_head:
+            out["logits"] = torch.empty(rows, g.vocab, dtype=torch.float32, device=self.device)
+            out["argmax"] = torch.empty(rows, dtype=torch.int32, device=self.device)
+        if hidden:
+            out["hidden"] = torch.empty(g.n_layers + 1, rows, g.d_model, dtype=torch.float32, device=self.device)
+        out["_slots"] = d_slots  # kept alive until the window has run
+        check(L.lfm3_verify(self.ctx, C.byref(st.struct), len(h_slots), h_slots.ctypes.data_as(C.POINTER(C.c_int32)),
+                            _ptr(d_slots), W, _ptr(tokens), _ptr(embeds), _ptr(out.get("logits")),
+                            _ptr(out.get("argmax")), _ptr(out.get("hidden")), _stream(stream)), self.ctx)
+        return out
+
+    def commit(self, st, slots, accept, stream=None):
+        h_slots = np.ascontiguousarray(slots, dtype=np.int32)
+        h_acc = np.ascontiguousarray(accept, dtype=np.int32)
+        check(L.lfm3_commit(self.ctx, C.byref(st.struct), len(h_slots), h_slots.ctypes.data_as(C.POINTER(C.c_int32)),
+                            h_acc.ctypes.data_as(C.POINTER(C.c_int32)), _stream(stream)), self.ctx)
+
     def close(self):
         if getattr(self, "ctx", None):
             L.lfm3_free(self.ctx)

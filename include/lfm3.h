@@ -217,6 +217,34 @@ lfm3_status lfm3_decode_step(lfm3_ctx* ctx, const lfm3_state* st, int n_streams,
                              const int32_t* d_slots, const int32_t* d_tokens, const void* d_embeds,
                              float* d_logits, int32_t* d_argmax, float* d_hidden, void* stream);
 
+/* Drafted windows (TensorFold PR #1508, lfm2_moe.cu paragraph: "the short conv over each stream's
+ * state with every window row's snapshot, the commit of an accepted row's conv state"; its check
+ * is "drafted == plain"). lfm3_verify runs, for each listed slot, W rows (1..8: the stream's next
+ * token and W - 1 drafted ones) at positions seq_len[slot] .. + W - 1 in one pass and returns every
+ * row's logits and greedy id; it commits nothing. The full layers' keys and values of the window
+ * are written to the slot's pages past its cursor (where a later row overwrites them), the
+ * sliding layers' go to the workspace, and so does the conv state after every window row.
+ * lfm3_commit then makes the first accept[i] rows (1..W) of stream i the slot's state: the conv
+ * state after row accept[i] - 1, those rows' keys and values in the rings, and seq_len advanced by
+ * accept[i]. The result equals plain decode of the accepted tokens.
+ *   d_tokens  device int32 [n_streams][W] (row i*W + j is stream i's j-th row), or NULL
+ *   d_embeds  device bf16 [n_streams * W][d_model] (has_head == 0), or NULL
+ *   d_logits  device fp32 [n_streams * W][vocab] or NULL;  d_argmax  device int32 [n_streams * W]
+ *   d_hidden  device fp32 [n_layers+1][n_streams * W][d_model] or NULL
+ * Errors (nothing enqueued): those of lfm3_decode_step for the listed slots; LFM3_E_ARG if W is
+ * outside 1..8 or n_streams * W > max_batch; LFM3_E_CAPACITY if a slot's pages cannot hold the
+ * window. Only the last window can be committed, and only before any other call touches its
+ * slots: lfm3_commit refuses with LFM3_E_STATE otherwise (a decode step or another window ends
+ * it), and with LFM3_E_ARG for slots that differ from the window's or accept counts out of range. */
+lfm3_status lfm3_verify(lfm3_ctx* ctx, const lfm3_state* st, int n_streams, const int32_t* h_slots,
+                        const int32_t* d_slots, int W, const int32_t* d_tokens, const void* d_embeds, float* d_logits,
+                        int32_t* d_argmax, float* d_hidden, void* stream);
+
+/* Commits the last verify window (see lfm3_verify). h_slots: the window's slots, in its order;
+ * h_accept: HOST int32 [n_streams], rows accepted per stream (1..W). */
+lfm3_status lfm3_commit(lfm3_ctx* ctx, const lfm3_state* st, int n_streams, const int32_t* h_slots,
+                        const int32_t* h_accept, void* stream);
+
 /* The same decode step as lfm3_decode_step, for callers that cannot allocate device memory at
  * the point of the call - a host program that hands this library a finished arena and forbids
  * later allocation, or code running where an allocation would synchronise the device. The

@@ -55,8 +55,8 @@ def test_padded_chunk_equals_the_unpadded_rows(lib, n_real, n_rows):
     assert hb.shape[1] == n_rows
     assert torch.equal(ha, hb[:, :n_real])
     assert b.h_seq_len.tolist() == [n] and b.seq_len.cpu().tolist() == [n]
-    for t in ("conv", "ring_k", "ring_v"):
-        assert torch.equal(getattr(a, t), getattr(b, t)), t
+    for t in ("conv", "ring_k", "ring_v"):  # bitwise: slots the prompt has not reached still hold NaN poison
+        assert torch.equal(getattr(a, t).view(torch.int16), getattr(b, t).view(torch.int16)), t
     for t in range(n, n + 3):  # later steps read the committed state
         da = m.decode(a, [0], embeds=xd[t:t + 1], hidden=True)["hidden"].clone()
         db = m.decode(b, [0], embeds=xd[t:t + 1], hidden=True)["hidden"].clone()
