@@ -10,7 +10,7 @@ LIB_PATH = os.path.join(HERE, "liblfm3.so")
 
 LFM3_MAX_LAYERS = 64
 LFM3_LAYER_CONV, LFM3_LAYER_FULL, LFM3_LAYER_SLIDING = 0, 1, 2
-LFM3_FFN_BF16, LFM3_FFN_NVFP4 = 0, 1
+LFM3_FFN_BF16, LFM3_FFN_NVFP4, LFM3_FFN_AFFINE = 0, 1, 2
 
 STATUS = {0: "LFM3_OK", -1: "LFM3_E_ARG", -2: "LFM3_E_CONFIG", -3: "LFM3_E_CAPACITY", -4: "LFM3_E_CUDA",
           -5: "LFM3_E_UNSUPPORTED", -6: "LFM3_E_TIMEOUT", -7: "LFM3_E_STATE"}
@@ -29,14 +29,15 @@ class lfm3_config(C.Structure):
                 ("theta_full", C.c_float), ("theta_sliding", C.c_float), ("rope_pairs_full", C.c_int),
                 ("eps", C.c_float), ("has_head", C.c_int), ("ffn_format", C.c_int), ("page_size", C.c_int),
                 ("n_pages", C.c_int), ("max_streams", C.c_int), ("max_pages_per_stream", C.c_int),
-                ("max_chunk", C.c_int), ("max_batch", C.c_int)]
+                ("max_chunk", C.c_int), ("max_batch", C.c_int), ("ffn_bits", C.c_int)]
 
 
 class lfm3_layer_weights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in ("op_norm", "post_op_norm", "ffn_norm", "post_ffn_norm", "in_proj", "conv",
                                           "out_proj", "qkvg", "q_norm", "k_norm", "o_proj", "w1", "w3", "w2",
                                           "w1_codes", "w1_scales", "w3_codes", "w3_scales", "w2_codes",
-                                          "w2_scales")] + [("w13_scale", C.c_float), ("w2_scale", C.c_float)]
+                                          "w2_scales")] + [("w13_scale", C.c_float), ("w2_scale", C.c_float)] + \
+        [(n, C.c_void_p) for n in ("w1_biases", "w3_biases", "w2_biases")]
 
 
 class lfm3_weights(C.Structure):

@@ -283,16 +283,20 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
           make_float4(0.f, 0.f, 0.f, 0.f);
   }
 
-  // ---- the last block of (stream, kv head) merges the splits and applies the gates
-  __threadfence();
+  // ---- the last block of (stream, kv head) merges the splits and applies the gates. The count is
+  // taken with acquire-release semantics after the block barrier: it releases every thread's
+  // partial (ordered before it by the barrier) and, in the last block, acquires the others'.
   __syncthreads();
 #ifdef LFM3_TRACE
   if (tid == 0) TRACE(A.trace, A.trace_id, 3);
 #endif
-  if (tid == 0) last = atomicAdd(A.counters + b * HKV + kvh, 1u) == (unsigned)(nact - 1);
+  if (tid == 0) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(A.counters + b * HKV + kvh) : "memory");
+    last = old == (unsigned)(nact - 1);
+  }
   __syncthreads();
   if (!last) return;
-  __threadfence();
   // warp w: head w & 3 over the splits s = half, half + 2, ... (half = w >> 2)
   const int hh = warp & 3, half = warp >> 2;
   const size_t hb = hbase + (size_t)hh * splits;
@@ -311,7 +315,7 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
       if ((s & 1) == half) lsum += wgt * m2.y;
     }
     const int ns = min(32, nact - s0);
-#pragma unroll 8
+#pragma unroll 16
     for (int i = half; i < ns; i += 2) {
       const float wi = __shfl_sync(0xffffffffu, wgt, i);
       const float4 o = __ldcg(reinterpret_cast<const float4*>(part + (hb + s0 + i) * HD) + lane);

@@ -125,6 +125,7 @@ struct WsArgs {
   const bf16* w; const bf16* w3;                   // bf16 weights [N][K] (SwiGLU: w1, w3)
   const uint8_t* codes; const uint8_t* scales;     // NVFP4 (SwiGLU: w1)
   const uint8_t* codes3; const uint8_t* scales3;   // NVFP4 w3
+  int bits;                                        // affine: code width (4, 6, 8); scales and biases bf16
   float tscale;
   int K, N, rows, splits;
   int pro;                                         // WS_PRO_LOAD: x bf16 [rows][K]; WS_PRO_NORM: see below
@@ -146,13 +147,22 @@ struct WsArgs {
 #endif
 };
 struct WsMaps {
-  CUtensorMap w, w3, s, s3;  // weights (SwiGLU: w1, w3) or NVFP4 codes; NVFP4 scales
+  CUtensorMap w, w3, s, s3;  // weights (SwiGLU: w1, w3) or quantised codes; NVFP4 / affine scales
+  CUtensorMap b, b3;         // affine biases
 };
 bool make_ws_map(CUtensorMap* m, const void* w, int N, int K, int fp4, int br, int kch);
 bool make_ws_scale_map(CUtensorMap* m, const void* sc, int N, int K, int br, int kch);
 int ws_kch(int epi, int fp4);
-int ws_br(int epi);
-cudaError_t wstream(int epi, int nvfp4, const WsMaps& mp, const WsArgs& a, cudaStream_t s);
+int ws_br(int epi, int fp4);
+enum WsFormat { WS_BF16 = 0, WS_NVFP4 = 1, WS_AFFINE = 2 };
+cudaError_t wstream(int epi, int format, const WsMaps& mp, const WsArgs& a, cudaStream_t s);
+// Affine code maps ([N][K * bits / 8] bytes as 64- or 96-byte blocks) and bf16 scale / bias maps.
+bool make_aff_map(CUtensorMap* m, const void* codes, int N, int K, int bits, int br);
+bool make_aff_sb_map(CUtensorMap* m, const void* sb, int N, int K, int br);
+int aff_br(int epi);
+// Affine weights expanded to bf16 for the tensor-core GEMM: w = bf16(s * q + b).
+cudaError_t affine_to_bf16(const uint8_t* codes, const void* scales, const void* biases, int bits, int N, int K, bf16* out,
+                           cudaStream_t s);
 cudaError_t wstream_init();
 
 // ---------------------------------------------------------------- attention

@@ -143,7 +143,7 @@ size_t layout(lfm3_ctx* c, char* base) {
     c->rope_cos[k] = reinterpret_cast<float*>(take(4 * (size_t)c->max_pos * (HD / 2)));
     c->rope_sin[k] = reinterpret_cast<float*>(take(4 * (size_t)c->max_pos * (HD / 2)));
   }
-  c->deq = g.ffn_format == LFM3_FFN_NVFP4 ? reinterpret_cast<bf16*>(take(2 * (size_t)2 * F * D)) : nullptr;
+  c->deq = g.ffn_format != LFM3_FFN_BF16 ? reinterpret_cast<bf16*>(take(2 * (size_t)2 * F * D)) : nullptr;
   c->attn_cnt = reinterpret_cast<unsigned*>(take(4 * (size_t)g.max_batch * HKV));
   c->conv_snap = reinterpret_cast<bf16*>(take(2 * (size_t)c->n_conv * g.max_batch * CST * D));
   c->side_k = reinterpret_cast<bf16*>(take(2 * (size_t)c->n_sliding * g.max_batch * HKV * HD));
@@ -171,8 +171,10 @@ lfm3_status check_config(lfm3_ctx* c, const lfm3_config* g) {
     return fail(c, LFM3_E_CONFIG, "rope_pairs_full %d outside 0..%d", g->rope_pairs_full, HD / 2);
   if (!(g->theta_full > 0.f) || !(g->theta_sliding > 0.f) || !(g->eps > 0.f))
     return fail(c, LFM3_E_CONFIG, "rotary bases and eps must be positive");
-  if (g->ffn_format != LFM3_FFN_BF16 && g->ffn_format != LFM3_FFN_NVFP4)
+  if (g->ffn_format != LFM3_FFN_BF16 && g->ffn_format != LFM3_FFN_NVFP4 && g->ffn_format != LFM3_FFN_AFFINE)
     return fail(c, LFM3_E_UNSUPPORTED, "Lfm3UnsupportedFfnFormat: %d", g->ffn_format);
+  if (g->ffn_format == LFM3_FFN_AFFINE && g->ffn_bits != 4 && g->ffn_bits != 6 && g->ffn_bits != 8)
+    return fail(c, LFM3_E_UNSUPPORTED, "Lfm3UnsupportedAffineBits: %d (the kernels implement 4, 6 and 8)", g->ffn_bits);
   if (g->has_head && (g->vocab <= 0 || g->vocab % 16))
     return fail(c, LFM3_E_UNSUPPORTED, "Lfm3UnsupportedVocab: vocab %d must be a positive multiple of 16", g->vocab);
   if (g->max_streams < 1) return fail(c, LFM3_E_CONFIG, "max_streams %d < 1", g->max_streams);
@@ -181,7 +183,6 @@ lfm3_status check_config(lfm3_ctx* c, const lfm3_config* g) {
     return fail(c, LFM3_E_CONFIG, "a slot of %d pages exceeds 2^20 positions", g->max_pages_per_stream);
   if (g->max_chunk < 1 || g->max_chunk > 2048) return fail(c, LFM3_E_CONFIG, "max_chunk %d outside 1..2048", g->max_chunk);
   if (g->max_batch < 1 || g->max_batch > 64) return fail(c, LFM3_E_CONFIG, "max_batch %d outside 1..64", g->max_batch);
-  if (g->max_batch > g->max_streams) return fail(c, LFM3_E_CONFIG, "max_batch > max_streams");
   int nf = 0;
   for (int i = 0; i < g->n_layers; ++i) nf += g->layer_type[i] == LFM3_LAYER_FULL;
   if (nf && g->n_pages < 1) return fail(c, LFM3_E_CONFIG, "full-attention layers need n_pages >= 1");
@@ -205,6 +206,11 @@ lfm3_status check_weights(lfm3_ctx* c, const lfm3_config* g, const lfm3_weights*
     }
     if (g->ffn_format == LFM3_FFN_BF16) {
       need[n++] = L.w1; need[n++] = L.w3; need[n++] = L.w2;
+    } else if (g->ffn_format == LFM3_FFN_AFFINE) {
+      need[n++] = L.w1_codes; need[n++] = L.w1_scales; need[n++] = L.w1_biases;
+      need[n++] = L.w3_codes; need[n++] = L.w3_scales; need[n++] = L.w3_biases;
+      need[n++] = L.w2_codes; need[n++] = L.w2_scales;
+      if (!L.w2_biases) return fail(c, LFM3_E_ARG, "layer %d: w2_biases is NULL", i);
     } else {
       need[n++] = L.w1_codes; need[n++] = L.w1_scales; need[n++] = L.w3_codes; need[n++] = L.w3_scales;
       need[n++] = L.w2_codes; need[n++] = L.w2_scales;
@@ -245,13 +251,16 @@ double gemm_bytes(const GemmPlan& p, int M) {
   return 2.0 * nw * p.N * (double)p.K + 2.0 * M * p.K + (p.epi == GEMM_F32 ? 4.0 : 2.0) * M * p.N;
 }
 
-cudaError_t run_ws(lfm3_ctx* c, int epi, int fp4, const WsMaps& mp, const WsArgs& a, cudaStream_t s) {
+// format: WS_BF16, WS_NVFP4 or WS_AFFINE (a.bits wide codes)
+cudaError_t run_ws(lfm3_ctx* c, int epi, int format, const WsMaps& mp, const WsArgs& a, cudaStream_t s) {
   const double mats = (a.w3 || a.codes3) ? 2.0 : 1.0;
   const double rows = epi == GEMV_CONV ? 3.0 * D : (double)a.N;
-  const double w = fp4 ? rows * a.K / 2 + rows * a.K / 16 : 2.0 * rows * a.K;
+  const double w = format == WS_NVFP4    ? rows * a.K / 2 + rows * a.K / 16
+                   : format == WS_AFFINE ? rows * a.K * a.bits / 8.0 + 2.0 * 2 * rows * a.K / 64
+                                         : 2.0 * rows * a.K;
   const double bytes = mats * w + 2.0 * a.rows * a.K + 4.0 * a.rows * a.N;
   Bracket b(c, s, bytes, 2.0 * a.rows * rows * a.K * mats);
-  return wstream(epi, fp4, mp, a, s);
+  return wstream(epi, format, mp, a, s);
 }
 cudaError_t run_gemm(lfm3_ctx* c, const GemmPlan& p, int M, cudaStream_t s) {
   Bracket b(c, s, gemm_bytes(p, M), gemm_flops(p, M));
@@ -347,7 +356,14 @@ AttnLayer attn_layer(lfm3_ctx* ctx, const lfm3_state* st, int l, const Views& v)
 // FFN of n rows (prefill or large-batch decode) on the tensor-core GEMM: u = SwiGLU -> big, w2 -> part.
 lfm3_status ffn_gemm(lfm3_ctx* ctx, int l, int n, cudaStream_t s) {
   const lfm3_layer_weights& W = ctx->L[l];
-  if (ctx->cfg.ffn_format == LFM3_FFN_NVFP4) {
+  if (ctx->cfg.ffn_format == LFM3_FFN_AFFINE) {
+    const int bits = ctx->cfg.ffn_bits;
+    CK(affine_to_bf16(W.w1_codes, W.w1_scales, W.w1_biases, bits, F, D, ctx->deq, s));
+    CK(affine_to_bf16(W.w3_codes, W.w3_scales, W.w3_biases, bits, F, D, ctx->deq + (size_t)F * D, s));
+    CK(run_gemm(ctx, ctx->deq_w13, n, s));
+    CK(affine_to_bf16(W.w2_codes, W.w2_scales, W.w2_biases, bits, D, F, ctx->deq, s));
+    CK(run_gemm(ctx, ctx->deq_w2, n, s));
+  } else if (ctx->cfg.ffn_format == LFM3_FFN_NVFP4) {
     CK(nvfp4_to_bf16(W.w1_codes, W.w1_scales, W.w13_scale, F, D, ctx->deq, s));
     CK(nvfp4_to_bf16(W.w3_codes, W.w3_scales, W.w13_scale, F, D, ctx->deq + (size_t)F * D, s));
     GemmPlan p = ctx->deq_w13;
@@ -457,7 +473,7 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
     LayerPlan& P = ctx->plans[l];
     bool ok = true;
     auto bf = [&](CUtensorMap* m, const void* w, int N, int K, int epi) {
-      ok &= make_ws_map(m, w, N, K, 0, ws_br(epi), ws_kch(epi, 0));
+      ok &= make_ws_map(m, w, N, K, 0, ws_br(epi, 0), ws_kch(epi, 0));
     };
     if (g.layer_type[l] == LFM3_LAYER_CONV) {
       bf(&P.ws_in.w, W.in_proj, 3 * D, D, GEMV_CONV);
@@ -470,14 +486,28 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
       P.ws_qkvg.w3 = P.ws_qkvg.s = P.ws_qkvg.s3 = P.ws_qkvg.w;
       P.ws_o.w3 = P.ws_o.s = P.ws_o.s3 = P.ws_o.w;
     }
-    if (g.ffn_format == LFM3_FFN_NVFP4) {
+    if (g.ffn_format == LFM3_FFN_AFFINE) {
+      const int bits = g.ffn_bits;
+      ok &= make_aff_map(&P.ws_w13.w, W.w1_codes, F, D, bits, aff_br(GEMV_SWIGLU));
+      ok &= make_aff_map(&P.ws_w13.w3, W.w3_codes, F, D, bits, aff_br(GEMV_SWIGLU));
+      ok &= make_aff_sb_map(&P.ws_w13.s, W.w1_scales, F, D, aff_br(GEMV_SWIGLU));
+      ok &= make_aff_sb_map(&P.ws_w13.s3, W.w3_scales, F, D, aff_br(GEMV_SWIGLU));
+      ok &= make_aff_sb_map(&P.ws_w13.b, W.w1_biases, F, D, aff_br(GEMV_SWIGLU));
+      ok &= make_aff_sb_map(&P.ws_w13.b3, W.w3_biases, F, D, aff_br(GEMV_SWIGLU));
+      ok &= make_aff_map(&P.ws_w2.w, W.w2_codes, D, F, bits, aff_br(GEMV_PARTIAL));
+      ok &= make_aff_sb_map(&P.ws_w2.s, W.w2_scales, D, F, aff_br(GEMV_PARTIAL));
+      ok &= make_aff_sb_map(&P.ws_w2.b, W.w2_biases, D, F, aff_br(GEMV_PARTIAL));
+      P.ws_w2.w3 = P.ws_w2.w;
+      P.ws_w2.s3 = P.ws_w2.s;
+      P.ws_w2.b3 = P.ws_w2.b;
+    } else if (g.ffn_format == LFM3_FFN_NVFP4) {
       const int kch = ws_kch(GEMV_PARTIAL, 1);
-      ok &= make_ws_map(&P.ws_w13.w, W.w1_codes, F, D, 1, ws_br(GEMV_SWIGLU), kch);
-      ok &= make_ws_map(&P.ws_w13.w3, W.w3_codes, F, D, 1, ws_br(GEMV_SWIGLU), kch);
-      ok &= make_ws_scale_map(&P.ws_w13.s, W.w1_scales, F, D, ws_br(GEMV_SWIGLU), kch);
-      ok &= make_ws_scale_map(&P.ws_w13.s3, W.w3_scales, F, D, ws_br(GEMV_SWIGLU), kch);
-      ok &= make_ws_map(&P.ws_w2.w, W.w2_codes, D, F, 1, ws_br(GEMV_PARTIAL), kch);
-      ok &= make_ws_scale_map(&P.ws_w2.s, W.w2_scales, D, F, ws_br(GEMV_PARTIAL), kch);
+      ok &= make_ws_map(&P.ws_w13.w, W.w1_codes, F, D, 1, ws_br(GEMV_SWIGLU, 1), kch);
+      ok &= make_ws_map(&P.ws_w13.w3, W.w3_codes, F, D, 1, ws_br(GEMV_SWIGLU, 1), kch);
+      ok &= make_ws_scale_map(&P.ws_w13.s, W.w1_scales, F, D, ws_br(GEMV_SWIGLU, 1), kch);
+      ok &= make_ws_scale_map(&P.ws_w13.s3, W.w3_scales, F, D, ws_br(GEMV_SWIGLU, 1), kch);
+      ok &= make_ws_map(&P.ws_w2.w, W.w2_codes, D, F, 1, ws_br(GEMV_PARTIAL, 1), kch);
+      ok &= make_ws_scale_map(&P.ws_w2.s, W.w2_scales, D, F, ws_br(GEMV_PARTIAL, 1), kch);
       P.ws_w2.w3 = P.ws_w2.w;
       P.ws_w2.s3 = P.ws_w2.s;
     } else {
@@ -490,11 +520,11 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
     if (!ok) return fail(ctx, LFM3_E_CUDA, "layer %d: weight-streaming tensor map encoding failed", l);
   }
   if (g.has_head) {
-    if (!make_ws_map(&ctx->ws_head.w, ctx->embed, g.vocab, D, 0, ws_br(GEMV_HEAD), ws_kch(GEMV_HEAD, 0)))
+    if (!make_ws_map(&ctx->ws_head.w, ctx->embed, g.vocab, D, 0, ws_br(GEMV_HEAD, 0), ws_kch(GEMV_HEAD, 0)))
       return fail(ctx, LFM3_E_CUDA, "head weight-streaming tensor map encoding failed");
     ctx->ws_head.w3 = ctx->ws_head.s = ctx->ws_head.s3 = ctx->ws_head.w;
   }
-  if (g.ffn_format == LFM3_FFN_NVFP4) {
+  if (g.ffn_format != LFM3_FFN_BF16) {
     bool ok = plan_gemm(&ctx->deq_w13, GEMM_SWIGLU, ctx->xn, R, ctx->deq, ctx->deq + (size_t)F * D, F, D, ctx->big, F, 1.f);
     ok &= plan_gemm(&ctx->deq_w2, GEMM_F32, ctx->big, R, ctx->deq, nullptr, D, F, ctx->part, D, 1.f);
     if (!ok) return fail(ctx, LFM3_E_CUDA, "NVFP4 tensor map encoding failed");
@@ -614,7 +644,7 @@ lfm3_status prefill_rows(lfm3_ctx* ctx, const lfm3_state* st, int slot, const in
       a.logits = d_logits;
       a.amax = ctx->amax;
       a.err = ctx->err;
-      CK(run_ws(ctx, GEMV_HEAD, 0, ctx->ws_head, a, s));
+      CK(run_ws(ctx, GEMV_HEAD, WS_BF16, ctx->ws_head, a, s));
     }
     CK(finish_step(st->seq_len, ctx->row_slot, nc, nr, slot, head ? ctx->amax : nullptr, head ? d_argmax : nullptr, 1,
                    s));
@@ -715,7 +745,7 @@ lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, in
       a.logits = d_logits ? d_logits + (size_t)b0 * g.vocab : nullptr;
       a.amax = ctx->amax + b0;
       a.err = ctx->err;
-      CK(run_ws(ctx, GEMV_HEAD, 0, ctx->ws_head, a, s));
+      CK(run_ws(ctx, GEMV_HEAD, WS_BF16, ctx->ws_head, a, s));
     }
   }
   CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr,
@@ -731,6 +761,8 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, i
   const lfm3_config& g = ctx->cfg;
   const float eps = g.eps;
   const bool fp4 = g.ffn_format == LFM3_FFN_NVFP4;
+  const bool aff = g.ffn_format == LFM3_FFN_AFFINE;
+  const int ffmt = fp4 ? WS_NVFP4 : aff ? WS_AFFINE : WS_BF16;
   CK(setup_rows(0, 0, d_slots, st->seq_len, nb, win, ctx->row_slot, ctx->row_pos, ctx->amax, s));
   const Rows rows{ctx->row_slot, ctx->row_pos, nb};
   CK(embed_rows(d_tokens, ctx->embed, B(d_embeds), nb, ctx->x_res, d_hidden, s));
@@ -775,7 +807,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, i
       c.win = win;
       c.conv_snap = ctx->conv_snap + (size_t)ctx->kidx[l] * g.max_batch * CST * D;
       norm_in(c, B(W.op_norm), dump_l);
-      CK(run_ws(ctx, GEMV_CONV, 0, ctx->plans[l].ws_in, c, s));
+      CK(run_ws(ctx, GEMV_CONV, WS_BF16, ctx->plans[l].ws_in, c, s));
       advance();
       WsArgs o{};
       base(o, D, D, SPLIT_DD);
@@ -783,7 +815,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, i
       o.x = ctx->y;
       o.w = B(W.out_proj);
       o.part_out = ctx->part;
-      CK(run_ws(ctx, GEMV_PARTIAL, 0, ctx->plans[l].ws_out, o, s));
+      CK(run_ws(ctx, GEMV_PARTIAL, WS_BF16, ctx->plans[l].ws_out, o, s));
     } else {
       const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
       WsArgs q{};
@@ -791,7 +823,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, i
       q.w = B(W.qkvg);
       q.part_out = ctx->part3;
       norm_in(q, B(W.op_norm), dump_l);
-      CK(run_ws(ctx, GEMV_PARTIAL, 0, ctx->plans[l].ws_qkvg, q, s));
+      CK(run_ws(ctx, GEMV_PARTIAL, WS_BF16, ctx->plans[l].ws_qkvg, q, s));
       advance();
       AttnDecodeArgs A = attn_args(ctx, l, win);
       CK(attn_decode_fused(ctx->part3, rows, attn_layer(ctx, st, l, v), A, full ? splits_full : WIN / DEC_KEYS,
@@ -802,7 +834,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, i
       o.x = ctx->y;
       o.w = B(W.o_proj);
       o.part_out = ctx->part;
-      CK(run_ws(ctx, GEMV_PARTIAL, 0, ctx->plans[l].ws_o, o, s));
+      CK(run_ws(ctx, GEMV_PARTIAL, WS_BF16, ctx->plans[l].ws_o, o, s));
     }
     pend = ctx->part;
     pend_n = SPLIT_DD;
@@ -810,27 +842,29 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, i
     WsArgs f{};
     base(f, D, F, 1);
     f.out = ctx->big;
-    if (fp4) {
+    if (fp4 || aff) {
       f.codes = W.w1_codes; f.scales = W.w1_scales; f.codes3 = W.w3_codes; f.scales3 = W.w3_scales;
       f.tscale = W.w13_scale;
+      f.bits = g.ffn_bits;
     } else {
       f.w = B(W.w1);
       f.w3 = B(W.w3);
     }
     norm_in(f, B(W.ffn_norm), nullptr);
-    CK(run_ws(ctx, GEMV_SWIGLU, fp4, ctx->plans[l].ws_w13, f, s));
+    CK(run_ws(ctx, GEMV_SWIGLU, ffmt, ctx->plans[l].ws_w13, f, s));
     advance();
     WsArgs d{};
     base(d, F, D, SPLIT_W2);
     d.pro = WS_PRO_LOAD;
     d.x = ctx->big;
     d.part_out = ctx->part2;
-    if (fp4) {
+    if (fp4 || aff) {
       d.codes = W.w2_codes; d.scales = W.w2_scales; d.tscale = W.w2_scale;
+      d.bits = g.ffn_bits;
     } else {
       d.w = B(W.w2);
     }
-    CK(run_ws(ctx, GEMV_PARTIAL, fp4, ctx->plans[l].ws_w2, d, s));
+    CK(run_ws(ctx, GEMV_PARTIAL, ffmt, ctx->plans[l].ws_w2, d, s));
     pend = ctx->part2;
     pend_n = SPLIT_W2;
     pend_g = B(W.post_ffn_norm);
@@ -844,7 +878,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, i
     h.logits = d_logits;
     h.amax = ctx->amax;
     norm_in(h, ctx->final_norm, dump_last);
-    CK(run_ws(ctx, GEMV_HEAD, 0, ctx->ws_head, h, s));
+    CK(run_ws(ctx, GEMV_HEAD, WS_BF16, ctx->ws_head, h, s));
     advance();
   } else if (dump_last) {
     CK(resid_norm(cur, pend, pend_n, (long)nb * D, pend_g, nullptr, nullptr, nb, eps, dump_last, s));

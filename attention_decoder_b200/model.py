@@ -42,6 +42,7 @@ class Lfm3Model:
         self.geom = g
         self.device = torch.device(device)
         self.nvfp4 = weights["ffn"] == "nvfp4"
+        self.affine = weights["ffn"].startswith("affine")
         max_batch = max_batch or max_streams
         if n_pages is None:
             n_pages = max_streams * max_pages_per_stream
@@ -54,7 +55,8 @@ class Lfm3Model:
         cfg.theta_full, cfg.theta_sliding = g.theta_full, g.theta_sliding
         cfg.rope_pairs_full, cfg.eps = g.rope_pairs_full, g.eps
         cfg.has_head = 1 if g.has_head else 0
-        cfg.ffn_format = L.LFM3_FFN_NVFP4 if self.nvfp4 else L.LFM3_FFN_BF16
+        cfg.ffn_format = L.LFM3_FFN_NVFP4 if self.nvfp4 else (L.LFM3_FFN_AFFINE if self.affine else L.LFM3_FFN_BF16)
+        cfg.ffn_bits = int(weights["ffn"][6:]) if self.affine else 0
         cfg.page_size = 64
         cfg.n_pages = n_pages
         cfg.max_streams = max_streams
@@ -86,7 +88,12 @@ class Lfm3Model:
                 # q | k | v | gate rows as one projection weight
                 lw.qkvg = up(np.concatenate([Lw["q_proj"], Lw["k_proj"], Lw["v_proj"], Lw["gate_proj"]], axis=0))
                 lw.q_norm, lw.k_norm, lw.o_proj = up(Lw["q_norm"]), up(Lw["k_norm"]), up(Lw["o_proj"])
-            if self.nvfp4:
+            if self.affine:
+                for nm in ("w1", "w3", "w2"):
+                    setattr(lw, nm + "_codes", up8(Lw[nm + "_codes"].view(np.uint8)))
+                    setattr(lw, nm + "_scales", up(Lw[nm + "_scales"]))
+                    setattr(lw, nm + "_biases", up(Lw[nm + "_biases"]))
+            elif self.nvfp4:
                 lw.w1_codes, lw.w1_scales = up8(Lw["w1_codes"]), up8(Lw["w1_scales"])
                 lw.w3_codes, lw.w3_scales = up8(Lw["w3_codes"]), up8(Lw["w3_scales"])
                 lw.w2_codes, lw.w2_scales = up8(Lw["w2_codes"]), up8(Lw["w2_scales"])

@@ -56,7 +56,7 @@ typedef enum {
 } lfm3_status;
 
 enum { LFM3_LAYER_CONV = 0, LFM3_LAYER_FULL = 1, LFM3_LAYER_SLIDING = 2 };
-enum { LFM3_FFN_BF16 = 0, LFM3_FFN_NVFP4 = 1 };
+enum { LFM3_FFN_BF16 = 0, LFM3_FFN_NVFP4 = 1, LFM3_FFN_AFFINE = 2 };
 #define LFM3_MAX_LAYERS 64
 
 /* Geometry and capacity. The kernels implement d_model 2048, d_ffn 7680, 16 q / 4 kv heads of
@@ -70,13 +70,14 @@ typedef struct {
   int rope_pairs_full;             /* rotated (i, i + head_dim/2) pairs on full layers (32) */
   float eps;                       /* RMSNorm epsilon (1e-5)                              */
   int has_head;                    /* 1: token ids in, embedding + tied head + argmax out; 0: vectors in/out */
-  int ffn_format;                  /* LFM3_FFN_BF16 or LFM3_FFN_NVFP4                     */
+  int ffn_format;                  /* LFM3_FFN_BF16, LFM3_FFN_NVFP4 or LFM3_FFN_AFFINE    */
   int page_size;                   /* positions per KV page (64)                          */
   int n_pages;                     /* pages in the pool, per full-attention layer         */
   int max_streams;                 /* slots in the state                                  */
   int max_pages_per_stream;        /* page-table width; a slot holds at most this x page_size positions */
   int max_chunk;                   /* rows per prefill pass (1..2048); longer prompts run in chunks */
-  int max_batch;                   /* streams per decode step (1..64)                     */
+  int max_batch;                   /* rows per decode step (1..64): streams, or streams x window rows in lfm3_verify */
+  int ffn_bits;                    /* LFM3_FFN_AFFINE: code width, 4, 6 or 8 (ignored otherwise) */
 } lfm3_config;
 
 /* One layer's weights: device pointers, bf16 unless stated; unused fields may be NULL. */
@@ -108,6 +109,14 @@ typedef struct {
   const uint8_t* w2_scales; /* [d_model][d_ffn/16] */
   float w13_scale;          /* fp32 tensor scale shared by w1 and w3 */
   float w2_scale;
+  /* Affine FFN (MLX affine groups of 64; TensorFold issue #1491, "Checkpoint handling"): w = s * q + b
+   * with q an unsigned ffn_bits-bit code, s and b bf16 per group of 64 inputs. The codes of a row
+   * are one little-endian bit stream (code k at bits [k * bits, k * bits + bits)) in the *_codes
+   * fields, [rows][cols * bits / 8] bytes; the scales in the *_scales fields and the biases here
+   * are bf16 [rows][cols / 64]. */
+  const uint8_t* w1_biases;
+  const uint8_t* w3_biases;
+  const uint8_t* w2_biases;
 } lfm3_layer_weights;
 
 typedef struct {

@@ -14,5 +14,5 @@ from .gen import (  # noqa: F401
     CONV, FULL, SLIDING,
     Lfm3Geometry, lfm3_1p7b, lfm3_slice3, tiny_geometry,
     rng_for, bf16_bits, make_weights, make_tokens, make_embeds,
-    nvfp4_draw, page_permutation, context_lengths, synthetic_state,
+    nvfp4_draw, affine_draw, page_permutation, context_lengths, synthetic_state,
 )

@@ -143,11 +143,28 @@ def nvfp4_draw(seed: int, tag: str, n: int, k: int):
 NVFP4_TENSOR_SCALE = np.float32(2.0 ** -8)
 
 
+def affine_draw(seed: int, tag: str, n: int, k: int, bits: int):
+    """One MLX-style affine weight [n, k] in groups of 64 along k: codes uniform over the
+    2^bits values, packed as one little-endian bit stream per row into uint32 words; per group a
+    bf16 scale s = 2^u * 0.04 / (2^bits - 1), u ~ U(-1, 1), and a bf16 bias drawn around
+    -s * (2^bits - 1) / 2, so that s * q + b spans about +-0.02 like the bf16 weights."""
+    assert k % 64 == 0 and (k * bits) % 32 == 0
+    g = rng_for(seed, tag + ".codes")
+    codes = g.integers(0, 1 << bits, size=(n, k), dtype=np.uint8)
+    bitsarr = ((codes[:, :, None] >> np.arange(bits, dtype=np.uint8)[None, None, :]) & 1).reshape(n, k * bits)
+    packed = np.packbits(bitsarr, axis=1, bitorder="little").view(np.uint32)
+    g2 = rng_for(seed, tag + ".scales")
+    s = (np.exp2(g2.uniform(-1.0, 1.0, size=(n, k // 64))) * (0.04 / ((1 << bits) - 1))).astype(np.float32)
+    g3 = rng_for(seed, tag + ".biases")
+    b = (-s * ((1 << bits) - 1) / 2.0 * (1.0 + 0.05 * g3.standard_normal((n, k // 64)))).astype(np.float32)
+    return np.ascontiguousarray(packed), bf16_bits(s), bf16_bits(b)
+
+
 def make_weights(geom: Lfm3Geometry, seed: int = 0, ffn: str = "bf16", threads: int | None = None) -> dict:
     """Random-init weights: linear and conv weights N(0, 0.02), norm gains 1 + N(0, 0.02),
     all rounded to bf16 once. ``ffn='nvfp4'`` draws the FFN (w1, w3, w2) as NVFP4.
     Each tensor has its own seeded stream, so tensors are drawn in parallel threads."""
-    if ffn not in ("bf16", "nvfp4"):
+    if ffn not in ("bf16", "nvfp4", "affine4", "affine6", "affine8"):
         raise ValueError(ffn)
     D, F, d = geom.d_model, geom.d_ffn, geom.head_dim
     W = {"geometry": geom, "ffn": ffn, "layers": []}
@@ -181,6 +198,11 @@ def make_weights(geom: Lfm3Geometry, seed: int = 0, ffn: str = "bf16", threads: 
             normal("w1", (F, D), 0.02)
             normal("w3", (F, D), 0.02)
             normal("w2", (D, F), 0.02)
+        elif ffn.startswith("affine"):
+            bits = int(ffn[6:])
+            L["affine_bits"] = bits
+            for nm, (n, k) in (("w1", (F, D)), ("w3", (F, D)), ("w2", (D, F))):
+                jobs.append((L, nm, lambda nm=nm, n=n, k=k, p=p: affine_draw(seed, p + nm, n, k, bits)))
         else:
             for nm, (n, k) in (("w1", (F, D)), ("w3", (F, D)), ("w2", (D, F))):
                 jobs.append((L, nm, lambda nm=nm, n=n, k=k, p=p: nvfp4_draw(seed, p + nm, n, k)))
@@ -190,7 +212,9 @@ def make_weights(geom: Lfm3Geometry, seed: int = 0, ffn: str = "bf16", threads: 
     with ThreadPoolExecutor(max_workers=workers) as ex:
         results = list(ex.map(lambda j: j[2](), jobs))
     for (box, key, _), val in zip(jobs, results):
-        if isinstance(val, tuple):
+        if isinstance(val, tuple) and len(val) == 3:
+            box[key + "_codes"], box[key + "_scales"], box[key + "_biases"] = val
+        elif isinstance(val, tuple):
             box[key + "_codes"], box[key + "_scales"] = val
         else:
             box[key] = val

@@ -17,6 +17,8 @@ the pages fix (``bf16=True``; see lfm3.py):
   incremental mode (conv columns, a growing KV list, a 256-slot ring).
 * ``nvfp4.py`` - E2M1 / E4M3 decoding from the OCP definitions and exact
   NVFP4 dequantisation.
+* ``affine.py`` - MLX affine (4/6/8-bit, groups of 64) unpacking and
+  dequantisation.
 
 Every function is pinned by the ``-m "not gpu"`` tests (library routines,
 brute force, closed forms, invariants and the pages' own totals). The pages
@@ -26,3 +28,4 @@ geometry (tests/test_oracle_head_pins.py), beside the invariants above.
 """
 from .lfm3 import Lfm3Oracle, OracleState, rms_norm, rope_inv_freq, apply_rope, round_bf16  # noqa: F401
 from .nvfp4 import e2m1_value, e4m3_value, nvfp4_dequant  # noqa: F401
+from .affine import affine_unpack, affine_dequant  # noqa: F401

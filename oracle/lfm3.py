@@ -48,6 +48,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 from lfm3_inputs import CONV, FULL, SLIDING
+from .affine import affine_dequant
 from .nvfp4 import nvfp4_block_values
 
 
@@ -170,6 +171,13 @@ class Lfm3Oracle:
                 O["o_proj"] = _bf16(L["o_proj"])
             if "w1" in L:
                 O["w1"], O["w3"], O["w2"] = _bf16(L["w1"]), _bf16(L["w3"]), _bf16(L["w2"])
+                O["s13"] = O["s2"] = 1.0
+            elif "affine_bits" in L:
+                # MLX affine groups of 64: w = s * q + b, exact in float64
+                bits = L["affine_bits"]
+                for nm in ("w1", "w3", "w2"):
+                    cols = g.d_model if nm != "w2" else g.d_ffn
+                    O[nm] = affine_dequant(L[nm + "_codes"], L[nm + "_scales"], L[nm + "_biases"], bits, cols)
                 O["s13"] = O["s2"] = 1.0
             else:
                 # exact E2M1 x E4M3 products in float32; the fp32 tensor scale is applied
