@@ -73,6 +73,15 @@ DEVI void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The same with f16 operands.
+DEVI void mma_f16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 DEVI float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
 DEVI float siluf_(float x) { return x / (1.f + __expf(-x)); }
 

@@ -102,26 +102,29 @@ DEVI int ws_row(int tile, int rt, int g, int& which) {
   }
 }
 
-// E2M1 code (bit 3 sign, bits 2..1 exponent with bias 1, bit 0 mantissa) -> bf16 bits, exact:
-// 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives.
-DEVI uint32_t e2m1_bf16_bits(uint32_t c) {
-  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
-  const uint32_t mag = e == 0 ? (m ? 0x3F00u : 0u) : (((e + 126u) << 7) | (m << 6));
-  return mag | ((c & 8u) << 12);
+// bf16x2 -> f16x2 of the same values (rounding only outside f16's range).
+DEVI uint32_t ws_bf2h(uint32_t w) {
+  __half2 h = __floats2half2_rn(bflo(w), bfhi(w));
+  return *reinterpret_cast<uint32_t*>(&h);
 }
-
-DEVI uint32_t ws_e4m3x2(uint32_t b) {
-  const uint32_t s = (b & 0x80u) << 8;
-  const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
-  uint32_t bits = e == 0 ? (__float_as_uint((float)m * (1.0f / 512.0f)) >> 16) : (((e + 120u) << 7) | (m << 4));
-  bits |= s;
-  return bits | (bits << 16);
+// Four E2M1 codes pairs (the four bytes of w, element 2b in the low nibble) -> four f16x2, exact.
+DEVI void ws_e2m1x8_f16(uint32_t w, uint32_t& c01, uint32_t& c23, uint32_t& c45, uint32_t& c67) {
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+      " cvt.rn.f16x2.e2m1x2 %1, b1;\n cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(c01), "=r"(c23), "=r"(c45), "=r"(c67)
+      : "r"(w));
 }
-
-DEVI uint32_t ws_hmul2(uint32_t a, uint32_t b) {
-  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a), y = *reinterpret_cast<__nv_bfloat162*>(&b);
-  __nv_bfloat162 r = __hmul2(x, y);
-  return *reinterpret_cast<uint32_t*>(&r);
+// An E4M3 byte -> f16x2 holding its value twice, exact.
+DEVI uint32_t ws_e4m3_f16x2(uint32_t b) {
+  uint32_t r;
+  const uint32_t two = (b & 0xFFu) * 0x0101u;
+  asm("{\n .reg .b16 h;\n cvt.u16.u32 h, %1;\n cvt.rn.f16x2.e4m3x2 %0, h;\n}" : "=r"(r) : "r"(two));
+  return r;
+}
+DEVI uint32_t ws_hmul2_f16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
 // Weights are read once per step: their copies carry an evict-first L2 policy, so that the small
@@ -175,17 +178,16 @@ DEVI void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(WS_CW * 32) : 
 // Activations in shared memory: a 128-byte zero block (the MMA columns of absent streams read
 // it), then one row per stream of the block's K range, 64-byte skewed against bank conflicts.
 __host__ __device__ inline size_t ws_x_bytes(int rows, int Kc) { return 128 + (size_t)rows * (Kc + 32) * 2; }
-// Stages start on a 1024-byte boundary after the activations (and the NVFP4 table).
-__host__ __device__ inline size_t ws_stage_base(int rows, int Kc, bool fp4) {
-  return (ws_x_bytes(rows, Kc) + (fp4 ? 256 * 32 * 4 : 0) + 1023) / 1024 * 1024;
-}
+// Stages start on a 1024-byte boundary after the activations.
+__host__ __device__ inline size_t ws_stage_base(int rows, int Kc) { return (ws_x_bytes(rows, Kc) + 1023) / 1024 * 1024; }
 
-// Consumer prologue of the weight-streaming kernels (consumer threads only): the NVFP4 code
-// table, then the activations of the block's K range into xs (bf16), either as given (LOAD) or
-// through the sandwich-norm step (NORM). Ends with the consumers synchronised.
-template <bool FP4>
-DEVI void ws_prologue(const WsArgs& a, unsigned char* smem, bf16* xs, int XS, int Kc, int kcta, uint32_t* lut,
-                      float* redn, unsigned long long* trb, int trid) {
+// Consumer prologue of the weight-streaming kernels (consumer threads only): the activations of
+// the block's K range into xs, either as given (LOAD) or through the sandwich-norm step (NORM), as
+// bf16 - or, with X16, as f16 copies of the same bf16 values (exact for magnitudes in f16's
+// normal range, which the normed activations and the SwiGLU products of this model stay in) for
+// the NVFP4 kernel's f16 MMAs. Ends with the consumers synchronised.
+template <bool X16>
+DEVI void ws_prologue(const WsArgs& a, unsigned char* smem, bf16* xs, int XS, int Kc, int kcta, float* redn, unsigned long long* trb, int trid) {
   (void)XS; (void)Kc; (void)trb; (void)trid;
   const int ct = threadIdx.x, warp = ct >> 5, lane = ct & 31;
   // the norm gains are weights: requested before waiting for the previous kernel
@@ -204,12 +206,6 @@ DEVI void ws_prologue(const WsArgs& a, unsigned char* smem, bf16* xs, int XS, in
       }
     }
   }
-  if constexpr (FP4) {
-    for (int i = ct; i < 256 * 32; i += WS_CW * 32) {
-      const uint32_t v = (uint32_t)i >> 5;
-      lut[i] = e2m1_bf16_bits(v & 15u) | (e2m1_bf16_bits(v >> 4) << 16);
-    }
-  }
   pdl_wait();
   pdl_launch_dependents();
 #ifdef LFM3_TRACE
@@ -220,7 +216,9 @@ DEVI void ws_prologue(const WsArgs& a, unsigned char* smem, bf16* xs, int XS, in
     const int chunks = Kc / 8;
     for (int idx = ct; idx < a.rows * chunks; idx += WS_CW * 32) {
       const int b = idx / chunks, c = idx - b * chunks;
-      *reinterpret_cast<uint4*>(xs + (size_t)b * XS + c * 8) = ldg16(a.x + (size_t)b * a.K + kcta + c * 8);
+      uint4 v = ldg16(a.x + (size_t)b * a.K + kcta + c * 8);
+      if constexpr (X16) v = make_uint4(ws_bf2h(v.x), ws_bf2h(v.y), ws_bf2h(v.z), ws_bf2h(v.w));
+      *reinterpret_cast<uint4*>(xs + (size_t)b * XS + c * 8) = v;
     }
   } else {
     // residual + post-norm of the previous projection, then this projection's input norm. The
@@ -299,6 +297,7 @@ DEVI void ws_prologue(const WsArgs& a, unsigned char* smem, bf16* xs, int XS, in
           for (int j = 0; j < 4; ++j) {
             const int e = 8 * h + 2 * j;
             w[j] = pack_bf2(gn[e] * (x[e] * inv), gn[e + 1] * (x[e + 1] * inv));
+            if constexpr (X16) w[j] = ws_bf2h(w[j]);
           }
           *reinterpret_cast<uint4*>(xs + (size_t)b * XS + (c0 - kcta) + 8 * h) = make_uint4(w[0], w[1], w[2], w[3]);
         }
@@ -324,9 +323,7 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream(const __grid_constant
   const int XS = Kc + 32;  // activations row stride (elements): 64-byte skew against bank conflicts
   const bf16* xzero = reinterpret_cast<const bf16*>(smem);
   bf16* xs = reinterpret_cast<bf16*>(smem + 128);
-  // NVFP4: byte (two E2M1 codes) -> bf16x2, 256 entries x 32 copies (one per bank)
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + ws_x_bytes(a.rows, Kc));
-  unsigned char* stages = smem + ws_stage_base(a.rows, Kc, FP4);
+  unsigned char* stages = smem + ws_stage_base(a.rows, Kc);
   const int NS = a.stages;  // ring depth chosen by the launcher
   float* red = reinterpret_cast<float*>(stages + (size_t)NS * G::STAGE_BYTES);
   float* res = red + WS_CW * NRT * NT * 128;
@@ -404,9 +401,9 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream(const __grid_constant
 
   // -------------------------------------------------------------- consumers: prologue
 #ifdef LFM3_TRACE
-  ws_prologue<FP4>(a, smem, xs, XS, Kc, kcta, lut, redn, trb, trid);
+  ws_prologue<FP4>(a, smem, xs, XS, Kc, kcta, redn, trb, trid);
 #else
-  ws_prologue<FP4>(a, smem, xs, XS, Kc, kcta, lut, redn, nullptr, 0);
+  ws_prologue<FP4>(a, smem, xs, XS, Kc, kcta, redn, nullptr, 0);
 #endif
   const int ct = tid;
   // -------------------------------------------------------------- consumers: main loop
@@ -565,9 +562,11 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream(const __grid_constant
 // SWIGLU rows g of w1 and of w3 sit in MMA rows g and g + 8 of one tile, so SiLU(w1 x) * (w3 x)
 // needs nothing from other lanes) and K half w >> 2 of every stage; one reduction of the two K
 // halves per unit. A stage is 256 codes of each row (64 rows x 128 B) and their 16 E4M3 scales
-// per row; a lane step reads 8 B (16 codes, one scale) of rows g and g + 8, expands them exactly
-// through the byte -> bf16x2 table, multiplies by the block scale (exact in bf16) and issues two
-// m16n8k16 MMAs per 8 codes with the streams as the 8 columns.
+// per row; a lane step reads 8 B (16 codes, one scale) of rows g and g + 8, expands each code
+// byte to an f16 pair with the hardware E2M1 conversion, multiplies by the block scale (E4M3 ->
+// f16, also exact; so is the product: at most 5 significant bits, between 2^-10 and 2688) and
+// issues two f16 m16n8k16 MMAs per 8 codes with the streams as the 8 columns. No code table in
+// shared memory, so two blocks share an SM.
 constexpr int Q4_UR = 64;                        // weight rows per unit
 constexpr int Q4_KST = 256;                      // codes per row per stage
 constexpr int Q4_CODE_B = Q4_UR * Q4_KST / 2;    // 8 KB
@@ -575,9 +574,7 @@ constexpr int Q4_SC_B = Q4_UR * Q4_KST / 16;     // 1 KB
 constexpr int Q4_STAGE_B = Q4_CODE_B + Q4_SC_B;
 constexpr int Q4_STAGES = 8;
 
-__host__ __device__ inline size_t q4_stage_base(int rows, int Kc) {
-  return (ws_x_bytes(rows, Kc) + 256 * 32 * 4 + 1023) / 1024 * 1024;
-}
+__host__ __device__ inline size_t q4_stage_base(int rows, int Kc) { return ws_stage_base(rows, Kc); }
 
 template <int EPI, int NT>
 __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream_fp4(const __grid_constant__ CUtensorMap tw,
@@ -592,7 +589,6 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream_fp4(const __grid_cons
   const int XS = Kc + 32;
   const bf16* xzero = reinterpret_cast<const bf16*>(smem);
   bf16* xs = reinterpret_cast<bf16*>(smem + 128);
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + ws_x_bytes(a.rows, Kc));
   unsigned char* stages = smem + q4_stage_base(a.rows, Kc);
   const int NS = a.stages;
   float* red = reinterpret_cast<float*>(stages + (size_t)NS * Q4_STAGE_B);  // [4 tiles][NT][32 lanes][4]
@@ -667,10 +663,10 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream_fp4(const __grid_cons
   }
 
 #ifdef LFM3_TRACE
-  ws_prologue<true>(a, smem, xs, XS, Kc, kcta, lut, redn, trb, trid);
+  ws_prologue<true>(a, smem, xs, XS, Kc, kcta, redn, trb, trid);
   if (tid == 0) TRACE(trb, trid, 3);
 #else
-  ws_prologue<true>(a, smem, xs, XS, Kc, kcta, lut, redn, nullptr, 0);
+  ws_prologue<true>(a, smem, xs, XS, Kc, kcta, redn, nullptr, 0);
 #endif
 
   // -------------------------------------------------------------- consumers: main loop
@@ -681,7 +677,6 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream_fp4(const __grid_cons
   const int rb = SW ? 8 * rt + g : 16 * rt + g + 8;
   const int ca = ra * 64 + t * 8, cb = (SW ? Q4_CODE_B / 2 : 0) + rb * 64 + t * 8;
   const int sa = Q4_CODE_B + ra * 16 + t, sbo = Q4_CODE_B + (SW ? Q4_SC_B / 2 : 0) + rb * 16 + t;
-  const uint32_t* tab = lut + lane;  // this lane's copy of the table
   int it = 0;
   bool ok = true;
   for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x) {
@@ -714,23 +709,22 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream_fp4(const __grid_cons
           const int off = (hs >> 1) * (RR * 64) + (hs & 1) * 32;
           const uint2 wa = *reinterpret_cast<const uint2*>(sb + ca + off);
           const uint2 wb = *reinterpret_cast<const uint2*>(sb + cb + off);
-          const uint32_t sA = ws_e4m3x2(sb[sa + 4 * hs]), sB = ws_e4m3x2(sb[sbo + 4 * hs]);
+          const uint32_t sA = ws_e4m3_f16x2(sb[sa + 4 * hs]), sB = ws_e4m3_f16x2(sb[sbo + 4 * hs]);
           const int kx = st * Q4_KST + 64 * hs + 16 * t;  // K offset in the block's range
           const uint32_t wA[2] = {wa.x, wa.y}, wB[2] = {wb.x, wb.y};
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
-            uint32_t a01 = tab[(wA[q] & 0xFFu) << 5], a23 = tab[((wA[q] >> 8) & 0xFFu) << 5];
-            uint32_t a45 = tab[((wA[q] >> 16) & 0xFFu) << 5], a67 = tab[(wA[q] >> 24) << 5];
-            uint32_t b01 = tab[(wB[q] & 0xFFu) << 5], b23 = tab[((wB[q] >> 8) & 0xFFu) << 5];
-            uint32_t b45 = tab[((wB[q] >> 16) & 0xFFu) << 5], b67 = tab[(wB[q] >> 24) << 5];
-            a01 = ws_hmul2(a01, sA); a23 = ws_hmul2(a23, sA); a45 = ws_hmul2(a45, sA); a67 = ws_hmul2(a67, sA);
-            b01 = ws_hmul2(b01, sB); b23 = ws_hmul2(b23, sB); b45 = ws_hmul2(b45, sB); b67 = ws_hmul2(b67, sB);
+            uint32_t a01, a23, a45, a67, b01, b23, b45, b67;
+            ws_e2m1x8_f16(wA[q], a01, a23, a45, a67);
+            ws_e2m1x8_f16(wB[q], b01, b23, b45, b67);
+            a01 = ws_hmul2_f16(a01, sA); a23 = ws_hmul2_f16(a23, sA); a45 = ws_hmul2_f16(a45, sA); a67 = ws_hmul2_f16(a67, sA);
+            b01 = ws_hmul2_f16(b01, sB); b23 = ws_hmul2_f16(b23, sB); b45 = ws_hmul2_f16(b45, sB); b67 = ws_hmul2_f16(b67, sB);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               const int sr = nt * 8 + g;
               const uint4 xv = *reinterpret_cast<const uint4*>(sr < a.rows ? xs + (size_t)sr * XS + kx + 8 * q : xzero);
-              mma_bf16_16816(acc[nt], a01, b01, a23, b23, xv.x, xv.y);
-              mma_bf16_16816(acc[nt], a45, b45, a67, b67, xv.z, xv.w);
+              mma_f16_16816(acc[nt], a01, b01, a23, b23, xv.x, xv.y);
+              mma_f16_16816(acc[nt], a45, b45, a67, b67, xv.z, xv.w);
             }
           }
         }
@@ -777,7 +771,7 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream_fp4(const __grid_cons
 #endif
 }
 
-inline size_t q4_smem(int NT, int rows, int Kc, int stages) {
+inline size_t q4_smem(int NT, int rows, int Kc, int stages) {  // no code table: expansion is by cvt
   return 1024 + q4_stage_base(rows, Kc) + (size_t)stages * Q4_STAGE_B + (size_t)4 * NT * 32 * 4 * 4 + 2 * stages * 8;
 }
 
@@ -885,7 +879,7 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream_aff(const __grid_cons
     return;
   }
 
-  ws_prologue<false>(a, smem, xs, XS, Kc, kcta, nullptr, redn, nullptr, 0);
+  ws_prologue<false>(a, smem, xs, XS, Kc, kcta, redn, nullptr, 0);
   // sums of the bf16 activations over each group of 64 (the bias term and the 128 + q offset)
   for (int e = tid; e < a.rows * NG; e += WS_CW * 32) {
     const int b = e / NG, gi = e % NG;
@@ -1103,7 +1097,7 @@ cudaError_t affine_to_bf16(const uint8_t* codes, const void* scales, const void*
 template <int EPI, bool FP4>
 size_t ws_smem(int NT, int rows, int Kc, int stages) {
   using G = WsGeom<EPI, FP4>;
-  const size_t x = ws_stage_base(rows, Kc, FP4);
+  const size_t x = ws_stage_base(rows, Kc);
   return 1024 + x + (size_t)stages * G::STAGE_BYTES + (size_t)WS_CW * G::NRT * NT * 128 * 4 +
          (size_t)G::NRT * 16 * NT * 8 * 4 + 2 * stages * 8;
 }
@@ -1165,14 +1159,16 @@ static cudaError_t launch_q4(const WsMaps& mp, const WsArgs& a, cudaStream_t s) 
   const int nunits = a.N / (EPI == GEMV_SWIGLU ? Q4_UR / 2 : Q4_UR);
   const int NT = a.rows <= 8 ? 1 : 2;
   WsArgs b = a;
-  b.stages = Q4_STAGES;
 #ifdef LFM3_TRACE
   b.trace = g_trace;
   b.trace_id = g_launches;
 #endif
+  auto kern = NT == 1 ? k_wstream_fp4<EPI, 1> : k_wstream_fp4<EPI, 2>;
+  // the deepest ring that still lets two blocks share an SM (wide batches hold more activations)
+  b.stages = Q4_STAGES;
+  while (b.stages > Q4_STAGES / 2 && ws_fit(kern, q4_smem(NT, a.rows, Kc, b.stages)) < 2) --b.stages;
   const size_t smem = q4_smem(NT, a.rows, Kc, b.stages);
   if (smem > (size_t)WS_SMEM_MAX) return cudaErrorInvalidValue;
-  auto kern = NT == 1 ? k_wstream_fp4<EPI, 1> : k_wstream_fp4<EPI, 2>;
   int gx = std::max(1, ws_fit(kern, smem) * g_num_sms / a.splits);
   gx = std::min(gx, nunits);
   const int per = (nunits + gx - 1) / gx;
