@@ -103,17 +103,23 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
 #endif
 
   // ---- queries and the new key / value (threads 0..127: thread = dimension d of each head)
-  const float* raw = qkvg + (size_t)b * NQKVG;
+  // element i of q|k|v|gate row r: the K-split partials summed in split order
+  auto rawat = [&](int r, int i) {
+    const float* e = qkvg + (size_t)r * NQKVG + i;
+    float v = e[0];
+    for (int p = 1; p < A.n_parts; ++p) v += e[p * A.part_stride];
+    return v;
+  };
   float qv[GQA], kv = 0.f, vv = 0.f;
   if (tid < HD) {
     float s2[GQA + 1];
 #pragma unroll
     for (int hh = 0; hh < GQA; ++hh) {
-      qv[hh] = raw[(kvh * GQA + hh) * HD + d];
+      qv[hh] = rawat(b, (kvh * GQA + hh) * HD + d);
       s2[hh] = warp_sum(qv[hh] * qv[hh]);
     }
-    kv = raw[HQ * HD + kvh * HD + d];
-    vv = raw[HQ * HD + HKV * HD + kvh * HD + d];
+    kv = rawat(b, HQ * HD + kvh * HD + d);
+    vv = rawat(b, HQ * HD + HKV * HD + kvh * HD + d);
     s2[GQA] = warp_sum(kv * kv);
     if (lane == 0)
 #pragma unroll
@@ -161,11 +167,10 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
     const int pp = pos - wi + ip;
     const int kidx = L.full ? pp : pp % WIN;
     if (kidx < j0 || kidx >= j0 + cnt) continue;  // uniform over the block
-    const float* rw = qkvg + (size_t)(b - wi + ip) * NQKVG;
     float k1 = 0.f, v1 = 0.f;
     if (tid < HD) {
-      k1 = rw[HQ * HD + kvh * HD + d];
-      v1 = rw[HQ * HD + HKV * HD + kvh * HD + d];
+      k1 = rawat(b - wi + ip, HQ * HD + kvh * HD + d);
+      v1 = rawat(b - wi + ip, HQ * HD + HKV * HD + kvh * HD + d);
       const float s2 = warp_sum(k1 * k1);
       if (lane == 0) red[0][warp] = s2;
     }
@@ -331,7 +336,7 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
   if (half == 0) {
     const float4 t = *reinterpret_cast<const float4*>(&obuf[0][hh][4 * lane]);
     const float l = lsum + lx[hh];
-    const float gt = sigmoidf_(raw[HQ * HD + 2 * HKV * HD + kvh * GQA + hh]) / l;
+    const float gt = sigmoidf_(rawat(b, HQ * HD + 2 * HKV * HD + kvh * GQA + hh)) / l;
     bf16* yo = y + (size_t)b * HQ * HD + (kvh * GQA + hh) * HD + 4 * lane;
     uint2 w;
     w.x = pack_bf2(gt * (acc.x + t.x), gt * (acc.y + t.y));

@@ -136,19 +136,25 @@ cudaError_t resid_norm(float* x_res, const float* part, int n_part, long part_st
 // in_proj output (fp32 accumulators), bx = bf16(B * x); over win = [state(6) | bx], z_t = sum_k w[c][k] win[t+k]
 // (tap 6 on the newest column); y = bf16(C * z); the new state is win[n : n + 6].
 // Decode: one row per stream, state [slot][6][D] shifts by one column.
-__global__ void __launch_bounds__(256) k_conv_decode(const float* __restrict__ bcx, const bf16* __restrict__ conv_w,
-                                                     bf16* __restrict__ state, const int32_t* __restrict__ row_slot,
-                                                     int win, bf16* __restrict__ snap, bf16* __restrict__ y) {
+__global__ void __launch_bounds__(256) k_conv_decode(const float* __restrict__ bcx, int n_parts, long part_stride,
+                                                     const bf16* __restrict__ conv_w, bf16* __restrict__ state,
+                                                     const int32_t* __restrict__ row_slot, int win,
+                                                     bf16* __restrict__ snap, bf16* __restrict__ y) {
   pdl_wait();
   pdl_launch_dependents();
   const int b = blockIdx.y;
   const int c = blockIdx.x * 256 + threadIdx.x;
-  const float* row = bcx + (size_t)b * 3 * D;
-  const float Cv = row[D + c];
+  auto at = [&](int r, int i) {  // column i of in_proj row r: the partials summed in split order
+    const float* e = bcx + (size_t)r * 3 * D + i;
+    float v = e[0];
+    for (int p = 1; p < n_parts; ++p) v += e[p * part_stride];
+    return v;
+  };
+  const float Cv = at(b, D + c);
   bf16* st = state + (size_t)row_slot[b] * CST * D + c;
   const bf16* w = conv_w + (size_t)c * TAPS;
   if (win <= 1) {
-    const float bx = round_bf(row[c] * row[2 * D + c]);
+    const float bx = round_bf(at(b, c) * at(b, 2 * D + c));
     float win6[CST];
 #pragma unroll
     for (int j = 0; j < CST; ++j) win6[j] = bf2f(st[(size_t)j * D]);
@@ -167,10 +173,7 @@ __global__ void __launch_bounds__(256) k_conv_decode(const float* __restrict__ b
   float wnd[CST + MAX_WIN];
 #pragma unroll
   for (int j = 0; j < CST; ++j) wnd[j] = bf2f(st[(size_t)j * D]);
-  for (int i = 0; i <= wi; ++i) {
-    const float* ri = bcx + (size_t)(b0 + i) * 3 * D;
-    wnd[CST + i] = round_bf(ri[c] * ri[2 * D + c]);
-  }
+  for (int i = 0; i <= wi; ++i) wnd[CST + i] = round_bf(at(b0 + i, c) * at(b0 + i, 2 * D + c));
   float z = 0.f;
 #pragma unroll
   for (int k = 0; k < TAPS; ++k) z += bf2f(w[k]) * wnd[wi + k];
@@ -179,9 +182,10 @@ __global__ void __launch_bounds__(256) k_conv_decode(const float* __restrict__ b
   for (int j = 0; j < CST; ++j) snap[((size_t)b * CST + j) * D + c] = f2bf(wnd[wi + 1 + j]);
 }
 
-cudaError_t conv_decode(const float* bcx, const bf16* conv_w, bf16* state_layer, const int32_t* row_slot, int rows,
-                        int win, bf16* snap, bf16* y, cudaStream_t s) {
-  return launch(k_conv_decode, dim3(D / 256, rows), dim3(256), 0, s, bcx, conv_w, state_layer, row_slot, win, snap, y);
+cudaError_t conv_decode(const float* bcx, int n_parts, long part_stride, const bf16* conv_w, bf16* state_layer,
+                        const int32_t* row_slot, int rows, int win, bf16* snap, bf16* y, cudaStream_t s) {
+  return launch(k_conv_decode, dim3(D / 256, rows), dim3(256), 0, s, bcx, n_parts, part_stride, conv_w, state_layer,
+                row_slot, win, snap, y);
 }
 
 // Prefill: n consecutive rows of one slot. Block (channel group, row group of 32). Only the

@@ -158,7 +158,23 @@ struct GemmArgs {
   void* out;
   float alpha;
   int* err;
+  int splits;                  // K splits (fp32 partial sums at out + s * M * ld)
+  unsigned long long* amax;    // GEMM_HEAD
 };
+
+// Tile t of a launch: M tiles fastest (consecutive blocks share a weight tile through L2), then
+// N tiles, then K splits; the split's 64-column K blocks are [kb0, kb1).
+struct GemmTile { int m0, n0, s, kb0, kb1; };
+DEVI GemmTile gemm_tile(int t, int num_m, int num_n, int bm, int nout, int nk, int splits) {
+  GemmTile r;
+  r.m0 = (t % num_m) * bm;
+  const int q = t / num_m;
+  r.n0 = (q % num_n) * nout;
+  r.s = q / num_n;
+  r.kb0 = r.s * nk / splits;
+  r.kb1 = (r.s + 1) * nk / splits;
+  return r;
+}
 
 template <int BN>
 struct GemmGeom {
@@ -193,17 +209,32 @@ constexpr uint32_t GM_STG = 4 * GM_STG_WARP;
 // past M (the last tile of a ragged chunk) take plain per-thread stores instead; column chunks past
 // N are skipped, and a chunk that straddles N is clipped by the store.
 template <int BN, int EPI>
-DEVI void gemm_epilogue(uint32_t tbase, int wrow0, int n0, const GemmArgs& g, const CUtensorMap* to, uint32_t stg,
-                        int lane) {
+DEVI void gemm_epilogue(uint32_t tbase, int wrow0, int n0, int split, const GemmArgs& g, const CUtensorMap* to,
+                        uint32_t stg, int lane) {
   constexpr int NOUT = EPI == GEMM_SWIGLU ? BN / 2 : BN;
-  constexpr int CPC = EPI == GEMM_F32 ? 32 : 64;  // output columns per 128-byte row segment
+  constexpr int CPC = (EPI == GEMM_F32 || EPI == GEMM_HEAD) ? 32 : 64;  // output columns per 128-byte row segment
   const int row = wrow0 + lane;
-  const bool staged = wrow0 + 32 <= g.M;
+  // K-split partial sums and head logits take plain stores (no output map covers them)
+  const bool staged = wrow0 + 32 <= g.M && g.splits == 1 && EPI != GEMM_HEAD;
+  float best = -INFINITY;  // GEMM_HEAD: this row's maximum over the tile and its first column
+  int best_col = -1;
 #pragma unroll 1
   for (int c = 0; c < NOUT / CPC; ++c) {
     const int col = n0 + c * CPC;
     uint32_t w[32];  // this row's 128 output bytes
-    if constexpr (EPI == GEMM_F32) {
+    if constexpr (EPI == GEMM_HEAD) {
+      float v[32];
+      tmem_ld32(tbase + c * 32, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        w[j] = __float_as_uint(v[j]);
+        if (col + j < g.N && v[j] > best) {  // strictly greater: the first column of a tie
+          best = v[j];
+          best_col = col + j;
+        }
+      }
+      if (g.out == nullptr) continue;
+    } else if constexpr (EPI == GEMM_F32) {
       float v[32];
       tmem_ld32(tbase + c * 32, v);
 #pragma unroll
@@ -237,8 +268,8 @@ DEVI void gemm_epilogue(uint32_t tbase, int wrow0, int n0, const GemmArgs& g, co
         bulk_commit();
       }
     } else if (row < g.M) {
-      if constexpr (EPI == GEMM_F32) {
-        float* dst = reinterpret_cast<float*>(g.out) + (size_t)row * g.ld + col;
+      if constexpr (EPI == GEMM_F32 || EPI == GEMM_HEAD) {
+        float* dst = reinterpret_cast<float*>(g.out) + ((size_t)split * g.M + row) * g.ld + col;
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if (col + j < g.N) dst[j] = __uint_as_float(w[j]);
@@ -248,6 +279,13 @@ DEVI void gemm_epilogue(uint32_t tbase, int wrow0, int n0, const GemmArgs& g, co
         for (int j = 0; j < 32; ++j)  // output widths are even
           if (col + 2 * j < g.N) dst[j] = w[j];
       }
+    }
+  }
+  if constexpr (EPI == GEMM_HEAD) {
+    if (row < g.M && best_col >= 0) {
+      uint32_t u = __float_as_uint(best);
+      u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+      atomicMax(g.amax + row, ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)best_col));
     }
   }
 }
@@ -273,7 +311,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_m = (g.M + GM_BM - 1) / GM_BM, num_n = (g.N + NOUT - 1) / NOUT;
-  const int ntiles = num_m * num_n;
+  const int ntiles = num_m * num_n * g.splits;
   const int nk = g.K / GM_BK;
 
   if (threadIdx.x == 0) {
@@ -307,8 +345,9 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % num_m) * GM_BM, n0 = (tile / num_m) * NOUT;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        const GemmTile T = gemm_tile(tile, num_m, num_n, GM_BM, NOUT, nk, g.splits);
+        const int m0 = T.m0, n0 = T.n0;
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
           if (!mbar_wait(empty0 + 8 * s, ph ^ 1, g.err)) {
@@ -318,7 +357,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
           const uint32_t a_s = su32(smem + s * G::STAGE), b_s = a_s + G::A_BYTES;
           mbar_expect_tx(full0 + 8 * s, G::STAGE);
           tma_load_2d(a_s, &ta, kb * GM_BK, m0, full0 + 8 * s);
-          if constexpr (EPI == GEMM_SWIGLU) {
+          if constexpr (EPI == GEMM_SWIGLU) {  // BN / 2 rows of w1, then the same rows of w3
             tma_load_2d(b_s, &tb, kb * GM_BK, n0, full0 + 8 * s);
             tma_load_2d(b_s + G::B_BYTES / 2, &tb3, kb * GM_BK, n0, full0 + 8 * s);
           } else {  // weight boxes are 128 rows: a 256-wide tile takes two
@@ -341,13 +380,14 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
         const int buf = i & 1;
+        const GemmTile T = gemm_tile(tile, num_m, num_n, GM_BM, NOUT, nk, g.splits);
         if (!mbar_wait(acce0 + 8 * buf, ((i >> 1) & 1) ^ 1, g.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t td = tmem + buf * BN;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
           const int s = it % S;
           if (!mbar_wait(full0 + 8 * s, (it / S) & 1, g.err)) {
             ok = false;
@@ -356,7 +396,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
           const uint32_t sa = smem0 + s * G::STAGE;
           const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + G::A_BYTES);
 #pragma unroll
-          for (int k = 0; k < GM_BK / 16; ++k) umma_f16(td, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+          for (int k = 0; k < GM_BK / 16; ++k) umma_f16(td, ad + 2 * k, bd + 2 * k, idesc, (kb != T.kb0 || k) ? 1u : 0u);
           umma_commit(empty0 + 8 * s);
         }
         if (ok) umma_commit(accf0 + 8 * buf);
@@ -376,12 +416,12 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
       const int buf = i & 1;
-      const int m0 = (tile % num_m) * GM_BM, n0 = (tile / num_m) * NOUT;
+      const GemmTile T = gemm_tile(tile, num_m, num_n, GM_BM, NOUT, nk, g.splits);
       ok = mbar_wait(accf0 + 8 * buf, (i >> 1) & 1, g.err);
       tc_fence_after();
       if (!ok) break;
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
-      gemm_epilogue<BN, EPI>(tbase, m0 + quarter * 32, n0, g, &to, stg0 + quarter * GM_STG_WARP, lane);
+      gemm_epilogue<BN, EPI>(tbase, T.m0 + quarter * 32, T.n0, T.s, g, &to, stg0 + quarter * GM_STG_WARP, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce0 + 8 * buf);
@@ -572,7 +612,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm2(const __grid_constant__ CUtens
       tc_fence_after();
       if (!ok) break;
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
-      gemm_epilogue<BN, EPI>(tbase, m0 + quarter * 32, n0, g, &to, stg0 + quarter * GM_STG_WARP, lane);
+      gemm_epilogue<BN, EPI>(tbase, m0 + quarter * 32, n0, 0, g, &to, stg0 + quarter * GM_STG_WARP, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(peer_addr(acce0 + 8 * buf, 0));
@@ -600,11 +640,15 @@ template <int BN, int EPI>
 static cudaError_t launch_gemm(const GemmPlan& p, int M, int* err, cudaStream_t s) {
   constexpr size_t smem = gemm_smem<BN>();
   auto k = k_gemm<BN, EPI>;
-  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err};
+  const int splits = EPI == GEMM_F32 ? std::max(1, p.splits) : 1;
+  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, splits, p.amax};
   const int ntile = EPI == GEMM_SWIGLU ? BN / 2 : BN;
-  const int tiles = ((p.N + ntile - 1) / ntile) * ((M + GM_BM - 1) / GM_BM);
+  const int tiles = ((p.N + ntile - 1) / ntile) * ((M + GM_BM - 1) / GM_BM) * splits;
   dim3 grid(std::min(tiles, g_gemm_sms > 0 ? g_gemm_sms : 148));
-  return launch(k, grid, dim3(192), smem, s, p.a, p.b, EPI == GEMM_SWIGLU ? p.b3 : p.b, p.o, g);
+  // a 128-column SwiGLU tile takes w1 and w3 in boxes of 64 rows
+  const CUtensorMap& b1 = (EPI == GEMM_SWIGLU && BN == 128) ? p.bh : p.b;
+  const CUtensorMap& b3 = EPI == GEMM_SWIGLU ? (BN == 128 ? p.b3h : p.b3) : p.b;
+  return launch(k, grid, dim3(192), smem, s, p.a, b1, b3, p.o, g);
 }
 
 template <int BN>
@@ -631,7 +675,7 @@ template <int EPI>
 static cudaError_t launch_gemm2(const GemmPlan& p, int M, int* err, cudaStream_t s) {
   constexpr int BN = 256;
   constexpr int ntile = EPI == GEMM_SWIGLU ? BN / 2 : BN;
-  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err};
+  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, 1, nullptr};
   const int tiles = ((p.N + ntile - 1) / ntile) * ((M + 2 * GM_BM - 1) / (2 * GM_BM));
   cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config(std::min(tiles, g_gemm_pairs), gemm2_smem<BN>(), s, attr);
@@ -658,6 +702,10 @@ cudaError_t gemm_init() {
     return e;
   if ((e = cudaFuncSetAttribute(k_gemm<256, GEMM_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem<256>())))
     return e;
+  if ((e = cudaFuncSetAttribute(k_gemm<128, GEMM_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem<128>())))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_gemm<128, GEMM_HEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem<128>())))
+    return e;
   if ((e = cudaFuncSetAttribute(k_gemm2<256, GEMM_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm2_smem<256>())))
     return e;
   if ((e = cudaFuncSetAttribute(k_gemm2<256, GEMM_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm2_smem<256>())))
@@ -680,6 +728,18 @@ bool gemm_wide(int N) { return N >= g_gemm_wide_min; }
 
 cudaError_t gemm(const GemmPlan& p, int M, int* err, cudaStream_t s) {
   if (p.K % GM_BK) return cudaErrorInvalidValue;
+  if (p.splits > 1 && (p.epi != GEMM_F32 || M > GM_BM || p.splits > p.K / GM_BK)) return cudaErrorInvalidValue;
+  if (p.epi == GEMM_HEAD) return p.amax ? launch_gemm<128, GEMM_HEAD>(p, M, err, s) : cudaErrorInvalidValue;
+  if (M <= GM_BM) {
+    // one row tile (a batch of decode rows): 128-column weight tiles, so that more of them stream
+    // at once; fp32 outputs may also be split along K
+    switch (p.epi) {
+      case GEMM_F32: return launch_gemm<128, GEMM_F32>(p, M, err, s);
+      case GEMM_BF16: return launch_gemm<128, GEMM_BF16>(p, M, err, s);
+      case GEMM_SWIGLU: return launch_gemm<128, GEMM_SWIGLU>(p, M, err, s);
+    }
+    return cudaErrorInvalidValue;
+  }
   if (M >= g_gemm_pair_min_m && (p.epi == GEMM_SWIGLU || p.N >= 4096 || p.K >= 4096)) {
     switch (p.epi) {
       case GEMM_F32: return launch_gemm2<GEMM_F32>(p, M, err, s);

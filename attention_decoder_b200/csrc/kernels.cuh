@@ -64,8 +64,9 @@ cudaError_t resid_norm(float* x_res, const float* part, int n_part, long part_st
                        const bf16* g_next, bf16* xn, int rows, float eps, float* dump, cudaStream_t s);
 // one row per stream (win 1: the state shifts), or verify windows of `win` rows per stream (the
 // state is left alone; the state after each row goes to snap [rows][CST][D])
-cudaError_t conv_decode(const float* bcx, const bf16* conv_w, bf16* state_layer, const int32_t* row_slot,
-                        int rows, int win, bf16* snap, bf16* y, cudaStream_t s);
+// bcx: the in_proj rows as the sum of n_parts K-split partials, part_stride floats apart
+cudaError_t conv_decode(const float* bcx, int n_parts, long part_stride, const bf16* conv_w, bf16* state_layer,
+                        const int32_t* row_slot, int rows, int win, bf16* snap, bf16* y, cudaStream_t s);
 // n rows; the new state is columns [n_state, n_state + 6) of [state | bx] (n_state <= n)
 cudaError_t conv_prefill(const float* bcx, const bf16* conv_w, bf16* state_slot, int n, int n_state, bf16* y,
                          cudaStream_t s);
@@ -188,6 +189,9 @@ struct AttnDecodeArgs {
   int win;
   bf16* side_k;
   bf16* side_v;
+  // the q|k|v|gate rows are the sum of n_parts K-split partials, part_stride floats apart (>= 1)
+  int n_parts;
+  long part_stride;
 #ifdef LFM3_TRACE
   unsigned long long* trace;
   int trace_id;
@@ -218,16 +222,23 @@ cudaError_t attn_prefill_tc(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             cudaStream_t s);
 
 // ---------------------------------------------------------------- tensor-core GEMM (prefill)
-enum GemmEpi { GEMM_F32 = 0, GEMM_BF16 = 1, GEMM_SWIGLU = 2 };
+// GEMM_HEAD: fp32 logits (optional) and the per-row argmax of the tied head, as the packed key
+// of the weight-streaming head (see the HEAD epilogue there).
+enum GemmEpi { GEMM_F32 = 0, GEMM_BF16 = 1, GEMM_SWIGLU = 2, GEMM_HEAD = 3 };
 struct GemmPlan {
   CUtensorMap a;      // activations [M][K] bf16, box 64 x 128
   CUtensorMap b;      // weights [N][K] bf16 (SwiGLU: w1)
   CUtensorMap b3;     // SwiGLU: w3
+  CUtensorMap bh, b3h;  // SwiGLU with 128-column tiles: w1 and w3 in 64-row boxes
   CUtensorMap o;      // output [M][ld] (fp32, or bf16), 32-row boxes of 128 bytes for TMA stores
   int epi, M, N, K;
-  void* out;          // fp32 or bf16 [M][ld]
+  void* out;          // fp32 or bf16 [M][ld]; GEMM_HEAD: logits [M][N] or null
   int ld;
   float alpha;        // scales the accumulator (NVFP4 tensor scale; 1 otherwise)
+  // set per call (defaults 1 / 0 / null): K splits of an fp32 output, written as partial sums to
+  // out + s * M * ld (plain stores); the argmax keys of GEMM_HEAD
+  int splits;
+  unsigned long long* amax;
 };
 bool tma_init();
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);

@@ -63,6 +63,7 @@ struct lfm3_ctx {
   bf16* deq = nullptr;
   std::vector<LayerPlan> plans;
   GemmPlan deq_w13, deq_w2;  // NVFP4: maps over the dequantised weights (b, b3)
+  GemmPlan head_gemm;        // decode batches over 16 rows: the tied head with the argmax epilogue
   CUtensorMap tm_q, tm_sk, tm_sv;  // prefill attention: q rows, sliding scratch K / V
   WsMaps ws_head;                  // decode: tied head
   unsigned* attn_cnt = nullptr;    // workspace: decode attention split counts [max_batch][n_kv]
@@ -276,12 +277,31 @@ bool plan_gemm(GemmPlan* p, int epi, const void* a, int a_rows, const void* b, c
   p->out = out;
   p->ld = ld;
   p->alpha = alpha;
+  p->splits = 1;
+  p->amax = nullptr;
   const uint32_t box_b = 128;  // weight boxes: 128 rows (wide and paired tiles issue several)
   if (!make_tmap_bf16(&p->a, a, a_rows, K, 128)) return false;
   if (!make_tmap_bf16(&p->b, b, N, K, box_b)) return false;
   if (b3 && !make_tmap_bf16(&p->b3, b3, N, K, box_b)) return false;
   if (!b3) p->b3 = p->b;
+  p->bh = p->b;
+  p->b3h = p->b3;
+  if (epi == GEMM_SWIGLU && (!make_tmap_bf16(&p->bh, b, N, K, 64) || !make_tmap_bf16(&p->b3h, b3, N, K, 64)))
+    return false;
+  if (epi == GEMM_HEAD) return true;  // logits take plain stores
   return make_tmap_out(&p->o, out, epi == GEMM_F32, a_rows, N, ld);
+}
+
+// K splits for an fp32 projection of a decode batch (one 128-row tile): enough 128-column tiles x
+// splits to give every SM one, at most SPLIT_MAX and one 64-column K block per split.
+int batch_splits(int N, int K) {
+  const int tiles = (N + 127) / 128;
+  return std::max(1, std::min({SPLIT_MAX, K / 64, 148 / tiles}));
+}
+GemmPlan split_plan(const GemmPlan& p, int splits) {
+  GemmPlan q = p;
+  q.splits = splits;
+  return q;
 }
 
 // Host check that every position a call writes or reads in slot s, [0, end), has a page.
@@ -353,8 +373,9 @@ AttnLayer attn_layer(lfm3_ctx* ctx, const lfm3_state* st, int l, const Views& v)
   return a;
 }
 
-// FFN of n rows (prefill or large-batch decode) on the tensor-core GEMM: u = SwiGLU -> big, w2 -> part.
-lfm3_status ffn_gemm(lfm3_ctx* ctx, int l, int n, cudaStream_t s) {
+// FFN of n rows (prefill or large-batch decode) on the tensor-core GEMM: u = SwiGLU -> big, w2 ->
+// part (as w2_splits K-split partials, n rows apart).
+lfm3_status ffn_gemm(lfm3_ctx* ctx, int l, int n, int w2_splits, cudaStream_t s) {
   const lfm3_layer_weights& W = ctx->L[l];
   if (ctx->cfg.ffn_format == LFM3_FFN_AFFINE) {
     const int bits = ctx->cfg.ffn_bits;
@@ -362,7 +383,7 @@ lfm3_status ffn_gemm(lfm3_ctx* ctx, int l, int n, cudaStream_t s) {
     CK(affine_to_bf16(W.w3_codes, W.w3_scales, W.w3_biases, bits, F, D, ctx->deq + (size_t)F * D, s));
     CK(run_gemm(ctx, ctx->deq_w13, n, s));
     CK(affine_to_bf16(W.w2_codes, W.w2_scales, W.w2_biases, bits, D, F, ctx->deq, s));
-    CK(run_gemm(ctx, ctx->deq_w2, n, s));
+    CK(run_gemm(ctx, split_plan(ctx->deq_w2, w2_splits), n, s));
   } else if (ctx->cfg.ffn_format == LFM3_FFN_NVFP4) {
     CK(nvfp4_to_bf16(W.w1_codes, W.w1_scales, W.w13_scale, F, D, ctx->deq, s));
     CK(nvfp4_to_bf16(W.w3_codes, W.w3_scales, W.w13_scale, F, D, ctx->deq + (size_t)F * D, s));
@@ -370,12 +391,12 @@ lfm3_status ffn_gemm(lfm3_ctx* ctx, int l, int n, cudaStream_t s) {
     p.alpha = W.w13_scale;
     CK(run_gemm(ctx, p, n, s));
     CK(nvfp4_to_bf16(W.w2_codes, W.w2_scales, W.w2_scale, D, F, ctx->deq, s));
-    GemmPlan p2 = ctx->deq_w2;
+    GemmPlan p2 = split_plan(ctx->deq_w2, w2_splits);
     p2.alpha = W.w2_scale;
     CK(run_gemm(ctx, p2, n, s));
   } else {
     CK(run_gemm(ctx, ctx->plans[l].w13, n, s));
-    CK(run_gemm(ctx, ctx->plans[l].w2, n, s));
+    CK(run_gemm(ctx, split_plan(ctx->plans[l].w2, w2_splits), n, s));
   }
   return LFM3_OK;
 }
@@ -524,6 +545,9 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
       return fail(ctx, LFM3_E_CUDA, "head weight-streaming tensor map encoding failed");
     ctx->ws_head.w3 = ctx->ws_head.s = ctx->ws_head.s3 = ctx->ws_head.w;
   }
+  if (g.has_head && !plan_gemm(&ctx->head_gemm, GEMM_HEAD, ctx->xn, R, ctx->embed, nullptr, g.vocab, D, nullptr,
+                                g.vocab, 1.f))
+    return fail(ctx, LFM3_E_CUDA, "head GEMM tensor map encoding failed");
   if (g.ffn_format != LFM3_FFN_BF16) {
     bool ok = plan_gemm(&ctx->deq_w13, GEMM_SWIGLU, ctx->xn, R, ctx->deq, ctx->deq + (size_t)F * D, F, D, ctx->big, F, 1.f);
     ok &= plan_gemm(&ctx->deq_w2, GEMM_F32, ctx->big, R, ctx->deq, nullptr, D, F, ctx->part, D, 1.f);
@@ -625,7 +649,7 @@ lfm3_status prefill_rows(lfm3_ctx* ctx, const lfm3_state* st, int slot, const in
         CK(run_gemm(ctx, P.o_proj, nc, s));
       }
       CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nc, eps, nullptr, s));
-      lfm3_status fs = ffn_gemm(ctx, l, nc, s);
+      lfm3_status fs = ffn_gemm(ctx, l, nc, 1, s);
       if (fs != LFM3_OK) return fs;
       const bf16* gnext = l + 1 < g.n_layers ? B(ctx->L[l + 1].op_norm) : (g.has_head ? ctx->final_norm : nullptr);
       CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_ffn_norm), gnext, ctx->xn, nc, eps,
@@ -689,6 +713,8 @@ AttnDecodeArgs attn_args(lfm3_ctx* ctx, int l, int win) {
   A.counters = ctx->attn_cnt;
   A.err = ctx->err;
   A.win = win;
+  A.n_parts = 1;
+  A.part_stride = 0;
   if (k == 1) {
     const size_t per = (size_t)ctx->cfg.max_batch * HKV * HD;
     A.side_k = ctx->side_k + (size_t)ctx->kidx[l] * per;
@@ -711,42 +737,45 @@ lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, in
     const lfm3_layer_weights& W = ctx->L[l];
     const LayerPlan& P = ctx->plans[l];
     const Views v = views(ctx, st, l);
+    // a batch that fits one 128-row tile splits the projections along K (partials nb rows apart)
+    const bool one = nb <= 128;
+    int sp_o = 1;
     if (g.layer_type[l] == LFM3_LAYER_CONV) {
-      CK(run_gemm(ctx, P.in_proj, nb, s));
-      CK(conv_decode(ctx->part, B(W.conv), v.conv_layer, ctx->row_slot, nb, win,
+      const int sp = one ? batch_splits(3 * D, D) : 1;
+      sp_o = one ? batch_splits(D, D) : 1;
+      CK(run_gemm(ctx, split_plan(P.in_proj, sp), nb, s));
+      CK(conv_decode(ctx->part, sp, (long)nb * 3 * D, B(W.conv), v.conv_layer, ctx->row_slot, nb, win,
                      ctx->conv_snap + (size_t)ctx->kidx[l] * g.max_batch * CST * D, ctx->y, s));
-      CK(run_gemm(ctx, P.out_proj, nb, s));
+      CK(run_gemm(ctx, split_plan(P.out_proj, sp_o), nb, s));
     } else {
       const bool full = g.layer_type[l] == LFM3_LAYER_FULL;
-      CK(run_gemm(ctx, P.qkvg, nb, s));
+      // q|k|v|gate is not split: every attention split block reads its rows (a sum of partials
+      // there costs more than the unsplit projection)
+      const int sp = 1;
+      sp_o = one ? batch_splits(D, HQ * HD) : 1;
+      CK(run_gemm(ctx, split_plan(P.qkvg, sp), nb, s));
       AttnDecodeArgs A = attn_args(ctx, l, win);
+      A.n_parts = sp;
+      A.part_stride = (long)nb * NQKVG;
       CK(attn_decode_fused(ctx->part, rows, attn_layer(ctx, st, l, v), A, full ? splits_full : WIN / DEC_KEYS,
                            attn_part, ctx->y, s));
-      CK(run_gemm(ctx, P.o_proj, nb, s));
+      CK(run_gemm(ctx, split_plan(P.o_proj, sp_o), nb, s));
     }
-    CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nb, eps, nullptr, s));
-    lfm3_status fs = ffn_gemm(ctx, l, nb, s);
+    CK(resid_norm(ctx->x_res, ctx->part, sp_o, (long)nb * D, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nb, eps,
+                  nullptr, s));
+    const int sp_2 = one ? batch_splits(D, F) : 1;
+    lfm3_status fs = ffn_gemm(ctx, l, nb, sp_2, s);
     if (fs != LFM3_OK) return fs;
     const bf16* gnext = l + 1 < g.n_layers ? B(ctx->L[l + 1].op_norm) : (g.has_head ? ctx->final_norm : nullptr);
-    CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_ffn_norm), gnext, ctx->xn, nb, eps,
+    CK(resid_norm(ctx->x_res, ctx->part, sp_2, (long)nb * D, B(W.post_ffn_norm), gnext, ctx->xn, nb, eps,
                   d_hidden ? d_hidden + (size_t)(l + 1) * nb * D : nullptr, s));
   }
   const bool head = g.has_head && (d_logits || d_argmax);
   if (head) {
-    for (int b0 = 0; b0 < nb; b0 += GEMV_MAX_ROWS) {
-      WsArgs a{};
-      a.w = ctx->embed;
-      a.pro = WS_PRO_LOAD;
-      a.x = ctx->xn + (size_t)b0 * D;
-      a.K = D;
-      a.N = g.vocab;
-      a.rows = std::min(GEMV_MAX_ROWS, nb - b0);
-      a.splits = 1;
-      a.logits = d_logits ? d_logits + (size_t)b0 * g.vocab : nullptr;
-      a.amax = ctx->amax + b0;
-      a.err = ctx->err;
-      CK(run_ws(ctx, GEMV_HEAD, WS_BF16, ctx->ws_head, a, s));
-    }
+    GemmPlan h = ctx->head_gemm;  // logits (if asked for) and the argmax keys in one pass
+    h.out = d_logits;
+    h.amax = ctx->amax;
+    CK(run_gemm(ctx, h, nb, s));
   }
   CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr,
                  win == 1, s));
