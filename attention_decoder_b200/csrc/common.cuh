@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #define DEVI __device__ __forceinline__
@@ -80,6 +81,31 @@ DEVI void mma_f16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// bf16x2 -> f16x2 of the same two values (exact within f16's range).
+DEVI uint32_t bf2_to_h2(uint32_t w) {
+  __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// Four bytes of E2M1 code pairs (element 2j in the low nibble of byte j) -> four f16x2, exact.
+DEVI void e2m1x8_to_h2(uint32_t w, uint32_t& c01, uint32_t& c23, uint32_t& c45, uint32_t& c67) {
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+      " cvt.rn.f16x2.e2m1x2 %1, b1;\n cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(c01), "=r"(c23), "=r"(c45), "=r"(c67)
+      : "r"(w));
+}
+// An E4M3 byte -> f16x2 holding its value twice, exact.
+DEVI uint32_t e4m3_to_h2(uint32_t b) {
+  uint32_t r;
+  const uint32_t two = (b & 0xFFu) * 0x0101u;
+  asm("{\n .reg .b16 h;\n cvt.u16.u32 h, %1;\n cvt.rn.f16x2.e4m3x2 %0, h;\n}" : "=r"(r) : "r"(two));
+  return r;
+}
+DEVI uint32_t hmul2_u(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
 DEVI float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }

@@ -72,7 +72,7 @@ cudaError_t embed_rows(const int32_t* tokens, const bf16* table, const bf16* vec
 __global__ void __launch_bounds__(256) k_resid_norm(float* __restrict__ x_res, const float* __restrict__ part,
                                                     int n_part, long part_stride, const bf16* __restrict__ g_post,
                                                     const bf16* __restrict__ g_next, bf16* __restrict__ xn, float eps,
-                                                    float* __restrict__ dump) {
+                                                    float* __restrict__ dump, int xn_f16) {
   __shared__ float red[8];
   pdl_wait();
   pdl_launch_dependents();
@@ -121,14 +121,15 @@ __global__ void __launch_bounds__(256) k_resid_norm(float* __restrict__ x_res, c
     o.y = pack_bf2(g[2] * (x[2] * inv), g[3] * (x[3] * inv));
     o.z = pack_bf2(g[4] * (x[4] * inv), g[5] * (x[5] * inv));
     o.w = pack_bf2(g[6] * (x[6] * inv), g[7] * (x[7] * inv));
+    if (xn_f16) o = make_uint4(bf2_to_h2(o.x), bf2_to_h2(o.y), bf2_to_h2(o.z), bf2_to_h2(o.w));
     stg16(xn + (size_t)r * D + i, o);
   }
 }
 
 cudaError_t resid_norm(float* x_res, const float* part, int n_part, long part_stride, const bf16* g_post,
-                       const bf16* g_next, bf16* xn, int rows, float eps, float* dump, cudaStream_t s) {
+                       const bf16* g_next, bf16* xn, int rows, float eps, float* dump, int xn_f16, cudaStream_t s) {
   return launch(k_resid_norm, dim3(rows), dim3(256), 0, s, x_res, part, n_part, part_stride, g_post, g_next, xn,
-                eps, dump);
+                eps, dump, xn_f16);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -160,6 +160,7 @@ struct GemmArgs {
   int* err;
   int splits;                  // K splits (fp32 partial sums at out + s * M * ld)
   unsigned long long* amax;    // GEMM_HEAD
+  int f16out;                  // GEMM_SWIGLU: the bf16-rounded products stored as f16
 };
 
 // Tile t of a launch: M tiles fastest (consecutive blocks share a weight tile through L2), then
@@ -252,6 +253,9 @@ DEVI void gemm_epilogue(uint32_t tbase, int wrow0, int n0, int split, const Gemm
       for (int j = 0; j < 32; ++j)
         w[j] = pack_bf2(silu_fast(g.alpha * va[2 * j]) * (g.alpha * vb[2 * j]),
                         silu_fast(g.alpha * va[2 * j + 1]) * (g.alpha * vb[2 * j + 1]));
+      if (g.f16out)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) w[j] = bf2_to_h2(w[j]);
     }
     if (col >= g.N) continue;  // the same for the whole warp
     if (staged) {
@@ -641,7 +645,7 @@ static cudaError_t launch_gemm(const GemmPlan& p, int M, int* err, cudaStream_t 
   constexpr size_t smem = gemm_smem<BN>();
   auto k = k_gemm<BN, EPI>;
   const int splits = EPI == GEMM_F32 ? std::max(1, p.splits) : 1;
-  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, splits, p.amax};
+  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, splits, p.amax, 0};
   const int ntile = EPI == GEMM_SWIGLU ? BN / 2 : BN;
   const int tiles = ((p.N + ntile - 1) / ntile) * ((M + GM_BM - 1) / GM_BM) * splits;
   dim3 grid(std::min(tiles, g_gemm_sms > 0 ? g_gemm_sms : 148));
@@ -675,12 +679,266 @@ template <int EPI>
 static cudaError_t launch_gemm2(const GemmPlan& p, int M, int* err, cudaStream_t s) {
   constexpr int BN = 256;
   constexpr int ntile = EPI == GEMM_SWIGLU ? BN / 2 : BN;
-  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, 1, nullptr};
+  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, 1, nullptr, 0};
   const int tiles = ((p.N + ntile - 1) / ntile) * ((M + 2 * GM_BM - 1) / (2 * GM_BM));
   cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config(std::min(tiles, g_gemm_pairs), gemm2_smem<BN>(), s, attr);
   ++g_launches;
   return cudaLaunchKernelEx(&cfg, k_gemm2<BN, EPI>, p.a, p.b, EPI == GEMM_SWIGLU ? p.b3 : p.b, p.o, g);
+}
+
+// ---------------------------------------------------------------- NVFP4 weights (128-column tiles)
+// The weight operand is expanded on the chip: warp 0 streams each tile's E2M1 codes (128 rows x
+// 64 K = 4 KB per K block) through a 16-deep ring, four expansion warps turn a block into the f16
+// operand tile (code pairs by the hardware E2M1 conversion, times the block's E4M3 scale: both
+// exact in f16, and so is their product) in the 128-byte-swizzled layout the MMA reads, and warp
+// 10 streams the activations, which are f16 copies of the bf16 values. kind::f16 with f16
+// operands, fp32 accumulation, the tensor scale as alpha. Warps 1 (MMA) and 2..5 (epilogue) work
+// as in k_gemm. SwiGLU tiles are 64 rows of w1 over 64 rows of w3.
+constexpr int Q4G_S = 3;                    // operand stages (activations + expanded weights)
+constexpr int Q4G_RS = 16;                  // code stages
+constexpr uint32_t Q4G_AB = 128 * GM_BK * 2;  // one operand stage: 128 rows x 64 K
+constexpr uint32_t Q4G_RAW = 128 * GM_BK / 2; // codes of 128 rows x 64 K
+constexpr int Q4G_THREADS = 11 * 32;
+constexpr size_t q4g_smem() { return 1024 + 2 * Q4G_S * Q4G_AB + Q4G_RS * Q4G_RAW + GM_STG + 512; }
+
+template <int EPI>
+__global__ void __launch_bounds__(Q4G_THREADS, 1) k_gemm_q4(const __grid_constant__ CUtensorMap ta,
+                                                            const __grid_constant__ CUtensorMap tq,
+                                                            const __grid_constant__ CUtensorMap tq3,
+                                                            const __grid_constant__ CUtensorMap to, const GemmArgs g,
+                                                            const uint8_t* __restrict__ sc,
+                                                            const uint8_t* __restrict__ sc3) {
+  constexpr int BN = 128;
+  constexpr bool SW = EPI == GEMM_SWIGLU;
+  constexpr int NOUT = SW ? BN / 2 : BN;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* ra = smem;                             // activations [S][128 rows][128 B]
+  unsigned char* rb = smem + Q4G_S * Q4G_AB;            // expanded weights [S][128 rows][128 B]
+  unsigned char* rc = smem + 2 * Q4G_S * Q4G_AB;        // codes [RS][128 rows][32 B]
+  const uint32_t stg0 = su32(rc + Q4G_RS * Q4G_RAW);    // epilogue staging (GM_STG bytes)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rc + Q4G_RS * Q4G_RAW + GM_STG);
+  const uint32_t a_full = su32(bars), b_full = a_full + 8 * Q4G_S, ab_empty = b_full + 8 * Q4G_S;
+  const uint32_t r_full = ab_empty + 8 * Q4G_S, r_empty = r_full + 8 * Q4G_RS;
+  const uint32_t accf0 = r_empty + 8 * Q4G_RS, acce0 = accf0 + 16, fin = acce0 + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * Q4G_S + 2 * Q4G_RS + 5);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (g.M + GM_BM - 1) / GM_BM, num_n = (g.N + NOUT - 1) / NOUT;
+  const int ntiles = num_m * num_n * g.splits;
+  const int nk = g.K / GM_BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Q4G_S; ++s) {
+      mbar_init(a_full + 8 * s, 1);
+      mbar_init(b_full + 8 * s, 4);
+      mbar_init(ab_empty + 8 * s, 1);
+    }
+    for (int r = 0; r < Q4G_RS; ++r) {
+      mbar_init(r_full + 8 * r, 1);
+      mbar_init(r_empty + 8 * r, 4);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf0 + 8 * b, 1);
+      mbar_init(acce0 + 8 * b, 4);
+    }
+    mbar_init(fin, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(tmem_slot)),
+                 "r"(2 * BN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ codes (constants: streamed before the wait)
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const GemmTile T = gemm_tile(tile, num_m, num_n, GM_BM, NOUT, nk, g.splits);
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
+          const int r = it % Q4G_RS;
+          if (!mbar_wait(r_empty + 8 * r, ((it / Q4G_RS) & 1) ^ 1, g.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = su32(rc + r * Q4G_RAW);
+          mbar_expect_tx(r_full + 8 * r, Q4G_RAW);
+          if constexpr (SW) {
+            tma_load_2d(dst, &tq, kb * (GM_BK / 2), T.n0, r_full + 8 * r);
+            tma_load_2d(dst + Q4G_RAW / 2, &tq3, kb * (GM_BK / 2), T.n0, r_full + 8 * r);
+          } else {
+            tma_load_2d(dst, &tq, kb * (GM_BK / 2), T.n0, r_full + 8 * r);
+          }
+        }
+      }
+      // every copy issued has landed before the block can exit (bounded)
+      for (int d = 1; d <= Q4G_RS && d <= it; ++d) mbar_wait(r_full + 8 * ((it - d) % Q4G_RS), ((it - d) / Q4G_RS) & 1, g.err);
+    }
+    pdl_wait();
+    pdl_launch_dependents();
+  } else if (warp == 10) {
+    // ------------------------------------------------ activations (written by the previous kernel)
+    pdl_wait();
+    pdl_launch_dependents();
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const GemmTile T = gemm_tile(tile, num_m, num_n, GM_BM, NOUT, nk, g.splits);
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
+          const int s = it % Q4G_S;
+          if (!mbar_wait(ab_empty + 8 * s, ((it / Q4G_S) & 1) ^ 1, g.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(a_full + 8 * s, Q4G_AB);
+          tma_load_2d(su32(ra + s * Q4G_AB), &ta, kb * GM_BK, T.m0, a_full + 8 * s);
+        }
+      }
+      for (int d = 1; d <= Q4G_S && d <= it; ++d) mbar_wait(a_full + 8 * ((it - d) % Q4G_S), ((it - d) / Q4G_S) & 1, g.err);
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------ expansion: thread c = row c of the tile
+    pdl_wait();
+    pdl_launch_dependents();
+    const int c = threadIdx.x - 6 * 32;
+    const uint32_t rowoff = (uint32_t)(c >> 3) * 1024 + (uint32_t)(c & 7) * 128;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      const GemmTile T = gemm_tile(tile, num_m, num_n, GM_BM, NOUT, nk, g.splits);
+      const int wrow = SW ? T.n0 + (c & 63) : T.n0 + c;  // weight row
+      const uint8_t* srow = (SW && c >= 64 ? sc3 : sc) + (size_t)wrow * (g.K / 16);
+      const bool valid = wrow < g.N;  // rows past N: codes are zero-filled, scales read as 0
+      // scales of four K blocks (16 bytes) per load; the next group is requested one group ahead
+      int grp = T.kb0 >> 2;
+      uint4 scv = valid ? ldg16(srow + grp * 16) : make_uint4(0, 0, 0, 0);
+      uint4 scn = (valid && (grp + 1) * 4 < nk) ? ldg16(srow + (grp + 1) * 16) : make_uint4(0, 0, 0, 0);
+      for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
+        if ((kb >> 2) != grp) {
+          grp = kb >> 2;
+          scv = scn;
+          scn = (valid && (grp + 1) * 4 < nk) ? ldg16(srow + (grp + 1) * 16) : make_uint4(0, 0, 0, 0);
+        }
+        const int r = it % Q4G_RS, s = it % Q4G_S;
+        if (!mbar_wait(r_full + 8 * r, (it / Q4G_RS) & 1, g.err) ||
+            !mbar_wait(ab_empty + 8 * s, ((it / Q4G_S) & 1) ^ 1, g.err)) {
+          ok = false;
+          break;
+        }
+        const uint4* cp = reinterpret_cast<const uint4*>(rc + r * Q4G_RAW + c * 32);
+        const uint4 w0 = cp[0], w1 = cp[1];
+        const uint32_t cw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const int kq = kb & 3;  // scales of this K block's four 16-code groups
+        const uint32_t sw4 = kq == 0 ? scv.x : kq == 1 ? scv.y : kq == 2 ? scv.z : scv.w;
+        const uint32_t bs = su32(rb + s * Q4G_AB) + rowoff;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {  // 8 codes -> one 16-byte chunk of the row
+          const uint32_t sc2 = e4m3_to_h2(sw4 >> (8 * (q >> 1)));
+          uint32_t h0, h1, h2, h3;
+          e2m1x8_to_h2(cw[q], h0, h1, h2, h3);
+          sts128(bs + ((uint32_t)(q ^ (c & 7)) << 4),
+                 make_uint4(hmul2_u(h0, sc2), hmul2_u(h1, sc2), hmul2_u(h2, sc2), hmul2_u(h3, sc2)));
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(b_full + 8 * s);
+          mbar_arrive(r_empty + 8 * r);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    pdl_wait();
+    pdl_launch_dependents();
+    if (lane == 0) {
+      constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(GM_BM >> 4) << 24);  // f16 x f16
+      int it = 0, i = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
+        const int buf = i & 1;
+        const GemmTile T = gemm_tile(tile, num_m, num_n, GM_BM, NOUT, nk, g.splits);
+        if (!mbar_wait(acce0 + 8 * buf, ((i >> 1) & 1) ^ 1, g.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t td = tmem + buf * BN;
+        for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
+          const int s = it % Q4G_S;
+          if (!mbar_wait(a_full + 8 * s, (it / Q4G_S) & 1, g.err) || !mbar_wait(b_full + 8 * s, (it / Q4G_S) & 1, g.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(su32(ra + s * Q4G_AB)), bd = sw128_desc(su32(rb + s * Q4G_AB));
+#pragma unroll
+          for (int k = 0; k < GM_BK / 16; ++k) umma_f16(td, ad + 2 * k, bd + 2 * k, idesc, (kb != T.kb0 || k) ? 1u : 0u);
+          umma_commit(ab_empty + 8 * s);
+        }
+        if (ok) umma_commit(accf0 + 8 * buf);
+      }
+      // nothing issued may still run when TMEM is released (bounded)
+      umma_commit(fin);
+      mbar_wait(fin, 0, g.err);
+    }
+  } else {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int quarter = warp & 3;
+    int i = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++i) {
+      const int buf = i & 1;
+      const GemmTile T = gemm_tile(tile, num_m, num_n, GM_BM, NOUT, nk, g.splits);
+      ok = mbar_wait(accf0 + 8 * buf, (i >> 1) & 1, g.err);
+      tc_fence_after();
+      if (!ok) break;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
+      gemm_epilogue<BN, EPI>(tbase, T.m0 + quarter * 32, T.n0, T.s, g, &to, stg0 + quarter * GM_STG_WARP, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce0 + 8 * buf);
+    }
+    if (lane == 0) bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * BN));
+}
+
+template <int EPI>
+static cudaError_t launch_gemm_q4(const GemmPlan& p, int M, int* err, cudaStream_t s) {
+  const int splits = EPI == GEMM_F32 ? std::max(1, p.splits) : 1;
+  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, splits, nullptr, EPI == GEMM_SWIGLU ? 1 : 0};
+  const int ntile = EPI == GEMM_SWIGLU ? 64 : 128;
+  const int tiles = ((p.N + ntile - 1) / ntile) * ((M + GM_BM - 1) / GM_BM) * splits;
+  dim3 grid(std::min(tiles, g_gemm_sms > 0 ? g_gemm_sms : 148));
+  return launch(k_gemm_q4<EPI>, grid, dim3(Q4G_THREADS), q4g_smem(), s, p.a, p.q, EPI == GEMM_SWIGLU ? p.q3 : p.q,
+                p.o, g, p.sc, EPI == GEMM_SWIGLU ? p.sc3 : p.sc);
+}
+
+bool make_tmap_codes(CUtensorMap* m, const void* codes, uint64_t rows, uint64_t K, uint32_t box_rows) {
+  if (!p_encode) return false;
+  const uint64_t cols = K / 2;  // bytes per row
+  if ((reinterpret_cast<uintptr_t>(codes) & 15) || cols % 16) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {GM_BK / 2, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = p_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 // Output widths from which a tile is 256 columns wide (fewer, more L2-efficient tiles) rather than
@@ -706,6 +964,10 @@ cudaError_t gemm_init() {
     return e;
   if ((e = cudaFuncSetAttribute(k_gemm<128, GEMM_HEAD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem<128>())))
     return e;
+  if ((e = cudaFuncSetAttribute(k_gemm_q4<GEMM_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q4g_smem())))
+    return e;
+  if ((e = cudaFuncSetAttribute(k_gemm_q4<GEMM_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q4g_smem())))
+    return e;
   if ((e = cudaFuncSetAttribute(k_gemm2<256, GEMM_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm2_smem<256>())))
     return e;
   if ((e = cudaFuncSetAttribute(k_gemm2<256, GEMM_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm2_smem<256>())))
@@ -730,6 +992,12 @@ cudaError_t gemm(const GemmPlan& p, int M, int* err, cudaStream_t s) {
   if (p.K % GM_BK) return cudaErrorInvalidValue;
   if (p.splits > 1 && (p.epi != GEMM_F32 || M > GM_BM || p.splits > p.K / GM_BK)) return cudaErrorInvalidValue;
   if (p.epi == GEMM_HEAD) return p.amax ? launch_gemm<128, GEMM_HEAD>(p, M, err, s) : cudaErrorInvalidValue;
+  if (p.q4) {
+    if (p.K % 256) return cudaErrorInvalidValue;  // scales are read 16 bytes (4 K blocks) at a time
+    if (p.epi == GEMM_F32) return launch_gemm_q4<GEMM_F32>(p, M, err, s);
+    if (p.epi == GEMM_SWIGLU) return launch_gemm_q4<GEMM_SWIGLU>(p, M, err, s);
+    return cudaErrorInvalidValue;
+  }
   if (M <= GM_BM) {
     // one row tile (a batch of decode rows): 128-column weight tiles, so that more of them stream
     // at once; fp32 outputs may also be split along K
@@ -754,44 +1022,6 @@ cudaError_t gemm(const GemmPlan& p, int M, int* err, cudaStream_t s) {
     case GEMM_SWIGLU: return launch_gemm<256, GEMM_SWIGLU>(p, M, err, s);
   }
   return cudaErrorInvalidValue;
-}
-
-// ---------------------------------------------------------------- NVFP4 -> bf16 (prefill)
-// w = e2m1(code) * e4m3(scale): exact in bf16; the tensor scale is the GEMM's alpha.
-__global__ void __launch_bounds__(256) k_nvfp4_to_bf16(const uint8_t* __restrict__ codes,
-                                                       const uint8_t* __restrict__ scales, long n8, int K,
-                                                       bf16* __restrict__ out) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const long i = (long)blockIdx.x * blockDim.x + threadIdx.x;  // group of 8 weights
-  if (i >= n8) return;
-  const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + i * 4);
-  const long e0 = i * 8;
-  const long row = e0 / K, col = e0 % K;
-  const uint8_t sb = scales[row * (K / 16) + col / 16];
-  const uint32_t se = (sb >> 3) & 0xF, sm = sb & 7;
-  float sc = se == 0 ? (float)sm * (1.0f / 512.0f) : __uint_as_float(((se + 120u) << 23) | (sm << 20));
-  if (sb & 0x80) sc = -sc;
-  // E2M1: exponent field e (bias 1), mantissa m; e == 0 is 0.5 * m
-  auto e2m1 = [](uint32_t c) -> float {
-    const uint32_t e = (c >> 1) & 3, m = c & 1;
-    const float mag = e == 0 ? 0.5f * (float)m : __uint_as_float(((e + 126u) << 23) | (m << 22));
-    return (c & 8) ? -mag : mag;
-  };
-  uint32_t o[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t c0 = (w >> (8 * j)) & 0xF, c1 = (w >> (8 * j + 4)) & 0xF;
-    o[j] = pack_bf2(e2m1(c0) * sc, e2m1(c1) * sc);
-  }
-  reinterpret_cast<uint4*>(out)[i] = make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-cudaError_t nvfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, float tscale, int N, int K, bf16* out,
-                          cudaStream_t s) {
-  (void)tscale;
-  const long n8 = (long)N * K / 8;
-  return launch(k_nvfp4_to_bf16, dim3((unsigned)((n8 + 255) / 256)), dim3(256), 0, s, codes, scales, n8, K, out);
 }
 
 }  // namespace lfm3

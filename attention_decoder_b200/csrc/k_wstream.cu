@@ -102,30 +102,6 @@ DEVI int ws_row(int tile, int rt, int g, int& which) {
   }
 }
 
-// bf16x2 -> f16x2 of the same values (rounding only outside f16's range).
-DEVI uint32_t ws_bf2h(uint32_t w) {
-  __half2 h = __floats2half2_rn(bflo(w), bfhi(w));
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-// Four E2M1 codes pairs (the four bytes of w, element 2b in the low nibble) -> four f16x2, exact.
-DEVI void ws_e2m1x8_f16(uint32_t w, uint32_t& c01, uint32_t& c23, uint32_t& c45, uint32_t& c67) {
-  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n cvt.rn.f16x2.e2m1x2 %0, b0;\n"
-      " cvt.rn.f16x2.e2m1x2 %1, b1;\n cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
-      : "=r"(c01), "=r"(c23), "=r"(c45), "=r"(c67)
-      : "r"(w));
-}
-// An E4M3 byte -> f16x2 holding its value twice, exact.
-DEVI uint32_t ws_e4m3_f16x2(uint32_t b) {
-  uint32_t r;
-  const uint32_t two = (b & 0xFFu) * 0x0101u;
-  asm("{\n .reg .b16 h;\n cvt.u16.u32 h, %1;\n cvt.rn.f16x2.e4m3x2 %0, h;\n}" : "=r"(r) : "r"(two));
-  return r;
-}
-DEVI uint32_t ws_hmul2_f16(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
 
 // Weights are read once per step: their copies carry an evict-first L2 policy, so that the small
 // data every kernel reads right after its dependency (residual, partials, gains, keys and values)
@@ -217,7 +193,7 @@ DEVI void ws_prologue(const WsArgs& a, unsigned char* smem, bf16* xs, int XS, in
     for (int idx = ct; idx < a.rows * chunks; idx += WS_CW * 32) {
       const int b = idx / chunks, c = idx - b * chunks;
       uint4 v = ldg16(a.x + (size_t)b * a.K + kcta + c * 8);
-      if constexpr (X16) v = make_uint4(ws_bf2h(v.x), ws_bf2h(v.y), ws_bf2h(v.z), ws_bf2h(v.w));
+      if constexpr (X16) v = make_uint4(bf2_to_h2(v.x), bf2_to_h2(v.y), bf2_to_h2(v.z), bf2_to_h2(v.w));
       *reinterpret_cast<uint4*>(xs + (size_t)b * XS + c * 8) = v;
     }
   } else {
@@ -297,7 +273,7 @@ DEVI void ws_prologue(const WsArgs& a, unsigned char* smem, bf16* xs, int XS, in
           for (int j = 0; j < 4; ++j) {
             const int e = 8 * h + 2 * j;
             w[j] = pack_bf2(gn[e] * (x[e] * inv), gn[e + 1] * (x[e + 1] * inv));
-            if constexpr (X16) w[j] = ws_bf2h(w[j]);
+            if constexpr (X16) w[j] = bf2_to_h2(w[j]);
           }
           *reinterpret_cast<uint4*>(xs + (size_t)b * XS + (c0 - kcta) + 8 * h) = make_uint4(w[0], w[1], w[2], w[3]);
         }
@@ -709,16 +685,16 @@ __global__ void __launch_bounds__(WS_THREADS, 2) k_wstream_fp4(const __grid_cons
           const int off = (hs >> 1) * (RR * 64) + (hs & 1) * 32;
           const uint2 wa = *reinterpret_cast<const uint2*>(sb + ca + off);
           const uint2 wb = *reinterpret_cast<const uint2*>(sb + cb + off);
-          const uint32_t sA = ws_e4m3_f16x2(sb[sa + 4 * hs]), sB = ws_e4m3_f16x2(sb[sbo + 4 * hs]);
+          const uint32_t sA = e4m3_to_h2(sb[sa + 4 * hs]), sB = e4m3_to_h2(sb[sbo + 4 * hs]);
           const int kx = st * Q4_KST + 64 * hs + 16 * t;  // K offset in the block's range
           const uint32_t wA[2] = {wa.x, wa.y}, wB[2] = {wb.x, wb.y};
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             uint32_t a01, a23, a45, a67, b01, b23, b45, b67;
-            ws_e2m1x8_f16(wA[q], a01, a23, a45, a67);
-            ws_e2m1x8_f16(wB[q], b01, b23, b45, b67);
-            a01 = ws_hmul2_f16(a01, sA); a23 = ws_hmul2_f16(a23, sA); a45 = ws_hmul2_f16(a45, sA); a67 = ws_hmul2_f16(a67, sA);
-            b01 = ws_hmul2_f16(b01, sB); b23 = ws_hmul2_f16(b23, sB); b45 = ws_hmul2_f16(b45, sB); b67 = ws_hmul2_f16(b67, sB);
+            e2m1x8_to_h2(wA[q], a01, a23, a45, a67);
+            e2m1x8_to_h2(wB[q], b01, b23, b45, b67);
+            a01 = hmul2_u(a01, sA); a23 = hmul2_u(a23, sA); a45 = hmul2_u(a45, sA); a67 = hmul2_u(a67, sA);
+            b01 = hmul2_u(b01, sB); b23 = hmul2_u(b23, sB); b45 = hmul2_u(b45, sB); b67 = hmul2_u(b67, sB);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               const int sr = nt * 8 + g;

@@ -59,9 +59,10 @@ cudaError_t setup_rows(int prefill, int slot, const int32_t* d_slots, const int3
                        int32_t* row_slot, int32_t* row_pos, unsigned long long* amax, cudaStream_t s);
 cudaError_t embed_rows(const int32_t* tokens, const bf16* table, const bf16* vecs, int rows, float* x_res,
                        float* dump, cudaStream_t s);
-// x_res[r] += g_post * RMS(sum_s part[s][r]) (if n_part > 0); dump x_res; xn = g_next * RMS(x_res)
+// x_res[r] += g_post * RMS(sum_s part[s][r]) (if n_part > 0); dump x_res; xn = g_next * RMS(x_res),
+// rounded to bf16 and stored as bf16, or (xn_f16) as the f16 of that bf16 value
 cudaError_t resid_norm(float* x_res, const float* part, int n_part, long part_stride, const bf16* g_post,
-                       const bf16* g_next, bf16* xn, int rows, float eps, float* dump, cudaStream_t s);
+                       const bf16* g_next, bf16* xn, int rows, float eps, float* dump, int xn_f16, cudaStream_t s);
 // one row per stream (win 1: the state shifts), or verify windows of `win` rows per stream (the
 // state is left alone; the state after each row goes to snap [rows][CST][D])
 // bcx: the in_proj rows as the sum of n_parts K-split partials, part_stride floats apart
@@ -239,7 +240,14 @@ struct GemmPlan {
   // out + s * M * ld (plain stores); the argmax keys of GEMM_HEAD
   int splits;
   unsigned long long* amax;
+  // NVFP4 weights (q4 = 1): codes [N][K/2] in 64-row (SwiGLU: w1 and w3) or 128-row boxes of one
+  // K block, E4M3 scales [N][K/16]; the activations (a) are f16 and the SwiGLU output is f16
+  int q4;
+  CUtensorMap q, q3;
+  const uint8_t* sc;
+  const uint8_t* sc3;
 };
+bool make_tmap_codes(CUtensorMap* m, const void* codes, uint64_t rows, uint64_t K, uint32_t box_rows);
 bool tma_init();
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 // Output map of a GEMM: [rows][cols] with row pitch ld elements, fp32 (32-column boxes) or bf16
@@ -248,8 +256,5 @@ bool make_tmap_out(CUtensorMap* m, void* base, bool fp32, uint64_t rows, uint64_
 cudaError_t gemm(const GemmPlan& p, int M, int* err, cudaStream_t s);
 bool gemm_wide(int N);  // 256-column tiles for this output width
 cudaError_t gemm_init();
-// NVFP4 prefill: dequantise a weight to bf16 [N][K] in scratch, then run the bf16 GEMM.
-cudaError_t nvfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, float tscale, int N, int K, bf16* out,
-                          cudaStream_t s);
 
 }  // namespace lfm3

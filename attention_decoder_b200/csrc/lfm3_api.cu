@@ -62,7 +62,7 @@ struct lfm3_ctx {
   float* rope_sin[2] = {nullptr, nullptr};
   bf16* deq = nullptr;
   std::vector<LayerPlan> plans;
-  GemmPlan deq_w13, deq_w2;  // NVFP4: maps over the dequantised weights (b, b3)
+  GemmPlan deq_w13, deq_w2;  // affine: maps over the expanded bf16 weights (b, b3)
   GemmPlan head_gemm;        // decode batches over 16 rows: the tied head with the argmax epilogue
   CUtensorMap tm_q, tm_sk, tm_sv;  // prefill attention: q rows, sliding scratch K / V
   WsMaps ws_head;                  // decode: tied head
@@ -144,7 +144,7 @@ size_t layout(lfm3_ctx* c, char* base) {
     c->rope_cos[k] = reinterpret_cast<float*>(take(4 * (size_t)c->max_pos * (HD / 2)));
     c->rope_sin[k] = reinterpret_cast<float*>(take(4 * (size_t)c->max_pos * (HD / 2)));
   }
-  c->deq = g.ffn_format != LFM3_FFN_BF16 ? reinterpret_cast<bf16*>(take(2 * (size_t)2 * F * D)) : nullptr;
+  c->deq = g.ffn_format == LFM3_FFN_AFFINE ? reinterpret_cast<bf16*>(take(2 * (size_t)2 * F * D)) : nullptr;
   c->attn_cnt = reinterpret_cast<unsigned*>(take(4 * (size_t)g.max_batch * HKV));
   c->conv_snap = reinterpret_cast<bf16*>(take(2 * (size_t)c->n_conv * g.max_batch * CST * D));
   c->side_k = reinterpret_cast<bf16*>(take(2 * (size_t)c->n_sliding * g.max_batch * HKV * HD));
@@ -279,6 +279,8 @@ bool plan_gemm(GemmPlan* p, int epi, const void* a, int a_rows, const void* b, c
   p->alpha = alpha;
   p->splits = 1;
   p->amax = nullptr;
+  p->q4 = 0;
+  p->sc = p->sc3 = nullptr;
   const uint32_t box_b = 128;  // weight boxes: 128 rows (wide and paired tiles issue several)
   if (!make_tmap_bf16(&p->a, a, a_rows, K, 128)) return false;
   if (!make_tmap_bf16(&p->b, b, N, K, box_b)) return false;
@@ -289,6 +291,30 @@ bool plan_gemm(GemmPlan* p, int epi, const void* a, int a_rows, const void* b, c
   if (epi == GEMM_SWIGLU && (!make_tmap_bf16(&p->bh, b, N, K, 64) || !make_tmap_bf16(&p->b3h, b3, N, K, 64)))
     return false;
   if (epi == GEMM_HEAD) return true;  // logits take plain stores
+  return make_tmap_out(&p->o, out, epi == GEMM_F32, a_rows, N, ld);
+}
+
+// NVFP4 weights expanded on the chip (k_gemm_q4): activations a are f16 [a_rows][K].
+bool plan_gemm_q4(GemmPlan* p, int epi, const void* a, int a_rows, const uint8_t* codes, const uint8_t* scales,
+                  const uint8_t* codes3, const uint8_t* scales3, int N, int K, void* out, int ld, float alpha) {
+  p->epi = epi;
+  p->N = N;
+  p->K = K;
+  p->M = a_rows;
+  p->out = out;
+  p->ld = ld;
+  p->alpha = alpha;
+  p->splits = 1;
+  p->amax = nullptr;
+  p->q4 = 1;
+  p->sc = scales;
+  p->sc3 = scales3 ? scales3 : scales;
+  const uint32_t box = epi == GEMM_SWIGLU ? 64 : 128;
+  if (!make_tmap_bf16(&p->a, a, a_rows, K, 128)) return false;
+  if (!make_tmap_codes(&p->q, codes, N, K, box)) return false;
+  p->q3 = p->q;
+  if (codes3 && !make_tmap_codes(&p->q3, codes3, N, K, box)) return false;
+  p->b = p->b3 = p->bh = p->b3h = p->a;  // unused
   return make_tmap_out(&p->o, out, epi == GEMM_F32, a_rows, N, ld);
 }
 
@@ -384,17 +410,7 @@ lfm3_status ffn_gemm(lfm3_ctx* ctx, int l, int n, int w2_splits, cudaStream_t s)
     CK(run_gemm(ctx, ctx->deq_w13, n, s));
     CK(affine_to_bf16(W.w2_codes, W.w2_scales, W.w2_biases, bits, D, F, ctx->deq, s));
     CK(run_gemm(ctx, split_plan(ctx->deq_w2, w2_splits), n, s));
-  } else if (ctx->cfg.ffn_format == LFM3_FFN_NVFP4) {
-    CK(nvfp4_to_bf16(W.w1_codes, W.w1_scales, W.w13_scale, F, D, ctx->deq, s));
-    CK(nvfp4_to_bf16(W.w3_codes, W.w3_scales, W.w13_scale, F, D, ctx->deq + (size_t)F * D, s));
-    GemmPlan p = ctx->deq_w13;
-    p.alpha = W.w13_scale;
-    CK(run_gemm(ctx, p, n, s));
-    CK(nvfp4_to_bf16(W.w2_codes, W.w2_scales, W.w2_scale, D, F, ctx->deq, s));
-    GemmPlan p2 = split_plan(ctx->deq_w2, w2_splits);
-    p2.alpha = W.w2_scale;
-    CK(run_gemm(ctx, p2, n, s));
-  } else {
+  } else {  // bf16, or NVFP4 expanded inside the GEMM (f16 activations)
     CK(run_gemm(ctx, ctx->plans[l].w13, n, s));
     CK(run_gemm(ctx, split_plan(ctx->plans[l].w2, w2_splits), n, s));
   }
@@ -485,6 +501,11 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
     if (g.ffn_format == LFM3_FFN_BF16) {
       ok &= plan_gemm(&P.w13, GEMM_SWIGLU, ctx->xn, R, W.w1, W.w3, F, D, ctx->big, F, 1.f);
       ok &= plan_gemm(&P.w2, GEMM_F32, ctx->big, R, W.w2, nullptr, D, F, ctx->part, D, 1.f);
+    } else if (g.ffn_format == LFM3_FFN_NVFP4) {  // f16 activations (xn, big) for these two
+      ok &= plan_gemm_q4(&P.w13, GEMM_SWIGLU, ctx->xn, R, W.w1_codes, W.w1_scales, W.w3_codes, W.w3_scales, F, D,
+                         ctx->big, F, W.w13_scale);
+      ok &= plan_gemm_q4(&P.w2, GEMM_F32, ctx->big, R, W.w2_codes, W.w2_scales, nullptr, nullptr, D, F, ctx->part, D,
+                         W.w2_scale);
     }
     if (!ok) return fail(ctx, LFM3_E_CUDA, "layer %d: tensor map encoding failed", l);
   }
@@ -548,7 +569,7 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
   if (g.has_head && !plan_gemm(&ctx->head_gemm, GEMM_HEAD, ctx->xn, R, ctx->embed, nullptr, g.vocab, D, nullptr,
                                 g.vocab, 1.f))
     return fail(ctx, LFM3_E_CUDA, "head GEMM tensor map encoding failed");
-  if (g.ffn_format != LFM3_FFN_BF16) {
+  if (g.ffn_format == LFM3_FFN_AFFINE) {
     bool ok = plan_gemm(&ctx->deq_w13, GEMM_SWIGLU, ctx->xn, R, ctx->deq, ctx->deq + (size_t)F * D, F, D, ctx->big, F, 1.f);
     ok &= plan_gemm(&ctx->deq_w2, GEMM_F32, ctx->big, R, ctx->deq, nullptr, D, F, ctx->part, D, 1.f);
     if (!ok) return fail(ctx, LFM3_E_CUDA, "NVFP4 tensor map encoding failed");
@@ -600,7 +621,7 @@ lfm3_status prefill_rows(lfm3_ctx* ctx, const lfm3_state* st, int slot, const in
     CK(embed_rows(d_tokens ? d_tokens + c0 : nullptr, ctx->embed,
                   d_embeds ? B(d_embeds) + (size_t)c0 * D : nullptr, nc, ctx->x_res,
                   d_hidden ? d_hidden + (size_t)c0 * D : nullptr, s));
-    CK(resid_norm(ctx->x_res, nullptr, 0, 0, nullptr, B(ctx->L[0].op_norm), ctx->xn, nc, eps, nullptr, s));
+    CK(resid_norm(ctx->x_res, nullptr, 0, 0, nullptr, B(ctx->L[0].op_norm), ctx->xn, nc, eps, nullptr, 0, s));
     for (int l = 0; l < g.n_layers; ++l) {
       const lfm3_layer_weights& W = ctx->L[l];
       const LayerPlan& P = ctx->plans[l];
@@ -648,12 +669,13 @@ lfm3_status prefill_rows(lfm3_ctx* ctx, const lfm3_state* st, int slot, const in
           CK(scratch_to_ring(ctx->sk, ctx->sv, ctx->scratch_rows, nr, p0, v.ring_k, v.ring_v, slot, g.max_streams, s));
         CK(run_gemm(ctx, P.o_proj, nc, s));
       }
-      CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nc, eps, nullptr, s));
+      CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nc, eps, nullptr,
+                    g.ffn_format == LFM3_FFN_NVFP4, s));
       lfm3_status fs = ffn_gemm(ctx, l, nc, 1, s);
       if (fs != LFM3_OK) return fs;
       const bf16* gnext = l + 1 < g.n_layers ? B(ctx->L[l + 1].op_norm) : (g.has_head ? ctx->final_norm : nullptr);
       CK(resid_norm(ctx->x_res, ctx->part, 1, 0, B(W.post_ffn_norm), gnext, ctx->xn, nc, eps,
-                    d_hidden ? d_hidden + ((size_t)(l + 1) * n + c0) * D : nullptr, s));
+                    d_hidden ? d_hidden + ((size_t)(l + 1) * n + c0) * D : nullptr, 0, s));
     }
     const bool head = last && g.has_head && (d_logits || d_argmax);
     if (head) {
@@ -732,7 +754,7 @@ lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, in
   CK(setup_rows(0, 0, d_slots, st->seq_len, nb, win, ctx->row_slot, ctx->row_pos, ctx->amax, s));
   const Rows rows{ctx->row_slot, ctx->row_pos, nb};
   CK(embed_rows(d_tokens, ctx->embed, B(d_embeds), nb, ctx->x_res, d_hidden, s));
-  CK(resid_norm(ctx->x_res, nullptr, 0, 0, nullptr, B(ctx->L[0].op_norm), ctx->xn, nb, eps, nullptr, s));
+  CK(resid_norm(ctx->x_res, nullptr, 0, 0, nullptr, B(ctx->L[0].op_norm), ctx->xn, nb, eps, nullptr, 0, s));
   for (int l = 0; l < g.n_layers; ++l) {
     const lfm3_layer_weights& W = ctx->L[l];
     const LayerPlan& P = ctx->plans[l];
@@ -762,13 +784,13 @@ lfm3_status enqueue_decode_large(lfm3_ctx* ctx, const lfm3_state* st, int nb, in
       CK(run_gemm(ctx, split_plan(P.o_proj, sp_o), nb, s));
     }
     CK(resid_norm(ctx->x_res, ctx->part, sp_o, (long)nb * D, B(W.post_op_norm), B(W.ffn_norm), ctx->xn, nb, eps,
-                  nullptr, s));
+                  nullptr, g.ffn_format == LFM3_FFN_NVFP4, s));
     const int sp_2 = one ? batch_splits(D, F) : 1;
     lfm3_status fs = ffn_gemm(ctx, l, nb, sp_2, s);
     if (fs != LFM3_OK) return fs;
     const bf16* gnext = l + 1 < g.n_layers ? B(ctx->L[l + 1].op_norm) : (g.has_head ? ctx->final_norm : nullptr);
     CK(resid_norm(ctx->x_res, ctx->part, sp_2, (long)nb * D, B(W.post_ffn_norm), gnext, ctx->xn, nb, eps,
-                  d_hidden ? d_hidden + (size_t)(l + 1) * nb * D : nullptr, s));
+                  d_hidden ? d_hidden + (size_t)(l + 1) * nb * D : nullptr, 0, s));
   }
   const bool head = g.has_head && (d_logits || d_argmax);
   if (head) {
@@ -910,7 +932,7 @@ lfm3_status enqueue_decode_stream(lfm3_ctx* ctx, const lfm3_state* st, int nb, i
     CK(run_ws(ctx, GEMV_HEAD, WS_BF16, ctx->ws_head, h, s));
     advance();
   } else if (dump_last) {
-    CK(resid_norm(cur, pend, pend_n, (long)nb * D, pend_g, nullptr, nullptr, nb, eps, dump_last, s));
+    CK(resid_norm(cur, pend, pend_n, (long)nb * D, pend_g, nullptr, nullptr, nb, eps, dump_last, 0, s));
   }
   CK(finish_step(st->seq_len, ctx->row_slot, nb, 0, 0, head ? ctx->amax : nullptr, head ? d_argmax : nullptr,
                  win == 1, s));
