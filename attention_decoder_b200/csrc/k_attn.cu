@@ -7,18 +7,20 @@
 // multiplies each head's output before o_proj (fused into the merge here).
 //
 // One launch per layer, from the raw q|k|v|gate projection rows (fp32, one row per stream):
-// block (split, kv head, stream) owns 64 keys - one 64-position page of that kv head on full
-// layers, a quarter of the 256-slot ring on sliding layers - so its keys and values are two
-// contiguous 16 KB tiles, copied with two bulk copies before the block waits for the projection
-// kernel (the cache does not depend on it). After the wait the block normalises and rotates its
-// four query heads and the head's new key, rounds them to bf16, writes the new key and value to
-// the cache (the block holding the current position does) and substitutes them for the stale
-// row in its shared copy. Scores: eight warps take 8 keys each; lane l holds dims 4l..4l+3 of
-// the four queries, and one transposing butterfly turns the 32 per-lane partial dots (8 keys x
-// 4 heads) into 32 finished scores, one per lane. Each block writes its unnormalised partial
-// (max, sum, o) per head; the last block of a (stream, kv head) - counted with an atomic -
-// merges the splits with every warp loading a different subset of them, applies the gate and
-// writes the bf16 output.
+// block (split, kv head, stream) owns whole 64-key pages - on full layers one page, or 2..8 pages
+// once the batch gives thousands of blocks; on sliding layers a quarter of the 256-slot ring - so
+// its keys and values arrive as contiguous 16 KB tiles, two bulk copies per page into one of two
+// buffers; the first two pages are requested before the block waits for the projection kernel
+// (the cache does not depend on it). After the wait the block normalises and rotates its four
+// query heads and the head's new key, rounds them to bf16, writes the new key and value to the
+// cache (the block holding the current position does) and substitutes them for the stale row
+// in its shared copy. Scores: eight warps take 8 keys of a page each; lane l holds dims
+// 4l..4l+3 of the four queries, and one transposing butterfly turns the 32 per-lane partial dots
+// (8 keys x 4 heads) into 32 finished scores, one per lane. Across a block's pages the softmax
+// runs online (running max and sum per head, the P V sums rescaled at a new max). Each block
+// writes its unnormalised partial (max, sum, o) per head; the last block of a (stream, kv head)
+// - counted with an atomic - merges the splits with every warp loading a different subset of
+// them, applies the gate and writes the bf16 output.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -33,7 +35,7 @@ namespace lfm3 {
 constexpr int DA_THREADS = 256;                  // 8 warps
 constexpr int DA_WARPS = DA_THREADS / 32;
 constexpr int DA_TILE = DEC_KEYS * HD * 2;       // bytes of one K or V tile
-constexpr int DA_SMEM = 2 * DA_TILE;             // dynamic shared memory: K and V tiles
+constexpr int DA_SMEM = 2 * DA_TILE;             // one page buffer: K and V tiles (two buffers)
 static_assert(DEC_KEYS == PAGE, "a decode split is one page");
 static_assert(DA_WARPS * 8 == DEC_KEYS, "eight keys per warp");
 
@@ -47,11 +49,9 @@ int attn_decode_splits(int max_pos) {
 DEVI size_t da_ml_offset(int nrows, int splits) { return (size_t)nrows * HQ * splits * HD; }
 
 __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* __restrict__ qkvg, Rows rows,
-                                                                  AttnLayer L, AttnDecodeArgs A, int splits,
+                                                                  AttnLayer L, AttnDecodeArgs A, int splits, int pps,
                                                                   float* __restrict__ part, bf16* __restrict__ y) {
-  extern __shared__ __align__(128) unsigned char dsm[];
-  bf16* ks = reinterpret_cast<bf16*>(dsm);
-  bf16* vs = ks + DEC_KEYS * HD;
+  extern __shared__ __align__(128) unsigned char dsm[];  // two buffers of one page: K then V
   __shared__ __align__(16) float qs[GQA][HD];
   __shared__ float kb[HD];
   __shared__ float sc[GQA][DEC_KEYS];
@@ -59,9 +59,10 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
   __shared__ __align__(16) float obuf[4][GQA][HD];       // PV of the four key quarters
   __shared__ float red[GQA + 1][4];
   __shared__ float lx[GQA];
+  __shared__ float alpha[GQA];                           // rescale of the running sums at a new max
   __shared__ __align__(16) bf16 wk[MAX_WIN][HD], wv[MAX_WIN][HD];  // earlier rows of a verify window
   __shared__ float kw[HD];
-  __shared__ __align__(8) uint64_t kv_bar;
+  __shared__ __align__(8) uint64_t kv_bar[2];
   __shared__ int last;
 
   const int sp = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -75,22 +76,35 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
   // rows were set by the first kernel of the step, which has completed (reads go to L2)
   const int slot = __ldcg(rows.slot + b), pos = __ldcg(rows.pos + b);
   const int nkeys = L.full ? pos + 1 : min(pos + 1, WIN);
-  const int nact = (nkeys + DEC_KEYS - 1) / DEC_KEYS;  // splits with keys
+  const int keys_per = pps * DEC_KEYS;                 // keys of one split: pps pages
+  const int nact = (nkeys + keys_per - 1) / keys_per;  // splits with keys
   if (sp >= nact) {
     pdl_wait();
     pdl_launch_dependents();
     return;
   }
   const int cur = L.full ? pos : pos % WIN;  // key index of the current position
-  const int j0 = sp * DEC_KEYS, cnt = min(nkeys - j0, DEC_KEYS);
-  const size_t tile = L.full ? ((size_t)L.page_table[(size_t)slot * L.max_pages + sp] * HKV + kvh) * PAGE * HD
-                             : (((size_t)slot * HKV + kvh) * WIN + j0) * HD;
+  const int j0 = sp * keys_per, cnt = min(nkeys - j0, keys_per);
+  const int np = (cnt + DEC_KEYS - 1) / DEC_KEYS;  // pages of this split
+  // the K / V tile of page i of the split (64 keys of this kv head, contiguous)
+  auto tile_of = [&](int i) -> size_t {
+    const int j = j0 + i * DEC_KEYS;
+    return L.full ? ((size_t)L.page_table[(size_t)slot * L.max_pages + j / DEC_KEYS] * HKV + kvh) * PAGE * HD
+                  : (((size_t)slot * HKV + kvh) * WIN + j) * HD;
+  };
+  auto fetch = [&](int i) {  // page i into buffer i & 1 (thread 0)
+    const uint32_t buf = su32(dsm) + (uint32_t)(i & 1) * DA_SMEM, bar = su32(&kv_bar[i & 1]);
+    const size_t t = tile_of(i);
+    mbar_expect_tx(bar, DA_SMEM);
+    bulk_g2s(buf, L.k + t, DA_TILE, bar);
+    bulk_g2s(buf + DA_TILE, L.v + t, DA_TILE, bar);
+  };
   if (tid == 0) {
-    mbar_init(su32(&kv_bar), 1);
+    mbar_init(su32(&kv_bar[0]), 1);
+    mbar_init(su32(&kv_bar[1]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    mbar_expect_tx(su32(&kv_bar), DA_SMEM);
-    bulk_g2s(su32(ks), L.k + tile, DA_TILE, su32(&kv_bar));
-    bulk_g2s(su32(vs), L.v + tile, DA_TILE, su32(&kv_bar));
+    fetch(0);
+    if (np > 1) fetch(1);
   }
   // gains and rotary coefficients of dimension d = tid (threads < 128) are weights too
   const int d = tid & (HD - 1), pd = d < 64 ? d + 64 : d - 64, ir = d & 63;
@@ -152,7 +166,7 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
     for (int hh = 0; hh < GQA; ++hh) qs[hh][d] = qr[hh] * scale;
     if (has_cur) {  // the new key and value into the cache, as every later step reads them
       if (L.full || A.win == 1) {
-        const size_t row = tile + (size_t)(cur - j0) * HD + d;
+        const size_t row = tile_of((cur - j0) / DEC_KEYS) + (size_t)((cur - j0) % DEC_KEYS) * HD + d;
         const_cast<bf16*>(L.k)[row] = f2bf(kr);
         const_cast<bf16*>(L.v)[row] = f2bf(vv);
       } else {  // a verify window's sliding rows wait for the commit in the side buffer
@@ -184,99 +198,127 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
     }
     __syncthreads();
   }
-  // ---- the staged split; the rows of the current position (and of the window's earlier ones)
-  // there are stale: put the new ones in
-  bool ok = mbar_wait(su32(&kv_bar), 0, A.err);
-  if (!ok) ok = mbar_wait(su32(&kv_bar), 0, A.err);  // a copy still in flight must land before exit
-  if (tid < HD) {
-    if (has_cur) {
-      ks[(cur - j0) * HD + d] = f2bf(kr);
-      vs[(cur - j0) * HD + d] = f2bf(vv);
-    }
-    for (int ip = 0; ip < wi; ++ip) {
-      const int pp = pos - wi + ip;
-      const int kidx = L.full ? pp : pp % WIN;
-      if (kidx >= j0 && kidx < j0 + cnt) {
-        ks[(kidx - j0) * HD + d] = wk[ip][d];
-        vs[(kidx - j0) * HD + d] = wv[ip][d];
-      }
-    }
-  }
-  __syncthreads();
 
+  // ---- the split's pages, two buffers deep, with an online softmax across them
   const size_t mloff = da_ml_offset(rows.n, splits);
   const size_t hbase = ((size_t)b * HQ + kvh * GQA) * splits;  // (stream, first head of the group) x splits
-  if (ok) {
-    // ---- scores: warp w takes keys 8w .. 8w+7; lane l holds dims 4l..4l+3 of the four queries
-    {
-      float4 q4[GQA];
-#pragma unroll
-      for (int hh = 0; hh < GQA; ++hh) q4[hh] = *reinterpret_cast<const float4*>(&qs[hh][4 * lane]);
-      float v[32];  // v[h * 8 + k]: this lane's partial dot of head h with key 8w + k
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint2 kk = *reinterpret_cast<const uint2*>(ks + (8 * warp + k) * HD + 4 * lane);
-        const float k0 = bflo(kk.x), k1 = bfhi(kk.x), k2 = bflo(kk.y), k3 = bfhi(kk.y);
-#pragma unroll
-        for (int hh = 0; hh < GQA; ++hh) v[hh * 8 + k] = q4[hh].x * k0 + q4[hh].y * k1 + q4[hh].z * k2 + q4[hh].w * k3;
+  const int qt = tid >> 6, dp = 2 * (tid & 63);                 // P V: key quarter, dimension pair
+  float o[GQA][2] = {};
+  float Mh = -INFINITY, Lh = 0.f;  // warp h < 4: running max and sum of head h
+  bool ok = true;
+  int issued = min(np, 2), done = 0;  // pages copied / pages landed
+  for (int i = 0; i < np; ++i) {
+    const bf16* ks = reinterpret_cast<const bf16*>(dsm + (size_t)(i & 1) * DA_SMEM);
+    const bf16* vs = ks + DEC_KEYS * HD;
+    const int pj0 = j0 + i * DEC_KEYS, pc = min(cnt - i * DEC_KEYS, DEC_KEYS);
+    if (ok) ok = mbar_wait(su32(&kv_bar[i & 1]), (i >> 1) & 1, A.err);
+    ok = __syncthreads_and(ok);  // the same for every thread of the block
+    if (ok) done = i + 1;
+    // the rows of the current position (and of the window's earlier ones) here are stale
+    if (tid < HD) {
+      bf16* kw2 = const_cast<bf16*>(ks);
+      bf16* vw2 = const_cast<bf16*>(vs);
+      if (cur >= pj0 && cur < pj0 + pc) {
+        kw2[(cur - pj0) * HD + d] = f2bf(kr);
+        vw2[(cur - pj0) * HD + d] = f2bf(vv);
       }
-      // butterfly: at offset o each lane keeps the half of its values selected by bit o of its
-      // lane id and adds the partner's; after five steps lane l holds the full sum of value l
-#pragma unroll
-      for (int o = 16, c = 32; o >= 1; o >>= 1, c >>= 1) {
-        const bool up = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < c / 2; ++i) {
-          const float send = up ? v[i] : v[i + c / 2];
-          const float keep = up ? v[i + c / 2] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      for (int ip = 0; ip < wi; ++ip) {
+        const int pp = pos - wi + ip;
+        const int kidx = L.full ? pp : pp % WIN;
+        if (kidx >= pj0 && kidx < pj0 + pc) {
+          kw2[(kidx - pj0) * HD + d] = wk[ip][d];
+          vw2[(kidx - pj0) * HD + d] = wv[ip][d];
         }
       }
-      const int hh = lane >> 3, j = 8 * warp + (lane & 7);
-      sc[hh][j] = j < cnt ? v[0] : -INFINITY;
     }
     __syncthreads();
-    // ---- softmax of this split: warp h < 4 takes head h
-    if (warp < GQA) {
-      const float s0 = sc[warp][lane], s1 = sc[warp][lane + 32];
-      const float m = warp_max(fmaxf(s0, s1));
-      const float p0 = __expf(s0 - m), p1 = __expf(s1 - m);
-      reinterpret_cast<float*>(&pr[lane])[warp] = p0;
-      reinterpret_cast<float*>(&pr[lane + 32])[warp] = p1;
-      const float l = warp_sum(p0 + p1);
-      if (lane == 0) {
-        part[mloff + 2 * (hbase + (size_t)warp * splits + sp)] = m;
-        part[mloff + 2 * (hbase + (size_t)warp * splits + sp) + 1] = l;
-      }
-    }
-    __syncthreads();
-    // ---- P V: thread = (key quarter, dimension pair); rows past the split's keys are never read
-    {
-      const int qt = tid >> 6, dp = 2 * (tid & 63);
-      const int je = min(cnt, 16 * qt + 16);
-      float o[GQA][2] = {};
-      for (int j = 16 * qt; j < je; ++j) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(vs + j * HD + dp);
-        const float v0 = bflo(w), v1 = bfhi(w);
-        const float4 p = pr[j];
-        o[0][0] += p.x * v0; o[0][1] += p.x * v1;
-        o[1][0] += p.y * v0; o[1][1] += p.y * v1;
-        o[2][0] += p.z * v0; o[2][1] += p.z * v1;
-        o[3][0] += p.w * v0; o[3][1] += p.w * v1;
-      }
+    if (ok) {
+      // scores: warp w takes keys 8w .. 8w+7; lane l holds dims 4l..4l+3 of the four queries
+      {
+        float4 q4[GQA];
 #pragma unroll
-      for (int hh = 0; hh < GQA; ++hh) *reinterpret_cast<float2*>(&obuf[qt][hh][dp]) = make_float2(o[hh][0], o[hh][1]);
+        for (int hh = 0; hh < GQA; ++hh) q4[hh] = *reinterpret_cast<const float4*>(&qs[hh][4 * lane]);
+        float v[32];  // v[h * 8 + k]: this lane's partial dot of head h with key 8w + k
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint2 kk = *reinterpret_cast<const uint2*>(ks + (8 * warp + k) * HD + 4 * lane);
+          const float k0 = bflo(kk.x), k1 = bfhi(kk.x), k2 = bflo(kk.y), k3 = bfhi(kk.y);
+#pragma unroll
+          for (int hh = 0; hh < GQA; ++hh) v[hh * 8 + k] = q4[hh].x * k0 + q4[hh].y * k1 + q4[hh].z * k2 + q4[hh].w * k3;
+        }
+        // butterfly: at offset o each lane keeps the half of its values selected by bit o of its
+        // lane id and adds the partner's; after five steps lane l holds the full sum of value l
+#pragma unroll
+        for (int o2 = 16, c = 32; o2 >= 1; o2 >>= 1, c >>= 1) {
+          const bool up = (lane & o2) != 0;
+#pragma unroll
+          for (int e = 0; e < c / 2; ++e) {
+            const float send = up ? v[e] : v[e + c / 2];
+            const float keep = up ? v[e + c / 2] : v[e];
+            v[e] = keep + __shfl_xor_sync(0xffffffffu, send, o2);
+          }
+        }
+        const int hh = lane >> 3, j = 8 * warp + (lane & 7);
+        sc[hh][j] = j < pc ? v[0] : -INFINITY;
+      }
+      __syncthreads();
+      // softmax: warp h < 4 takes head h; the running sums are rescaled at a new maximum
+      if (warp < GQA) {
+        const float s0 = sc[warp][lane], s1 = sc[warp][lane + 32];
+        const float mn = fmaxf(Mh, warp_max(fmaxf(s0, s1)));
+        const float p0 = __expf(s0 - mn), p1 = __expf(s1 - mn);
+        reinterpret_cast<float*>(&pr[lane])[warp] = p0;
+        reinterpret_cast<float*>(&pr[lane + 32])[warp] = p1;
+        const float a = __expf(Mh - mn);  // 0 on the first page
+        Lh = Lh * a + warp_sum(p0 + p1);
+        Mh = mn;
+        if (lane == 0) alpha[warp] = a;
+      }
+      __syncthreads();
+      // P V: thread = (key quarter, dimension pair); rows past the page's keys are never read
+      {
+        const int je = min(pc, 16 * qt + 16);
+#pragma unroll
+        for (int hh = 0; hh < GQA; ++hh) {
+          o[hh][0] *= alpha[hh];
+          o[hh][1] *= alpha[hh];
+        }
+        for (int j = 16 * qt; j < je; ++j) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(vs + j * HD + dp);
+          const float v0 = bflo(w), v1 = bfhi(w);
+          const float4 p = pr[j];
+          o[0][0] += p.x * v0; o[0][1] += p.x * v1;
+          o[1][0] += p.y * v0; o[1][1] += p.y * v1;
+          o[2][0] += p.z * v0; o[2][1] += p.z * v1;
+          o[3][0] += p.w * v0; o[3][1] += p.w * v1;
+        }
+      }
+    }
+    __syncthreads();  // the buffer is read; refill it with page i + 2
+    if (ok && i + 2 < np) {
+      if (tid == 0) fetch(i + 2);
+      issued = i + 3;
+    }
+  }
+  if (!ok && tid == 0)  // copies still in flight land before the block exits (bounded)
+    for (int p = done; p < issued; ++p) mbar_wait(su32(&kv_bar[p & 1]), (p >> 1) & 1, A.err);
+  if (ok) {
+#pragma unroll
+    for (int hh = 0; hh < GQA; ++hh) *reinterpret_cast<float2*>(&obuf[qt][hh][dp]) = make_float2(o[hh][0], o[hh][1]);
+    if (warp < GQA && lane == 0) {
+      part[mloff + 2 * (hbase + (size_t)warp * splits + sp)] = Mh;
+      part[mloff + 2 * (hbase + (size_t)warp * splits + sp) + 1] = Lh;
     }
     __syncthreads();
     if (tid < GQA * HD / 4) {
       const int hh = tid >> 5, d4 = 4 * lane;
-      float4 s = *reinterpret_cast<const float4*>(&obuf[0][hh][d4]);
+      float4 s4 = *reinterpret_cast<const float4*>(&obuf[0][hh][d4]);
 #pragma unroll
-      for (int qt = 1; qt < 4; ++qt) {
-        const float4 t = *reinterpret_cast<const float4*>(&obuf[qt][hh][d4]);
-        s.x += t.x; s.y += t.y; s.z += t.z; s.w += t.w;
+      for (int q = 1; q < 4; ++q) {
+        const float4 t = *reinterpret_cast<const float4*>(&obuf[q][hh][d4]);
+        s4.x += t.x; s4.y += t.y; s4.z += t.z; s4.w += t.w;
       }
-      *reinterpret_cast<float4*>(part + (hbase + (size_t)hh * splits + sp) * HD + d4) = s;
+      *reinterpret_cast<float4*>(part + (hbase + (size_t)hh * splits + sp) * HD + d4) = s4;
     }
   } else {  // a copy that never landed: this split contributes nothing
     if (tid < GQA) {
@@ -349,22 +391,33 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
 #endif
 }
 
+// Pages per split on full layers: one page while that keeps every SM busy, more (up to 8, each
+// split then streams its pages through two buffers) once the batch x kv heads x splits give
+// thousands of blocks; fewer, longer blocks spend less on their fixed work and on the merge.
+int attn_pages_per_split(int rows, int splits) {
+  int pps = 1;
+  while (pps < 8 && splits % (2 * pps) == 0 && (long)rows * HKV * (splits / (2 * pps)) >= 2048) pps *= 2;
+  return pps;
+}
+
 cudaError_t attn_decode_fused(const float* qkvg, Rows rows, AttnLayer L, const AttnDecodeArgs& A, int splits,
                               float* part, bf16* y, cudaStream_t s) {
+  const int pps = L.full ? attn_pages_per_split(rows.n, splits) : 1;
+  const int nsp = splits / pps;  // blocks (and partial slots) per (stream, kv head)
 #ifdef LFM3_TRACE
   AttnDecodeArgs At = A;
   At.trace = g_trace;
   At.trace_id = g_launches;
-  return launch(k_attn_decode_fused, dim3(splits, HKV, rows.n), dim3(DA_THREADS), DA_SMEM, s, qkvg, rows, L, At,
-                splits, part, y);
+  return launch(k_attn_decode_fused, dim3(nsp, HKV, rows.n), dim3(DA_THREADS), (pps > 1 ? 2 : 1) * DA_SMEM, s, qkvg,
+                rows, L, At, nsp, pps, part, y);
 #else
-  return launch(k_attn_decode_fused, dim3(splits, HKV, rows.n), dim3(DA_THREADS), DA_SMEM, s, qkvg, rows, L, A, splits,
-                part, y);
+  return launch(k_attn_decode_fused, dim3(nsp, HKV, rows.n), dim3(DA_THREADS), (pps > 1 ? 2 : 1) * DA_SMEM, s, qkvg,
+                rows, L, A, nsp, pps, part, y);
 #endif
 }
 
 cudaError_t attn_init() {
-  return cudaFuncSetAttribute(k_attn_decode_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, DA_SMEM);
+  return cudaFuncSetAttribute(k_attn_decode_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * DA_SMEM);
 }
 
 // ------------------------------------------------------------------------------------------ fixed scratch
