@@ -161,6 +161,7 @@ struct GemmArgs {
   int splits;                  // K splits (fp32 partial sums at out + s * M * ld)
   unsigned long long* amax;    // GEMM_HEAD
   int f16out;                  // GEMM_SWIGLU: the bf16-rounded products stored as f16
+  int w_const;                 // the weights are not written by an earlier kernel of the stream
 };
 
 // Tile t of a launch: M tiles fastest (consecutive blocks share a weight tile through L2), then
@@ -341,11 +342,32 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  pdl_wait();
-  pdl_launch_dependents();
-
   if (warp == 0) {
     if (lane == 0) {
+      // the weight boxes of one stage (the activations come from the previous kernel)
+      auto load_w = [&](uint32_t b_s, int kb, int n0, uint32_t bar) {
+        if constexpr (EPI == GEMM_SWIGLU) {  // BN / 2 rows of w1, then the same rows of w3
+          tma_load_2d(b_s, &tb, kb * GM_BK, n0, bar);
+          tma_load_2d(b_s + G::B_BYTES / 2, &tb3, kb * GM_BK, n0, bar);
+        } else {  // weight boxes are 128 rows: a 256-wide tile takes two
+#pragma unroll
+          for (int h = 0; h < BN / 128; ++h) tma_load_2d(b_s + h * (G::B_BYTES / (BN / 128)), &tb, kb * GM_BK, n0 + 128 * h, bar);
+        }
+      };
+      // constant weights: the first tile's first stages are requested before the wait for the
+      // previous kernel, so their latency overlaps its tail
+      int pre = 0;
+      if (g.w_const && (int)blockIdx.x < ntiles) {
+        const GemmTile T = gemm_tile(blockIdx.x, num_m, num_n, GM_BM, NOUT, nk, g.splits);
+        pre = min(S, T.kb1 - T.kb0);
+        for (int j = 0; j < pre; ++j) {
+          const uint32_t a_s = su32(smem + j * G::STAGE);
+          mbar_expect_tx(full0 + 8 * j, G::STAGE);
+          load_w(a_s + G::A_BYTES, T.kb0 + j, T.n0, full0 + 8 * j);
+        }
+      }
+      pdl_wait();
+      pdl_launch_dependents();
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -359,20 +381,22 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
             break;
           }
           const uint32_t a_s = su32(smem + s * G::STAGE), b_s = a_s + G::A_BYTES;
-          mbar_expect_tx(full0 + 8 * s, G::STAGE);
-          tma_load_2d(a_s, &ta, kb * GM_BK, m0, full0 + 8 * s);
-          if constexpr (EPI == GEMM_SWIGLU) {  // BN / 2 rows of w1, then the same rows of w3
-            tma_load_2d(b_s, &tb, kb * GM_BK, n0, full0 + 8 * s);
-            tma_load_2d(b_s + G::B_BYTES / 2, &tb3, kb * GM_BK, n0, full0 + 8 * s);
-          } else {  // weight boxes are 128 rows: a 256-wide tile takes two
-#pragma unroll
-            for (int h = 0; h < BN / 128; ++h)
-              tma_load_2d(b_s + h * (G::B_BYTES / (BN / 128)), &tb, kb * GM_BK, n0 + 128 * h, full0 + 8 * s);
+          if (it >= pre) {
+            mbar_expect_tx(full0 + 8 * s, G::STAGE);
+            load_w(b_s, kb, n0, full0 + 8 * s);
           }
+          tma_load_2d(a_s, &ta, kb * GM_BK, m0, full0 + 8 * s);
         }
       }
+      if (!ok)  // stages whose weights went out before the wait still complete (bounded)
+        for (int j = it; j < pre; ++j) mbar_wait(full0 + 8 * j, 0, g.err);
+    } else {
+      pdl_wait();
+      pdl_launch_dependents();
     }
   } else if (warp == 1) {
+    pdl_wait();
+    pdl_launch_dependents();
     if (lane == 0) {
       constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                  ((uint32_t)(GM_BM >> 4) << 24);
@@ -415,6 +439,8 @@ __global__ void __launch_bounds__(192, 1) k_gemm(const __grid_constant__ CUtenso
       }
     }
   } else {
+    pdl_wait();
+    pdl_launch_dependents();
     const int quarter = warp & 3;
     int i = 0;
     bool ok = true;
@@ -645,7 +671,7 @@ static cudaError_t launch_gemm(const GemmPlan& p, int M, int* err, cudaStream_t 
   constexpr size_t smem = gemm_smem<BN>();
   auto k = k_gemm<BN, EPI>;
   const int splits = EPI == GEMM_F32 ? std::max(1, p.splits) : 1;
-  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, splits, p.amax, 0};
+  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, splits, p.amax, 0, p.w_const};
   const int ntile = EPI == GEMM_SWIGLU ? BN / 2 : BN;
   const int tiles = ((p.N + ntile - 1) / ntile) * ((M + GM_BM - 1) / GM_BM) * splits;
   dim3 grid(std::min(tiles, g_gemm_sms > 0 ? g_gemm_sms : 148));
@@ -679,7 +705,7 @@ template <int EPI>
 static cudaError_t launch_gemm2(const GemmPlan& p, int M, int* err, cudaStream_t s) {
   constexpr int BN = 256;
   constexpr int ntile = EPI == GEMM_SWIGLU ? BN / 2 : BN;
-  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, 1, nullptr, 0};
+  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, 1, nullptr, 0, 0};
   const int tiles = ((p.N + ntile - 1) / ntile) * ((M + 2 * GM_BM - 1) / (2 * GM_BM));
   cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config(std::min(tiles, g_gemm_pairs), gemm2_smem<BN>(), s, attr);
@@ -807,8 +833,8 @@ __global__ void __launch_bounds__(Q4G_THREADS, 1) k_gemm_q4(const __grid_constan
     }
   } else if (warp >= 6) {
     // ------------------------------------------------ expansion: thread c = row c of the tile
-    pdl_wait();
-    pdl_launch_dependents();
+    // (codes and scales are constants: the first scales are requested before the wait)
+    bool waited = false;
     const int c = threadIdx.x - 6 * 32;
     const uint32_t rowoff = (uint32_t)(c >> 3) * 1024 + (uint32_t)(c & 7) * 128;
     int it = 0;
@@ -822,6 +848,11 @@ __global__ void __launch_bounds__(Q4G_THREADS, 1) k_gemm_q4(const __grid_constan
       int grp = T.kb0 >> 2;
       uint4 scv = valid ? ldg16(srow + grp * 16) : make_uint4(0, 0, 0, 0);
       uint4 scn = (valid && (grp + 1) * 4 < nk) ? ldg16(srow + (grp + 1) * 16) : make_uint4(0, 0, 0, 0);
+      if (!waited) {
+        pdl_wait();
+        pdl_launch_dependents();
+        waited = true;
+      }
       for (int kb = T.kb0; kb < T.kb1; ++kb, ++it) {
         if ((kb >> 2) != grp) {
           grp = kb >> 2;
@@ -855,6 +886,10 @@ __global__ void __launch_bounds__(Q4G_THREADS, 1) k_gemm_q4(const __grid_constan
           mbar_arrive(r_empty + 8 * r);
         }
       }
+    }
+    if (!waited) {
+      pdl_wait();
+      pdl_launch_dependents();
     }
   } else if (warp == 1) {
     pdl_wait();
@@ -919,7 +954,7 @@ __global__ void __launch_bounds__(Q4G_THREADS, 1) k_gemm_q4(const __grid_constan
 template <int EPI>
 static cudaError_t launch_gemm_q4(const GemmPlan& p, int M, int* err, cudaStream_t s) {
   const int splits = EPI == GEMM_F32 ? std::max(1, p.splits) : 1;
-  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, splits, nullptr, EPI == GEMM_SWIGLU ? 1 : 0};
+  GemmArgs g{M, p.N, p.K, p.ld, p.out, p.alpha, err, splits, nullptr, EPI == GEMM_SWIGLU ? 1 : 0, 1};
   const int ntile = EPI == GEMM_SWIGLU ? 64 : 128;
   const int tiles = ((p.N + ntile - 1) / ntile) * ((M + GM_BM - 1) / GM_BM) * splits;
   dim3 grid(std::min(tiles, g_gemm_sms > 0 ? g_gemm_sms : 148));

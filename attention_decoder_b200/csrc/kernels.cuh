@@ -240,6 +240,7 @@ struct GemmPlan {
   // out + s * M * ld (plain stores); the argmax keys of GEMM_HEAD
   int splits;
   unsigned long long* amax;
+  int w_const;        // 1: weights no kernel writes (read before the wait on the previous kernel)
   // NVFP4 weights (q4 = 1): codes [N][K/2] in 64-row (SwiGLU: w1 and w3) or 128-row boxes of one
   // K block, E4M3 scales [N][K/16]; the activations (a) are f16 and the SwiGLU output is f16
   int q4;

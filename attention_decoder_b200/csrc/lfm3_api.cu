@@ -279,6 +279,7 @@ bool plan_gemm(GemmPlan* p, int epi, const void* a, int a_rows, const void* b, c
   p->alpha = alpha;
   p->splits = 1;
   p->amax = nullptr;
+  p->w_const = 1;
   p->q4 = 0;
   p->sc = p->sc3 = nullptr;
   const uint32_t box_b = 128;  // weight boxes: 128 rows (wide and paired tiles issue several)
@@ -306,6 +307,7 @@ bool plan_gemm_q4(GemmPlan* p, int epi, const void* a, int a_rows, const uint8_t
   p->alpha = alpha;
   p->splits = 1;
   p->amax = nullptr;
+  p->w_const = 1;
   p->q4 = 1;
   p->sc = scales;
   p->sc3 = scales3 ? scales3 : scales;
@@ -572,6 +574,7 @@ extern "C" lfm3_status lfm3_bind_workspace(lfm3_ctx* ctx, void* d_ws, size_t byt
   if (g.ffn_format == LFM3_FFN_AFFINE) {
     bool ok = plan_gemm(&ctx->deq_w13, GEMM_SWIGLU, ctx->xn, R, ctx->deq, ctx->deq + (size_t)F * D, F, D, ctx->big, F, 1.f);
     ok &= plan_gemm(&ctx->deq_w2, GEMM_F32, ctx->big, R, ctx->deq, nullptr, D, F, ctx->part, D, 1.f);
+    ctx->deq_w13.w_const = ctx->deq_w2.w_const = 0;  // expanded into scratch by the kernel before
     if (!ok) return fail(ctx, LFM3_E_CUDA, "NVFP4 tensor map encoding failed");
   }
   CK(cudaDeviceSynchronize());
