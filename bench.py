@@ -258,6 +258,14 @@ def run_ours(args):
 
     if args.only == "prefill":
         return run_prefill_only(args, world, m, g, stream, clocks, Wm)
+    if args.only == "nvfp4":
+        del m
+        torch.cuda.empty_cache()
+        r = nvfp4_leg(world, g, stream, prompt, K, Wm, hbm)
+        if rank == 0:
+            print(json.dumps({"profiling_case": "NVFP4 decode at 1/4/8/64 streams", **r, "clocks": clocks.stop()}),
+                  flush=True)
+        return
     st, o = fresh_state(m)
     bufs = {"argmax": o["argmax"].clone(), "logits": torch.empty(1, g.vocab, device="cuda")}
     slots_d = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -368,55 +376,7 @@ def run_ours(args):
 
     # ---------------- NVFP4 FFN model: decode at 1 / 4 / 8 streams (2048 ctx) and 64 streams
     if not args.no_extra and args.only is None:
-        Wq = make_weights(g, 0, ffn="nvfp4")
-        S = 64
-        ctx64 = context_lengths(1, "ctx64", S, 256, 8192)
-        steps_q = max(4, min(K, 32))
-        mpp_q = (8192 + Wm + steps_q + 16) // 64 + 2
-        mq = Lfm3Model(Wq, max_streams=S, max_pages_per_stream=mpp_q, max_batch=S)
-        del Wq
-        stq = mq.new_state(page_table=page_permutation(1, "pages64", S * mpp_q).reshape(S, mpp_q))
-        for s in range(8):
-            mq.prefill(stq, s, tokens=prompt)
-        qb, qfrac = {}, {}
-        for B in (1, 4, 8):
-            sl = torch.arange(B, dtype=torch.int32, device="cuda")
-            ob = {"argmax": torch.zeros(B, dtype=torch.int32, device="cuda"),
-                  "logits": torch.empty(B, g.vocab, device="cuda")}
-
-            def qstep():
-                mq.decode(stq, list(range(B)), tokens=ob["argmax"], d_slots=sl, out=ob)
-
-            for _ in range(Wm):
-                qstep()
-            p0 = int(stq.h_seq_len[0])
-            qms = timed(world, qstep, steps_q, stream)
-            qb[B] = B * steps_q / (qms / 1e3)
-            qbytes = decode_step_bytes(g, [p0 + steps_q // 2] * B, nvfp4=True)
-            qfrac[B] = qbytes * (steps_q / (qms / 1e3)) / 1e9 / hbm
-        # 64 streams on drawn state: K/V, rings and conv columns N(0,1) drawn on the device
-        gen = torch.Generator(device="cuda").manual_seed(1)
-        for t in (stq.kv_k, stq.kv_v, stq.ring_k, stq.ring_v, stq.conv):
-            t.normal_(generator=gen)
-        stq.h_seq_len[:] = ctx64
-        stq.seq_len.copy_(torch.from_numpy(stq.h_seq_len))
-        sl = torch.arange(S, dtype=torch.int32, device="cuda")
-        ob = {"argmax": torch.from_numpy(make_tokens(1, "tok64", S, g.vocab)).cuda(),
-              "logits": torch.empty(S, g.vocab, device="cuda")}
-
-        def q64():
-            mq.decode(stq, list(range(S)), tokens=ob["argmax"], d_slots=sl, out=ob)
-
-        for _ in range(Wm):
-            q64()
-        qms = timed(world, q64, steps_q, stream)
-        qb[64] = S * steps_q / (qms / 1e3)
-        qbytes = decode_step_bytes(g, [int(c) + Wm + steps_q // 2 for c in ctx64], nvfp4=True)
-        qfrac[64] = qbytes * (steps_q / (qms / 1e3)) / 1e9 / hbm
-        res["decode_nvfp4"] = {f"b{b}_tok_s": v for b, v in qb.items()}
-        res["decode_nvfp4"].update({f"b{b}_hbm_frac": round(v, 4) for b, v in qfrac.items()})
-        res["decode_nvfp4"]["b64_contexts"] = "uniform [256, 8192], mean %.0f" % float(np.mean(ctx64))
-        del mq, stq
+        res.update(nvfp4_leg(world, g, stream, prompt, K, Wm, hbm))
     clk = clocks.stop()
 
     tok_s_rank = res["decode_b1"]["tok_s"]
@@ -483,6 +443,67 @@ def prefill_flops(g, n):
     return n * per_tok + attn + 2 * d * g.vocab
 
 
+def nvfp4_leg(world, g, stream, prompt, K, Wm, hbm):
+    """The NVFP4-FFN model: decode tok/s and HBM fraction at 1 / 4 / 8 streams (2048-token context,
+    prefilled) and at 64 streams on drawn state (contexts uniform in [256, 8192])."""
+    import torch
+    import numpy as np
+    from attention_decoder_b200.model import Lfm3Model
+    from lfm3_inputs import make_weights, make_tokens, page_permutation, context_lengths
+    res = {}
+    Wq = make_weights(g, 0, ffn="nvfp4")
+    S = 64
+    ctx64 = context_lengths(1, "ctx64", S, 256, 8192)
+    steps_q = max(4, min(K, 32))
+    mpp_q = (8192 + Wm + steps_q + 16) // 64 + 2
+    mq = Lfm3Model(Wq, max_streams=S, max_pages_per_stream=mpp_q, max_batch=S)
+    del Wq
+    stq = mq.new_state(page_table=page_permutation(1, "pages64", S * mpp_q).reshape(S, mpp_q))
+    for s in range(8):
+        mq.prefill(stq, s, tokens=prompt)
+    qb, qfrac = {}, {}
+    for B in (1, 4, 8):
+        sl = torch.arange(B, dtype=torch.int32, device="cuda")
+        ob = {"argmax": torch.zeros(B, dtype=torch.int32, device="cuda"),
+              "logits": torch.empty(B, g.vocab, device="cuda")}
+
+        def qstep():
+            mq.decode(stq, list(range(B)), tokens=ob["argmax"], d_slots=sl, out=ob)
+
+        for _ in range(Wm):
+            qstep()
+        p0 = int(stq.h_seq_len[0])
+        qms = timed(world, qstep, steps_q, stream)
+        qb[B] = B * steps_q / (qms / 1e3)
+        qbytes = decode_step_bytes(g, [p0 + steps_q // 2] * B, nvfp4=True)
+        qfrac[B] = qbytes * (steps_q / (qms / 1e3)) / 1e9 / hbm
+    # 64 streams on drawn state: K/V, rings and conv columns N(0,1) drawn on the device
+    gen = torch.Generator(device="cuda").manual_seed(1)
+    for t in (stq.kv_k, stq.kv_v, stq.ring_k, stq.ring_v, stq.conv):
+        t.normal_(generator=gen)
+    stq.h_seq_len[:] = ctx64
+    stq.seq_len.copy_(torch.from_numpy(stq.h_seq_len))
+    sl = torch.arange(S, dtype=torch.int32, device="cuda")
+    ob = {"argmax": torch.from_numpy(make_tokens(1, "tok64", S, g.vocab)).cuda(),
+          "logits": torch.empty(S, g.vocab, device="cuda")}
+
+    def q64():
+        mq.decode(stq, list(range(S)), tokens=ob["argmax"], d_slots=sl, out=ob)
+
+    for _ in range(Wm):
+        q64()
+    qms = timed(world, q64, steps_q, stream)
+    qb[64] = S * steps_q / (qms / 1e3)
+    qbytes = decode_step_bytes(g, [int(c) + Wm + steps_q // 2 for c in ctx64], nvfp4=True)
+    qfrac[64] = qbytes * (steps_q / (qms / 1e3)) / 1e9 / hbm
+    res["decode_nvfp4"] = {f"b{b}_tok_s": v for b, v in qb.items()}
+    res["decode_nvfp4"].update({f"b{b}_hbm_frac": round(v, 4) for b, v in qfrac.items()})
+    res["decode_nvfp4"]["b64_contexts"] = "uniform [256, 8192], mean %.0f" % float(np.mean(ctx64))
+    del mq, stq
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_prefill_only(args, world, m, g, stream, clocks, Wm):
     """Profiling leg: the 8192-token prompt pass (chunks of 2048, shuffled pages), timed."""
     import torch
@@ -542,8 +563,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--small", action="store_true", help="4-layer profiling case (not a bench line)")
     ap.add_argument("--long", action="store_true", help="also time the 32768-token prefill")
-    ap.add_argument("--only", choices=["decode", "prefill"], default=None,
-                    help="profiling: run only the bf16 decode or only the 8k prefill leg")
+    ap.add_argument("--only", choices=["decode", "prefill", "nvfp4"], default=None,
+                    help="profiling: run only the bf16 decode, the 8k prefill or the NVFP4 decode leg")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
