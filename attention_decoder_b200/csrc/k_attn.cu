@@ -14,13 +14,14 @@
 // (the cache does not depend on it). After the wait the block normalises and rotates its four
 // query heads and the head's new key, rounds them to bf16, writes the new key and value to the
 // cache (the block holding the current position does) and substitutes them for the stale row
-// in its shared copy. Scores: eight warps take 8 keys of a page each; lane l holds dims
-// 4l..4l+3 of the four queries, and one transposing butterfly turns the 32 per-lane partial dots
-// (8 keys x 4 heads) into 32 finished scores, one per lane. Across a block's pages the softmax
-// runs online (running max and sum per head, the P V sums rescaled at a new max). Each block
-// writes its unnormalised partial (max, sum, o) per head; the last block of a (stream, kv head)
-// - counted with an atomic - merges the splits with every warp loading a different subset of
-// them, applies the gate and writes the bf16 output.
+// in its shared copy. Each warp owns 8 keys of every page: lane l holds dims 4l..4l+3 of the
+// four queries, one transposing butterfly turns the 32 per-lane partial dots (8 keys x 4 heads)
+// into 32 finished scores, one per lane, and the warp keeps its own online softmax (running max
+// and sum per head, its P.V sums over dims 4l..4l+3 rescaled at a new max), so a page needs no
+// block barrier between scores, softmax and P.V; the eight warps' states merge once per split.
+// Each block writes its unnormalised partial (max, sum, o) per head; the last block of a
+// (stream, kv head) - counted with an atomic - merges the splits with every warp loading a
+// different subset of them, applies the gate and writes the bf16 output.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -54,12 +55,10 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
   extern __shared__ __align__(128) unsigned char dsm[];  // two buffers of one page: K then V
   __shared__ __align__(16) float qs[GQA][HD];
   __shared__ float kb[HD];
-  __shared__ float sc[GQA][DEC_KEYS];
-  __shared__ __align__(16) float4 pr[DEC_KEYS];          // the 4 heads' probabilities of each key
-  __shared__ __align__(16) float obuf[4][GQA][HD];       // PV of the four key quarters
+  __shared__ __align__(16) float obuf[DA_WARPS][GQA][HD];  // the warps' P.V sums (then the merge's halves)
+  __shared__ float wm[DA_WARPS][GQA], wl[DA_WARPS][GQA];     // the warps' running max and sum per head
   __shared__ float red[GQA + 1][4];
   __shared__ float lx[GQA];
-  __shared__ float alpha[GQA];                           // rescale of the running sums at a new max
   __shared__ __align__(16) bf16 wk[MAX_WIN][HD], wv[MAX_WIN][HD];  // earlier rows of a verify window
   __shared__ float kw[HD];
   __shared__ __align__(8) uint64_t kv_bar[2];
@@ -199,14 +198,17 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
     __syncthreads();
   }
 
-  // ---- the split's pages, two buffers deep, with an online softmax across them
+  // ---- the split's pages, two buffers deep. Each warp keeps its own online softmax over its
+  // eight keys of every page (running max and sum per head, its P.V sums rescaled at a new max):
+  // no block barrier between scores, softmax and P.V; the eight warps' states merge once at the
+  // end of the split.
   const size_t mloff = da_ml_offset(rows.n, splits);
   const size_t hbase = ((size_t)b * HQ + kvh * GQA) * splits;  // (stream, first head of the group) x splits
-  const int qt = tid >> 6, dp = 2 * (tid & 63);                 // P V: key quarter, dimension pair
-  float o[GQA][2] = {};
-  float Mh = -INFINITY, Lh = 0.f;  // warp h < 4: running max and sum of head h
+  float o[GQA][4] = {};                       // this lane's dims 4 lane .. 4 lane + 3 of each head
+  float Mw = -INFINITY, Lw = 0.f;             // head lane >> 3: this warp's running max and sum
+  float4 q4[GQA];                             // dims 4 lane .. of the four (scaled) queries
   bool ok = true;
-  int issued = min(np, 2), done = 0;  // pages copied / pages landed
+  int issued = min(np, 2), done = 0;          // pages copied / pages landed
   for (int i = 0; i < np; ++i) {
     const bf16* ks = reinterpret_cast<const bf16*>(dsm + (size_t)(i & 1) * DA_SMEM);
     const bf16* vs = ks + DEC_KEYS * HD;
@@ -232,65 +234,59 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
       }
     }
     __syncthreads();
-    if (ok) {
-      // scores: warp w takes keys 8w .. 8w+7; lane l holds dims 4l..4l+3 of the four queries
-      {
-        float4 q4[GQA];
+    if (ok && 8 * warp < pc) {
+      if (i == 0)
 #pragma unroll
         for (int hh = 0; hh < GQA; ++hh) q4[hh] = *reinterpret_cast<const float4*>(&qs[hh][4 * lane]);
-        float v[32];  // v[h * 8 + k]: this lane's partial dot of head h with key 8w + k
+      // scores: this warp's keys 8w .. 8w+7; one transposing butterfly turns the 32 per-lane
+      // partial dots into 32 finished scores, lane l holding (head l >> 3, key 8w + (l & 7))
+      float v[32];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint2 kk = *reinterpret_cast<const uint2*>(ks + (8 * warp + k) * HD + 4 * lane);
-          const float k0 = bflo(kk.x), k1 = bfhi(kk.x), k2 = bflo(kk.y), k3 = bfhi(kk.y);
+      for (int k = 0; k < 8; ++k) {
+        const uint2 kk = *reinterpret_cast<const uint2*>(ks + (8 * warp + k) * HD + 4 * lane);
+        const float k0 = bflo(kk.x), k1 = bfhi(kk.x), k2 = bflo(kk.y), k3 = bfhi(kk.y);
 #pragma unroll
-          for (int hh = 0; hh < GQA; ++hh) v[hh * 8 + k] = q4[hh].x * k0 + q4[hh].y * k1 + q4[hh].z * k2 + q4[hh].w * k3;
-        }
-        // butterfly: at offset o each lane keeps the half of its values selected by bit o of its
-        // lane id and adds the partner's; after five steps lane l holds the full sum of value l
-#pragma unroll
-        for (int o2 = 16, c = 32; o2 >= 1; o2 >>= 1, c >>= 1) {
-          const bool up = (lane & o2) != 0;
-#pragma unroll
-          for (int e = 0; e < c / 2; ++e) {
-            const float send = up ? v[e] : v[e + c / 2];
-            const float keep = up ? v[e + c / 2] : v[e];
-            v[e] = keep + __shfl_xor_sync(0xffffffffu, send, o2);
-          }
-        }
-        const int hh = lane >> 3, j = 8 * warp + (lane & 7);
-        sc[hh][j] = j < pc ? v[0] : -INFINITY;
+        for (int hh = 0; hh < GQA; ++hh) v[hh * 8 + k] = q4[hh].x * k0 + q4[hh].y * k1 + q4[hh].z * k2 + q4[hh].w * k3;
       }
-      __syncthreads();
-      // softmax: warp h < 4 takes head h; the running sums are rescaled at a new maximum
-      if (warp < GQA) {
-        const float s0 = sc[warp][lane], s1 = sc[warp][lane + 32];
-        const float mn = fmaxf(Mh, warp_max(fmaxf(s0, s1)));
-        const float p0 = __expf(s0 - mn), p1 = __expf(s1 - mn);
-        reinterpret_cast<float*>(&pr[lane])[warp] = p0;
-        reinterpret_cast<float*>(&pr[lane + 32])[warp] = p1;
-        const float a = __expf(Mh - mn);  // 0 on the first page
-        Lh = Lh * a + warp_sum(p0 + p1);
-        Mh = mn;
-        if (lane == 0) alpha[warp] = a;
+#pragma unroll
+      for (int o2 = 16, c = 32; o2 >= 1; o2 >>= 1, c >>= 1) {
+        const bool up = (lane & o2) != 0;
+#pragma unroll
+        for (int e = 0; e < c / 2; ++e) {
+          const float send = up ? v[e] : v[e + c / 2];
+          const float keep = up ? v[e + c / 2] : v[e];
+          v[e] = keep + __shfl_xor_sync(0xffffffffu, send, o2);
+        }
       }
-      __syncthreads();
-      // P V: thread = (key quarter, dimension pair); rows past the page's keys are never read
-      {
-        const int je = min(pc, 16 * qt + 16);
+      const float sj = 8 * warp + (lane & 7) < pc ? v[0] : -INFINITY;
+      // online softmax of head lane >> 3 over the warp's keys (groups of eight lanes)
+      float m8 = sj;
+      m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 1));
+      m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 2));
+      m8 = fmaxf(m8, __shfl_xor_sync(0xffffffffu, m8, 4));
+      const float mn = fmaxf(Mw, m8);  // finite: the warp's first key is valid
+      const float p = __expf(sj - mn);
+      const float a = __expf(Mw - mn);  // 0 on the warp's first page
+      float ps = p;
+      ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+      Lw = Lw * a + ps;
+      Mw = mn;
+      // P.V over the warp's valid keys: lane l accumulates dims 4l..4l+3 of the four heads
+#pragma unroll
+      for (int hh = 0; hh < GQA; ++hh) {
+        const float ah = __shfl_sync(0xffffffffu, a, 8 * hh);
+        o[hh][0] *= ah; o[hh][1] *= ah; o[hh][2] *= ah; o[hh][3] *= ah;
+      }
+      const int nk = min(8, pc - 8 * warp);
+      for (int k = 0; k < nk; ++k) {
+        const uint2 vw = *reinterpret_cast<const uint2*>(vs + (8 * warp + k) * HD + 4 * lane);
+        const float v0 = bflo(vw.x), v1 = bfhi(vw.x), v2 = bflo(vw.y), v3 = bfhi(vw.y);
 #pragma unroll
         for (int hh = 0; hh < GQA; ++hh) {
-          o[hh][0] *= alpha[hh];
-          o[hh][1] *= alpha[hh];
-        }
-        for (int j = 16 * qt; j < je; ++j) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(vs + j * HD + dp);
-          const float v0 = bflo(w), v1 = bfhi(w);
-          const float4 p = pr[j];
-          o[0][0] += p.x * v0; o[0][1] += p.x * v1;
-          o[1][0] += p.y * v0; o[1][1] += p.y * v1;
-          o[2][0] += p.z * v0; o[2][1] += p.z * v1;
-          o[3][0] += p.w * v0; o[3][1] += p.w * v1;
+          const float ph = __shfl_sync(0xffffffffu, p, 8 * hh + k);
+          o[hh][0] += ph * v0; o[hh][1] += ph * v1; o[hh][2] += ph * v2; o[hh][3] += ph * v3;
         }
       }
     }
@@ -303,22 +299,33 @@ __global__ void __launch_bounds__(DA_THREADS) k_attn_decode_fused(const float* _
   if (!ok && tid == 0)  // copies still in flight land before the block exits (bounded)
     for (int p = done; p < issued; ++p) mbar_wait(su32(&kv_bar[p & 1]), (p >> 1) & 1, A.err);
   if (ok) {
+    // merge the eight warps: weights exp(M_w - M) per head (a warp that saw no key has M_w = -inf)
 #pragma unroll
-    for (int hh = 0; hh < GQA; ++hh) *reinterpret_cast<float2*>(&obuf[qt][hh][dp]) = make_float2(o[hh][0], o[hh][1]);
-    if (warp < GQA && lane == 0) {
-      part[mloff + 2 * (hbase + (size_t)warp * splits + sp)] = Mh;
-      part[mloff + 2 * (hbase + (size_t)warp * splits + sp) + 1] = Lh;
+    for (int hh = 0; hh < GQA; ++hh)
+      *reinterpret_cast<float4*>(&obuf[warp][hh][4 * lane]) = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
+    if ((lane & 7) == 0) {
+      wm[warp][lane >> 3] = Mw;
+      wl[warp][lane >> 3] = Lw;
     }
     __syncthreads();
-    if (tid < GQA * HD / 4) {
-      const int hh = tid >> 5, d4 = 4 * lane;
-      float4 s4 = *reinterpret_cast<const float4*>(&obuf[0][hh][d4]);
+    // thread: head hh = tid >> 6, dims 2 (tid & 63) .. +1
+    const int hh = tid >> 6, d2 = 2 * (tid & 63);
+    float M = -INFINITY;
 #pragma unroll
-      for (int q = 1; q < 4; ++q) {
-        const float4 t = *reinterpret_cast<const float4*>(&obuf[q][hh][d4]);
-        s4.x += t.x; s4.y += t.y; s4.z += t.z; s4.w += t.w;
-      }
-      *reinterpret_cast<float4*>(part + (hbase + (size_t)hh * splits + sp) * HD + d4) = s4;
+    for (int w = 0; w < DA_WARPS; ++w) M = fmaxf(M, wm[w][hh]);
+    float s0 = 0.f, s1 = 0.f, l = 0.f;
+#pragma unroll
+    for (int w = 0; w < DA_WARPS; ++w) {
+      const float wt = wm[w][hh] == -INFINITY ? 0.f : __expf(wm[w][hh] - M);
+      const float2 t = *reinterpret_cast<const float2*>(&obuf[w][hh][d2]);
+      s0 += wt * t.x;
+      s1 += wt * t.y;
+      l += wt * wl[w][hh];
+    }
+    *reinterpret_cast<float2*>(part + (hbase + (size_t)hh * splits + sp) * HD + d2) = make_float2(s0, s1);
+    if ((tid & 63) == 0) {
+      part[mloff + 2 * (hbase + (size_t)hh * splits + sp)] = M;
+      part[mloff + 2 * (hbase + (size_t)hh * splits + sp) + 1] = l;
     }
   } else {  // a copy that never landed: this split contributes nothing
     if (tid < GQA) {
