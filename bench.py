@@ -261,7 +261,7 @@ def run_ours(args):
     if args.only == "nvfp4":
         del m
         torch.cuda.empty_cache()
-        r = nvfp4_leg(world, g, stream, prompt, K, Wm, hbm)
+        r = nvfp4_leg(world, g, stream, prompt, K, Wm, hbm, hi=2048 if args.small else 8192)
         if rank == 0:
             print(json.dumps({"profiling_case": "NVFP4 decode at 1/4/8/64 streams", **r, "clocks": clocks.stop()}),
                   flush=True)
@@ -443,9 +443,9 @@ def prefill_flops(g, n):
     return n * per_tok + attn + 2 * d * g.vocab
 
 
-def nvfp4_leg(world, g, stream, prompt, K, Wm, hbm):
-    """The NVFP4-FFN model: decode tok/s and HBM fraction at 1 / 4 / 8 streams (2048-token context,
-    prefilled) and at 64 streams on drawn state (contexts uniform in [256, 8192])."""
+def nvfp4_leg(world, g, stream, prompt, K, Wm, hbm, hi=8192):
+    """The NVFP4-FFN model: decode tok/s and HBM fraction at 1 / 4 / 8 streams (the prompt's
+    context, prefilled) and at 64 streams on drawn state (contexts uniform in [256, hi])."""
     import torch
     import numpy as np
     from attention_decoder_b200.model import Lfm3Model
@@ -453,9 +453,9 @@ def nvfp4_leg(world, g, stream, prompt, K, Wm, hbm):
     res = {}
     Wq = make_weights(g, 0, ffn="nvfp4")
     S = 64
-    ctx64 = context_lengths(1, "ctx64", S, 256, 8192)
+    ctx64 = context_lengths(1, "ctx64", S, 256, hi)
     steps_q = max(4, min(K, 32))
-    mpp_q = (8192 + Wm + steps_q + 16) // 64 + 2
+    mpp_q = (hi + Wm + steps_q + 16) // 64 + 2
     mq = Lfm3Model(Wq, max_streams=S, max_pages_per_stream=mpp_q, max_batch=S)
     del Wq
     stq = mq.new_state(page_table=page_permutation(1, "pages64", S * mpp_q).reshape(S, mpp_q))
@@ -498,7 +498,7 @@ def nvfp4_leg(world, g, stream, prompt, K, Wm, hbm):
     qfrac[64] = qbytes * (steps_q / (qms / 1e3)) / 1e9 / hbm
     res["decode_nvfp4"] = {f"b{b}_tok_s": v for b, v in qb.items()}
     res["decode_nvfp4"].update({f"b{b}_hbm_frac": round(v, 4) for b, v in qfrac.items()})
-    res["decode_nvfp4"]["b64_contexts"] = "uniform [256, 8192], mean %.0f" % float(np.mean(ctx64))
+    res["decode_nvfp4"]["b64_contexts"] = "uniform [256, %d], mean %.0f" % (hi, float(np.mean(ctx64)))
     del mq, stq
     torch.cuda.empty_cache()
     return res
