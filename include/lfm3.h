@@ -209,7 +209,11 @@ lfm3_status lfm3_prefill_padded(lfm3_ctx* ctx, const lfm3_state* st, int slot, c
  * lfm3_prefill the position comes from the state and there is no mask input - coreai-model-zoo
  * note "lfm3-1.7b-port", "window_size, with no mask input"). Streams share no state; the pages'
  * engine checks that concurrent == solo (TensorFold PR #1508, "Verification"), which holds here
- * bit for bit at up to 16 streams.
+ * bit for bit at up to 16 streams. Up to 16 rows stream every weight through the weight-streaming
+ * GEMVs; larger batches run the projections as tensor-core GEMMs (fp32 outputs split along K and
+ * summed in split order), so their results match those of smaller batches to fp32 rounding, not
+ * bit for bit. An NVFP4 FFN multiplies f16 copies of its bf16 activations: a value above 65504 in
+ * magnitude there would not be representable.
  *   h_slots     HOST int32 [n_streams] slot ids (checked; must equal d_slots)
  *   d_slots     device int32 [n_streams]
  *   d_tokens    device int32 [n_streams] (has_head == 1) or NULL; may alias d_argmax of the
