@@ -1,5 +1,6 @@
-// Prefill projections on the 5th-generation tensor cores: C[M][N] = alpha * A[M][K] . W[N][K]^T
-// with A the bf16 activations of a prompt chunk and W a bf16 weight, both K-major.
+// Projections on the 5th-generation tensor cores: C[M][N] = alpha * A[M][K] . W[N][K]^T with A
+// the bf16 activations of a prompt chunk (or of a decode batch over 16 rows) and W a bf16 weight,
+// both K-major. k_gemm_q4 (further down) takes NVFP4 weights and expands them on the chip.
 //
 // Persistent blocks (one per SM, 6 warps) walk output tiles:
 //   warp 0      TMA producer: A and W boxes of 64 K-columns per stage (128-byte swizzle) into a ring
@@ -13,8 +14,11 @@
 //               store per 32 rows x 128 bytes; then the accumulator is released.
 // k_gemm: one SM per 128 x BN tile (BN = 128 or 256). k_gemm2: a cluster of two SMs per 256 x 256
 // tile (tcgen05 cta_group::2), each SM staging its 128 rows of A and half of the weight rows.
-// Epilogues: fp32 out, bf16 out, and SwiGLU (the tile's 256 columns are 128 rows of w1 and the
-// same 128 rows of w3: u = silu(alpha a) * (alpha b), bf16).
+// Epilogues: fp32 out, bf16 out, SwiGLU (the tile's BN columns are BN/2 rows of w1 and the same
+// rows of w3: u = silu(alpha a) * (alpha b), bf16), and the head (fp32 logits, optional, and each
+// row's maximum and first index as a packed argmax key). A batch of at most 128 rows may split an
+// fp32 output along K: split s writes its partial sums at out + s * M * ld with plain stores, and
+// the consumer adds the splits in order.
 // Every mbarrier wait is bounded; a wait that gives up sets the device error word, and the MMA
 // thread drains (bounded) the stages still in flight so that TMEM is always released.
 #include <cudaTypedefs.h>
